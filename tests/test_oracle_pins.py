@@ -1,0 +1,334 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Each test names what fixes the expected value: a worked example printed on the pages
+(tests/golden), a closed form, an invariant of the method, a special case that reduces
+to a library routine (torch SDPA on rolled/folded tensors), or finite differences.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import s2_torch_formulation as ref
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _inputs(seed, B, N, Hq, Hkv, d, dtype="f64"):
+    q, k, v, do = synth.s2attn_inputs(seed, B, N, Hq, Hkv, d, 1.0, "f32")
+    return tuple(x.astype(np.float64) for x in (q, k, v, do))
+
+
+def _t(x):
+    return torch.from_numpy(np.ascontiguousarray(x))
+
+
+# ---------------------------------------------------------------- RoPE + PI (closed forms)
+
+def test_rope_matches_complex_closed_form():
+    """RoFormer's closed form: pair (x0, x1) -> (x0 + i x1) * exp(i (m/s) base^(-2i/d))."""
+    rng = np.random.default_rng(1)
+    d, n = 16, 40
+    x = rng.standard_normal((n, d))
+    pos = rng.integers(0, 100000, size=n)
+    for s in (1.0, 2.0, 8.0, 25.0):
+        y = oracle.rope(x, pos, s, 10000.0)
+        z = x[:, 0::2] + 1j * x[:, 1::2]
+        ang = (pos[:, None] / s) * 10000.0 ** (-np.arange(0, d, 2) / d)[None, :]
+        w = z * np.exp(1j * ang)
+        np.testing.assert_allclose(y[:, 0::2], w.real, rtol=0, atol=1e-9)
+        np.testing.assert_allclose(y[:, 1::2], w.imag, rtol=0, atol=1e-9)
+
+
+def test_rope_frequency_decreases_geometrically():
+    """The angle of pair i at m = 1, s = 1 is theta_i = base^(-2i/d): a geometric sequence."""
+    d = 8
+    x = np.zeros((d // 2, d))
+    for i in range(d // 2):
+        x[i, 2 * i] = 1.0
+    y = oracle.rope(x, np.ones(d // 2, dtype=np.int64), 1.0, 10000.0)
+    ang = np.array([math.atan2(y[i, 2 * i + 1], y[i, 2 * i]) for i in range(d // 2)])
+    np.testing.assert_allclose(ang, 10000.0 ** (-2.0 * np.arange(d // 2) / d), rtol=1e-12)
+    np.testing.assert_allclose(ang[1:] / ang[:-1], 10000.0 ** (-2.0 / d), rtol=1e-12)
+
+
+def test_rope_invariants():
+    """Orthogonal (norm-preserving), identity at m = 0, inverse undoes it, relative position."""
+    rng = np.random.default_rng(2)
+    d, n = 32, 16
+    x = rng.standard_normal((n, d))
+    kx = rng.standard_normal((n, d))
+    pos = rng.integers(0, 5000, size=n)
+    y = oracle.rope(x, pos, 4.0)
+    np.testing.assert_allclose(np.linalg.norm(y, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12)
+    np.testing.assert_array_equal(oracle.rope(x, np.zeros(n, np.int64), 4.0), x)
+    np.testing.assert_allclose(oracle.rope(y, pos, 4.0, inverse=True), x, atol=1e-12)
+    # <R(m) q, R(n) k> depends only on m - n.
+    m, nn, shift = 700, 300, 1234
+    a = oracle.rope(x[:1], [m], 4.0) @ oracle.rope(kx[:1], [nn], 4.0).T
+    b = oracle.rope(x[:1], [m + shift], 4.0) @ oracle.rope(kx[:1], [nn + shift], 4.0).T
+    np.testing.assert_allclose(a, b, rtol=1e-10)
+
+
+def test_position_interpolation_divides_position():
+    """PI: rotating at position m with scale s equals rotating at m/s with s = 1."""
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((5, 16))
+    for s in (2, 8, 25):
+        mp = rng.integers(0, 4096, size=5)
+        np.testing.assert_allclose(oracle.rope(x, mp * s, float(s)), oracle.rope(x, mp, 1.0),
+                                   atol=1e-12)
+
+
+# ---------------------------------------------------------------- attention special cases
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (4, 2)])
+def test_one_group_unshifted_heads_equal_dense_causal(Hq, Hkv):
+    """G = N: the unshifted heads are textbook dense causal attention (torch SDPA)."""
+    N, d = 32, 8
+    q, k, v, _ = _inputs(4, 1, N, Hq, Hkv, d)
+    o, _ = oracle.fwd(q, k, v, G=N, s=2.0)
+    dense = ref.dense_causal(_t(q), _t(k), _t(v), 2.0).numpy()
+    np.testing.assert_allclose(o[:, :, :Hq // 2], dense[:, :, :Hq // 2], atol=1e-12)
+
+
+@pytest.mark.parametrize("B,N,Hq,Hkv,d,G,causal", [
+    (1, 64, 4, 4, 8, 16, True), (2, 48, 4, 2, 8, 8, True), (1, 64, 8, 2, 16, 32, True),
+    (1, 32, 4, 4, 8, 8, False), (1, 256, 4, 4, 64, 64, True)])
+def test_oracle_equals_library_formulation(B, N, Hq, Hkv, d, G, causal):
+    """Oracle == roll / fold / SDPA / roll-back built from torch routines, O and LSE."""
+    q, k, v, _ = _inputs(5, B, N, Hq, Hkv, d)
+    o, lse = oracle.fwd(q, k, v, G=G, s=2.0, causal=causal)
+    o_r, lse_r = ref.s2attn(_t(q), _t(k), _t(v), G, 2.0, causal=causal, with_lse=True)
+    np.testing.assert_allclose(o, o_r.numpy(), atol=1e-12)
+    np.testing.assert_allclose(lse, lse_r.numpy(), atol=1e-12)
+
+
+def test_unshifted_heads_are_block_diagonal():
+    """Unshifted heads: each group alone is dense causal attention over its own rows."""
+    N, G, d = 64, 16, 8
+    q, k, v, _ = _inputs(6, 1, N, 2, 2, d)
+    o, _ = oracle.fwd(q, k, v, G=G, s=1.0)
+    qr = ref.rope_complex(_t(q), 1.0)
+    kr = ref.rope_complex(_t(k), 1.0)
+    for g in range(N // G):
+        sl = slice(g * G, (g + 1) * G)
+        og = torch.nn.functional.scaled_dot_product_attention(
+            qr[0, sl, 0][None], kr[0, sl, 0][None], _t(v)[0, sl, 0][None], is_causal=True)
+        np.testing.assert_allclose(o[0, sl, 0], og[0].numpy(), atol=1e-12)
+
+
+def _read_shift_examples():
+    rows = []
+    with open(os.path.join(GOLDEN, "shift_groups.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                rows.append(tuple(int(x) for x in line.split()))
+    return rows
+
+
+@pytest.mark.parametrize("G,first,last", _read_shift_examples())
+def test_first_shifted_group_worked_example(G, first, last):
+    """The shifted heads' first group is tokens G/2 .. 3G/2-1 (pages' worked examples).
+
+    Perturbing any token outside that range leaves the shifted head's outputs at those
+    tokens unchanged; the unit-row map of group 0 is exactly that range."""
+    N = 2 * G
+    rows = oracle.unit_rows(N, G, Hq=2, kvh=1, Hkv=2, g=0)
+    assert rows[0] == first and rows[-1] == last
+    np.testing.assert_array_equal(rows, np.arange(first, last + 1))
+    if G > 64:
+        return  # the index map is the pin at this size; the perturbation check runs small
+    q, k, v, _ = _inputs(7, 1, N, 2, 2, 4)
+    o, _ = oracle.fwd(q, k, v, G=G, s=1.0)
+    outside = np.r_[0:first, last + 1:N]
+    k2, v2 = k.copy(), v.copy()
+    k2[:, outside] += 3.0
+    v2[:, outside] -= 2.0
+    o2, _ = oracle.fwd(q, k2, v2, G=G, s=1.0)
+    np.testing.assert_array_equal(o2[0, first:last + 1, 1], o[0, first:last + 1, 1])
+    assert np.abs(o2[0, :G, 0] - o[0, :G, 0]).max() > 1e-3  # unshifted head does see them
+
+
+def test_wrap_group_mixes_end_and_start():
+    """np.roll wraps: the last shifted group holds tokens N-G/2..N-1 then 0..G/2-1, so the
+    shifted head's output at token 0 depends on the sequence's last tokens (and the
+    unshifted head's does not)."""
+    N, G, d = 32, 8, 4
+    q, k, v, _ = _inputs(8, 1, N, 2, 2, d)
+    o, _ = oracle.fwd(q, k, v, G=G, s=1.0)
+    rows = oracle.unit_rows(N, G, 2, 1, 2, N // G - 1)
+    np.testing.assert_array_equal(rows, np.r_[N - G // 2:N, 0:G // 2])
+    v2 = v.copy()
+    v2[0, N - 1] += 5.0
+    o2, _ = oracle.fwd(q, k, v2, G=G, s=1.0)
+    assert abs(o2[0, 0, 1] - o[0, 0, 1]).max() > 1e-6
+    np.testing.assert_array_equal(o2[0, 0, 0], o[0, 0, 0])
+
+
+def test_roll_forward_then_back_is_identity():
+    x = np.arange(40).reshape(1, 40, 1, 1)
+    for G in (2, 8, 40):
+        assert np.array_equal(np.roll(np.roll(x, -G // 2, axis=1), G // 2, axis=1), x)
+        rows = np.concatenate([oracle.unit_rows(40, G, 2, 1, 2, g) for g in range(40 // G)])
+        assert np.array_equal(np.sort(rows), np.arange(40))  # the roll is a bijection
+
+
+def test_first_row_of_each_group_is_its_value_row():
+    """Causal: local row 0 of every group sees one key, so O equals that token's v exactly."""
+    N, G, d = 64, 16, 8
+    q, k, v, _ = _inputs(9, 1, N, 4, 4, d)
+    o, _ = oracle.fwd(q, k, v, G=G, s=2.0)
+    for h in range(4):
+        for g in range(N // G):
+            t = oracle.unit_rows(N, G, 4, h, 4, g)[0]
+            np.testing.assert_array_equal(o[0, t, h], v[0, t, h])
+
+
+def test_output_in_convex_hull_of_visible_values():
+    N, G, d = 64, 16, 8
+    q, k, v, _ = _inputs(10, 1, N, 2, 2, d)
+    o, _ = oracle.fwd(q, k, v, G=G, s=2.0)
+    for h in range(2):
+        for g in range(N // G):
+            rows = oracle.unit_rows(N, G, 2, h, 2, g)
+            for i, t in enumerate(rows):
+                vis = v[0, rows[:i + 1], h]
+                assert np.all(o[0, t, h] <= vis.max(0) + 1e-12)
+                assert np.all(o[0, t, h] >= vis.min(0) - 1e-12)
+
+
+def test_relative_position_invariance_across_groups():
+    """With RoPE, a group whose rows repeat another group's rows at a constant offset gives
+    the same outputs: input periodic with period G -> outputs periodic off the wrap group."""
+    N, G, d = 64, 16, 8
+    q, k, v, _ = _inputs(11, 1, N, 2, 2, d)
+    for x in (q, k, v):
+        for g in range(1, N // G):
+            x[:, g * G:(g + 1) * G] = x[:, :G]
+    o, _ = oracle.fwd(q, k, v, G=G, s=2.0)
+    # unshifted head: every group equals group 0
+    for g in range(1, N // G):
+        np.testing.assert_allclose(o[0, g * G:(g + 1) * G, 0], o[0, :G, 0], atol=1e-12)
+    # shifted head: non-wrap groups start at G/2 + gG
+    a = o[0, G // 2:G // 2 + G, 1]
+    for g in range(1, N // G - 1):
+        b = o[0, G // 2 + g * G:G // 2 + (g + 1) * G, 1]
+        np.testing.assert_allclose(b, a, atol=1e-12)
+
+
+def test_gqa_equals_mha_with_repeated_kv_heads():
+    N, G, d, Hq, Hkv = 32, 8, 8, 8, 2
+    q, k, v, do = _inputs(12, 1, N, Hq, Hkv, d)
+    R = Hq // Hkv
+    kr, vr = np.repeat(k, R, axis=2), np.repeat(v, R, axis=2)
+    o, lse = oracle.fwd(q, k, v, G=G, s=2.0)
+    o2, lse2 = oracle.fwd(q, kr, vr, G=G, s=2.0)
+    np.testing.assert_allclose(o, o2, atol=1e-13)
+    np.testing.assert_allclose(lse, lse2, atol=1e-13)
+    dq, dk, dv = oracle.bwd(q, k, v, do, G=G, s=2.0)
+    dq2, dk2, dv2 = oracle.bwd(q, kr, vr, do, G=G, s=2.0)
+    np.testing.assert_allclose(dq, dq2, atol=1e-12)
+    np.testing.assert_allclose(dk, dk2.reshape(1, N, Hkv, R, d).sum(3), atol=1e-12)
+    np.testing.assert_allclose(dv, dv2.reshape(1, N, Hkv, R, d).sum(3), atol=1e-12)
+
+
+# ---------------------------------------------------------------- backward
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_gradients_match_finite_differences(causal):
+    """Central differences of L = sum(O * dO) match the oracle's analytic dq, dk, dv."""
+    B, N, Hq, Hkv, d, G, s = 1, 16, 4, 2, 8, 8, 2.0
+    q, k, v, do = _inputs(13, B, N, Hq, Hkv, d)
+    dq, dk, dv = oracle.bwd(q, k, v, do, G=G, s=s, causal=causal)
+    h = 1e-6
+
+    def loss(q_, k_, v_):
+        o, _ = oracle.fwd(q_, k_, v_, G=G, s=s, causal=causal)
+        return float((o * do).sum())
+
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.empty_like(x)
+        flat = x.reshape(-1)
+        for idx in range(flat.size):
+            old = flat[idx]
+            flat[idx] = old + h
+            lp = loss(q, k, v)
+            flat[idx] = old - h
+            lm = loss(q, k, v)
+            flat[idx] = old
+            num.reshape(-1)[idx] = (lp - lm) / (2 * h)
+        err = np.abs(num - g).max() / np.abs(g).max()
+        assert err < 1e-7, (name, err)
+
+
+@pytest.mark.parametrize("B,N,Hq,Hkv,d,G", [(1, 64, 4, 4, 16, 16), (1, 64, 8, 2, 8, 32),
+                                            (1, 256, 4, 4, 64, 64)])
+def test_gradients_match_autograd_of_library_formulation(B, N, Hq, Hkv, d, G):
+    q, k, v, do = _inputs(14, B, N, Hq, Hkv, d)
+    tq, tk, tv = (_t(x).clone().requires_grad_(True) for x in (q, k, v))
+    o = ref.s2attn(tq, tk, tv, G, 2.0)
+    (o * _t(do)).sum().backward()
+    dq, dk, dv = oracle.bwd(q, k, v, do, G=G, s=2.0)
+    np.testing.assert_allclose(dq, tq.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy(), atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy(), atol=1e-11)
+
+
+def test_unit_functions_agree_with_full_functions():
+    N, G, d, Hq, Hkv = 64, 16, 8, 8, 2
+    q, k, v, do = _inputs(15, 2, N, Hq, Hkv, d)
+    o, lse = oracle.fwd(q, k, v, G=G, s=2.0)
+    dq, dk, dv = oracle.bwd(q, k, v, do, G=G, s=2.0)
+    R = Hq // Hkv
+    for b, kvh, g in ((0, 0, 0), (1, 1, N // G - 1), (0, 1, 1)):
+        rows = oracle.unit_rows(N, G, Hq, kvh, Hkv, g)
+        o_u, l_u = oracle.fwd_unit(q, k, v, G, 2.0, b, kvh, g)
+        dq_u, dk_u, dv_u = oracle.bwd_unit(q, k, v, do, G, 2.0, b, kvh, g)
+        for r in range(R):
+            h = kvh * R + r
+            np.testing.assert_array_equal(o_u[r], o[b, rows, h])
+            np.testing.assert_array_equal(l_u[r], lse[b, h, rows])
+            np.testing.assert_array_equal(dq_u[r], dq[b, rows, h])
+        np.testing.assert_array_equal(dk_u, dk[b, rows, kvh])
+        np.testing.assert_array_equal(dv_u, dv[b, rows, kvh])
+
+
+def test_oracle_rejects_shapes_the_method_cannot_take():
+    assert oracle.check(1, 64, 4, 4, 8, 16)
+    assert not oracle.check(1, 60, 4, 4, 8, 16)   # N % G
+    assert not oracle.check(1, 64, 3, 3, 8, 16)   # odd heads: no half split
+    assert not oracle.check(1, 64, 4, 4, 8, 7)    # odd G: no G/2 shift
+    assert not oracle.check(1, 64, 4, 3, 8, 16)   # Hq % Hkv
+    assert not oracle.check(1, 16, 4, 4, 8, 32)   # G > N
+
+
+# ---------------------------------------------------------------- FLOP model (worked example)
+
+def _golden_flops():
+    vals = {}
+    with open(os.path.join(GOLDEN, "flop_counts.txt")) as f:
+        for line in f:
+            if "=" in line and not line.startswith("#"):
+                key, val = line.strip().split("=")
+                vals[key] = float(val)
+    return vals
+
+
+def test_flop_model_matches_pages_worked_example():
+    from longlora_shifted_sparse_b200 import flops
+    g = _golden_flops()
+    L, G, D = int(g["L"]), int(g["G"]), int(g["D"])
+    assert flops.toy_dense_ops(L, D) == int(g["dense_ops"])
+    assert flops.toy_s2_ops(L, G, D) == int(g["s2_ops"])
+    assert round((1 - flops.toy_s2_ops(L, G, D) / flops.toy_dense_ops(L, D)) * 100, 1) == \
+        g["reduction_percent"]
+    # The counted attention FLOPs scale the same way: dense / S2 = N / G, for any head split.
+    for causal in (True, False):
+        dense = flops.attention_fwd_flops(1, L, 8, D // 8, L, causal)
+        s2 = flops.attention_fwd_flops(1, L, 8, D // 8, G, causal)
+        assert dense / s2 == L / G
