@@ -1,0 +1,395 @@
+"""S2-Attn fwd+bwd throughput on B200 (TFLOP/s, counted FLOPs) through the library's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-e2e] [--no-cpu-baseline]
+
+A step = one forward (RoPE+PI stage, per-group attention) and one backward (RoPE+PI
+stage, dO.O row sums, dK/dV pass, dQ pass) over one batch of the workload, inputs resident
+in HBM. Counted FLOPs: forward 4*B*H*N*G*d/2 (causal), backward 2.5x forward.
+With N > 1 (torchrun), every rank runs its own batch (independent problems: no data-path
+collective); `value` is the sum over ranks of counted FLOPs / the slowest rank's time.
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same workload.
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+from workloads import HEADLINE, WORKLOADS  # noqa: E402
+from longlora_shifted_sparse_b200 import flops  # noqa: E402
+
+METRIC = "S2-Attn fwd+bwd TFLOP/s (bf16, 1 B200) and % of dense bf16 tensor-core peak"
+UNIT = "TFLOP/s"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=p["hbm_gbs"], bf16=p["bf16_tflops"],
+                    bf16_sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                    sm_max_mhz=p.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, sm_max_mhz=1965.0,
+                source="fallback")
+
+
+def _counted_step_flops(w, ranks=1):
+    f = flops.attention_fwd_flops(w.B, w.N, w.Hq, w.d, w.G, w.causal)
+    if w.backward:
+        f += flops.attention_bwd_flops(w.B, w.N, w.Hq, w.d, w.G, w.causal)
+    return f * ranks
+
+
+def _kernel_work(name, w, es):
+    """(bound, algorithmic work per launch, unit) of one library kernel."""
+    fwd = flops.attention_fwd_flops(w.B, w.N, w.Hq, w.d, w.G, w.causal)
+    if name.startswith("fwd_"):
+        work = fwd                      # S = QK^T and O = PV
+    elif name.startswith("bwd_dkdv"):
+        work = 2.0 * fwd                # S, dP = dO V^T, dV += P^T dO, dK += dS^T Q
+    elif name.startswith("bwd_dq"):
+        work = 1.5 * fwd                # S, dP, dQ += dS K
+    elif name == "rope_pi":
+        return "hbm", 2.0 * w.B * w.N * (w.Hq + w.Hkv) * w.d * es + w.N * w.d * 4, "GB/s"
+    elif name == "bwd_rowsum":
+        return "hbm", 2.0 * w.B * w.N * w.Hq * w.d * es + 4.0 * w.B * w.Hq * w.N, "GB/s"
+    else:
+        return None, 0.0, None
+    return ("tensor" if name.endswith("_tc") else "alu"), work, "TFLOP/s"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.REASONS, parts[3:]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _traffic(kernel: str):
+    """ncu DRAM bytes per launch of `kernel`, if recorded for the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    import hashlib
+    src = os.path.join(ROOT, "longlora_shifted_sparse_b200", "csrc", rec["source"])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest()[:16] != rec["sha256_16"]:
+            return None  # the kernel changed since the counters were taken
+    return rec["bytes_per_launch"]
+
+
+def _oracle_sample(w, inputs):
+    """One (batch 0, head 0, group 0) unit of the workload through the oracle: forward at
+    all G rows, then backward (dq at all rows, dk/dv at all rows); rows over host threads.
+    Returns (seconds, counted FLOPs of the unit, threads)."""
+    import oracle
+    q, k, v, do = inputs
+    rows = np.arange(w.G)
+    t0 = time.perf_counter()
+    oracle.fwd_rows(q, k, v, w.G, w.pi_scale, 0, 0, 0, rows, w.rope_base, w.causal)
+    if w.backward:
+        oracle.bwd_rows(q, k, v, do, w.G, w.pi_scale, 0, 0, 0, rows, rows, w.rope_base,
+                        w.causal)
+    dt = time.perf_counter() - t0
+    R = w.Hq // w.Hkv
+    unit_fwd = flops.attention_fwd_flops(1, w.G, 1, w.d, w.G, w.causal)
+    # head 0's forward, then the backward of all R query heads of kv head 0
+    counted = unit_fwd * (1 + 2.5 * R) if w.backward else unit_fwd
+    return dt, counted, oracle.max_threads()
+
+
+SAMPLE_DESC = ("fp64 oracle on one (batch 0, head 0, group 0) unit of {name}: forward at all "
+               "{G} rows + backward (dq, dk, dv) at all rows, rows spread over host threads; "
+               "FLOPs counted as for the GPU (fwd 2*G*G*d, bwd 2.5x)")
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    inputs = synth.s2attn_inputs(w.seed, w.B, w.N, w.Hq, w.Hkv, w.d, w.in_scale, w.dtype)
+    steps = []
+    for i in range(args.warmup + args.steps):
+        dt, counted, cores = _oracle_sample(w, inputs)
+        if i >= args.warmup:
+            steps.append(dt)
+    mean = sum(steps) / len(steps)
+    value = counted / mean / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": mean * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.Hq, "H_kv": w.Hkv,
+                   "d": w.d, "G": w.G, "pi_scale": w.pi_scale, "parallelism": "host threads"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": SAMPLE_DESC.format(name=w.name, G=w.G)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from longlora_shifted_sparse_b200 import s2attn as s2
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = WORKLOADS[args.workload]
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    es = 2 if w.dtype == "bf16" else 4
+
+    # seeded host inputs, one independent batch per rank
+    q, k, v, do = synth.s2attn_inputs(w.seed + 1000 * rank, w.B, w.N, w.Hq, w.Hkv, w.d,
+                                      w.in_scale, w.dtype)
+
+    def host_pinned(x):
+        t = torch.from_numpy(x.view(np.int16) if w.dtype == "bf16" else x)
+        t = t.view(tdt) if w.dtype == "bf16" else t
+        return t.pin_memory()
+
+    hq, hk, hv, hdo = (host_pinned(x) for x in (q, k, v, do))
+    dq_ = [hx.to(dev) for hx in (hq, hk, hv, hdo)]
+    tq, tk, tv, tdo = dq_
+    o = torch.empty_like(tq)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device=dev)
+    gq, gk, gv = torch.empty_like(tq), torch.empty_like(tk), torch.empty_like(tv)
+    code = s2.S2_BF16 if w.dtype == "bf16" else s2.S2_FP32
+    ws = s2.workspace(w.B, w.N, w.Hq, w.Hkv, w.d, code, dev)
+
+    def step():
+        s2.forward(tq, tk, tv, w.G, w.pi_scale, w.rope_base, w.causal, ws=ws, out=o, lse=lse)
+        if w.backward:
+            s2.backward(tq, tk, tv, o, lse, tdo, w.G, w.pi_scale, w.rope_base, w.causal, ws=ws,
+                        grads=(gq, gk, gv))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    if s2.device_status(ws) != s2.S2_OK:
+        raise RuntimeError("device status reports an expired wait during warm-up")
+
+    stream = torch.cuda.current_stream(dev)
+    props = torch.cuda.get_device_properties(dev)
+    gpu_uuid = str(getattr(props, "uuid", "")) or str(local)
+    if gpu_uuid and not gpu_uuid.startswith("GPU-") and len(gpu_uuid) > 8:
+        gpu_uuid = "GPU-" + gpu_uuid
+    sampler = ClockSampler(gpu_uuid)
+    sampler.start()
+    time.sleep(0.3)
+    s2.check(s2.s2attn_profile_enable(1))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    barrier()
+    prof = s2.profile_summary()
+    s2.check(s2.s2attn_profile_enable(0))
+    clocks = sampler.stop()
+    elapsed_ms = e0.elapsed_time(e1)
+    if s2.device_status(ws) != s2.S2_OK:
+        raise RuntimeError("device status reports an expired wait in the timed region")
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    step_flops = _counted_step_flops(w)
+    value = step_flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # end to end: pinned host inputs -> device, step, results -> pinned host, every step
+    e2e = None
+    if not args.no_e2e:
+        outs = [o, lse] + ([gq, gk, gv] if w.backward else [])
+        houts = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True) for x in outs]
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv) + ((hdo,) if w.backward
+                                                                        else ()))
+        d2h = sum(x.numel() * x.element_size() for x in outs)
+
+        def e2e_step():
+            tq.copy_(hq, non_blocking=True)
+            tk.copy_(hk, non_blocking=True)
+            tv.copy_(hv, non_blocking=True)
+            if w.backward:
+                tdo.copy_(hdo, non_blocking=True)
+            step()
+            for hx, x in zip(houts, outs):
+                hx.copy_(x, non_blocking=True)
+
+        e2e_step()
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": step_flops * world / (e2e_ms / args.steps * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    peaks = _peaks()
+    roofline = None
+    if prof:
+        name, (n, ms) = max(prof.items(), key=lambda kv: kv[1][1])
+        bound, work, unit = _kernel_work(name, w, es)
+        avg_s = ms / n * 1e-3
+        if bound == "tensor":
+            peak = peaks["bf16_sustained"]
+            achieved = work / avg_s / 1e12
+        elif bound == "alu":
+            # fp32 FMA pipes: 148 SMs x 128 lanes x 2 FLOP x max SM clock
+            peak = 148 * 128 * 2 * peaks["sm_max_mhz"] * 1e6 / 1e12
+            achieved = work / avg_s / 1e12
+        else:
+            peak = peaks["hbm_gbs"]
+            achieved = work / avg_s / 1e9
+        roofline = {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak,
+                    "unit": unit, "frac": achieved / peak, "traffic": _traffic(name),
+                    "peak_source": peaks["source"] + (" sustained bf16" if bound == "tensor"
+                                                      else ""),
+                    "launches": n, "avg_ms": ms / n,
+                    "kernels": {k_: {"launches": n_, "total_ms": t_} for k_, (n_, t_) in
+                                prof.items()}}
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, counted, cores = _oracle_sample(w, (q, k, v, do))
+        cpu_baseline = {"value": counted / dt / 1e12, "unit": UNIT, "cores": cores,
+                        "kind": "oracle", "sample": SAMPLE_DESC.format(name=w.name, G=w.G)}
+
+    paths = {s2.s2attn_kernel_path(w.B, w.N, w.Hq, w.Hkv, w.d, w.G, int(w.causal), code)}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.Hq, "H_kv": w.Hkv,
+                   "d": w.d, "G": w.G, "pi_scale": w.pi_scale, "causal": w.causal,
+                   "fwd_bwd": w.backward, "parallelism": "independent batch per GPU",
+                   "l2": "inputs exceed L2 (q, k, v, dO are %.0f MB each)" %
+                         (tq.numel() * es / 1e6),
+                   "kernel_path": "tcgen05" if paths == {1} else "cuda-core"},
+        "tflops_frac_of_peak": {"measured_burst": value / world / peaks["bf16"],
+                                "measured_sustained": value / world / peaks["bf16_sustained"],
+                                "spec_2250": value / world / 2250.0},
+        "clocks": clocks,
+        "gpu_launches": int(sum(n_ for n_, _ in prof.values())) if prof else 0,
+        "e2e": e2e,
+        "roofline": roofline,
+        "cpu_baseline": cpu_baseline,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=HEADLINE)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

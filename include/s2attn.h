@@ -1,0 +1,123 @@
+/*
+ * s2attn.h - C ABI of libs2attn.so: shifted sparse attention (S2-Attn) forward and backward
+ * on one NVIDIA B200 (sm_100a), with RoPE and linear position interpolation fused in.
+ *
+ * The operation (sources are web pages on LongLoRA, cited by title and section):
+ *  - RoPE with position interpolation ("LoRA for Long-Context Adaptation", sections
+ *    "Why vanilla LoRA under-delivers on long context" and "Position interpolation: the
+ *    prerequisite"): channel pair (2i, 2i+1) of q and of k at token m (0-based, original
+ *    order) is rotated by phi = (m / pi_scale) * rope_base^(-2i/d). v is not rotated.
+ *  - Half-group shift ("LongLoRA and Shifted Sparse Attention (S^2-Attn)", definition;
+ *    "LongLoRA: Efficient 100k Context LLM Fine-Tuning Guide", "How Shifted Short Attention
+ *    Works" and "Implementation ... Step 1"): query heads h >= H_q/2 (and kv heads
+ *    >= H_kv/2) see the sequence rolled by -G/2 with wrap-around: rolled row r holds
+ *    original token (r + G/2) mod N.
+ *  - Group fold: rolled rows are cut into N/G groups of G rows; inside each group,
+ *    softmax(q k^T / sqrt(d)) v with a causal mask on group-local positions (no mask
+ *    when causal == 0). GQA: query head h uses kv head h / (H_q / H_kv).
+ *  - Roll back: each shifted head's output row r is stored at token (r + G/2) mod N.
+ *  - Backward: gradients of the above with respect to the pre-RoPE q, k and to v; dk and
+ *    dv of a kv head are summed over the query heads that share it.
+ *
+ * Layouts (all dense, row-major, element = dtype unless noted):
+ *    q, o, dout, dq : [B][N][H_q][d]      k, v, dk, dv : [B][N][H_kv][d]
+ *    lse            : [B][H_q][N] float32, natural log of the softmax normaliser of the
+ *                     scaled scores, in original token order.
+ * Every pointer argument is a DEVICE pointer (cudaMalloc'd or equivalent), 16-byte aligned.
+ * The caller owns every buffer, including the workspace; the library allocates no device
+ * memory in these calls. All work is enqueued on cuda_stream (a cudaStream_t; NULL = the
+ * legacy default stream) and runs asynchronously; no call synchronises.
+ * Outputs are overwritten, never accumulated into.
+ *
+ * Errors: argument errors are returned before anything is enqueued and leave the outputs
+ * untouched. A failed CUDA launch or query returns S2_ERR_CUDA. Device-side bounded waits
+ * that expire set a status word in the workspace; s2attn_device_status() reads it.
+ * No C++ exception crosses this interface. All functions are thread-safe.
+ */
+#ifndef S2ATTN_H
+#define S2ATTN_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define S2_API __attribute__((visibility("default")))
+#else
+#define S2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  S2_OK = 0,
+  S2_ERR_NULL = 1,           /* a required pointer is NULL */
+  S2_ERR_SHAPE = 2,          /* B, N, H_q, H_kv, G <= 0; G > N; N % G != 0; G odd;
+                                H_q or H_kv odd; H_q % H_kv != 0 */
+  S2_ERR_DTYPE = 3,          /* dtype is not an s2_dtype value */
+  S2_ERR_HEADDIM = 4,        /* d is not a multiple of 32 in [32, 256] */
+  S2_ERR_ALIGN = 5,          /* a pointer is not 16-byte aligned */
+  S2_ERR_WORKSPACE = 6,      /* workspace NULL or ws_bytes < s2attn_workspace_bytes(...) */
+  S2_ERR_CUDA = 7,           /* a CUDA runtime/driver call failed */
+  S2_ERR_DEVICE_TIMEOUT = 8, /* a bounded device-side wait expired (see s2attn_device_status) */
+  S2_ERR_ARG = 9             /* pi_scale or rope_base not finite and > 0, or causal not 0/1 */
+} s2_status;
+
+typedef enum {
+  S2_BF16 = 0, /* bfloat16 storage, fp32 accumulation, tensor cores where the shape allows */
+  S2_FP32 = 1  /* float32 storage and arithmetic (CUDA cores) */
+} s2_dtype;
+
+/* Bytes of device workspace that s2attn_fwd / s2attn_bwd need for this shape (it does not
+ * depend on G or causal). Returns 0 for arguments that s2attn_fwd would reject with
+ * S2_ERR_SHAPE, S2_ERR_HEADDIM or S2_ERR_DTYPE. The workspace holds the rotated q and k
+ * (head-major, original token order), the RoPE cos/sin table, the backward's row sums
+ * D = rowsum(dO * O) and the device status word. */
+S2_API size_t s2attn_workspace_bytes(int B, int N, int H_q, int H_kv, int d, int dtype);
+
+/* Forward: o and lse from q, k, v. See the header comment for the operation and layouts.
+ * G: group size (even, divides N). causal: 1 = causal mask inside each group, 0 = none.
+ * pi_scale: position interpolation factor s = L_new / L_orig (1 = plain RoPE).
+ * rope_base: RoPE base (10000 for LLaMA2). */
+S2_API s2_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int N, int H_q, int H_kv, int d, int G, int causal,
+                     float pi_scale, float rope_base, int dtype,
+                     void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* Backward: dq, dk, dv from q, k, v, the forward's o and lse, and dout = dL/do.
+ * Same shape arguments as the forward; o and lse must come from s2attn_fwd with the same
+ * arguments. The workspace may be the forward's or another one of the same size. */
+S2_API s2_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                     const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                     int B, int N, int H_q, int H_kv, int d, int G, int causal,
+                     float pi_scale, float rope_base, int dtype,
+                     void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* Which kernel family s2attn_fwd/s2attn_bwd launch for these arguments:
+ * 1 = tcgen05 tensor-core kernels (bf16, d == 128, G % 256 == 0),
+ * 0 = CUDA-core kernels (any other valid shape, and every fp32 call), -1 = invalid. */
+S2_API int s2attn_kernel_path(int B, int N, int H_q, int H_kv, int d, int G, int causal, int dtype);
+
+/* Waits for cuda_stream, then reads and clears the device status word of the workspace
+ * used by the last call on it: S2_OK, or S2_ERR_DEVICE_TIMEOUT if a bounded wait in a
+ * kernel expired (that kernel's outputs are then undefined). S2_ERR_CUDA on a CUDA error. */
+S2_API s2_status s2attn_device_status(void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* Static, NUL-terminated description of a status code. */
+S2_API const char* s2attn_status_string(int status);
+
+/* Kernel timing for measurement. When enabled, every kernel the library launches is
+ * bracketed by two CUDA events recorded on its launching stream (a bounded pool; records
+ * beyond it are dropped and counted). s2attn_profile_query() waits for those events and
+ * returns per-kernel launch counts and summed durations. */
+S2_API s2_status s2attn_profile_enable(int on);  /* on = 1 starts afresh, 0 stops recording */
+S2_API int s2attn_profile_num_kernels(void);     /* number of kernel ids */
+S2_API s2_status s2attn_profile_query(int kernel_id, const char** name, int* launches,
+                               double* total_ms);
+S2_API int s2attn_profile_dropped(void);         /* records dropped since the last enable */
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* S2ATTN_H */

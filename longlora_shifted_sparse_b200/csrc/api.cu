@@ -1,0 +1,334 @@
+// extern "C" entry points of libs2attn.so: argument checks, workspace carving, kernel
+// selection and launch, device status, and optional per-kernel event timing.
+#include <math.h>
+#include <stdint.h>
+
+#include <mutex>
+#include <vector>
+
+#include "../../include/s2attn.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace s2 {
+namespace {
+
+// ----------------------------------------------------------------------------- profiling
+
+enum KernelId {
+  kRopePi = 0,
+  kFwdTc,
+  kFwdSimt,
+  kBwdRowsum,
+  kBwdDkdvTc,
+  kBwdDqTc,
+  kBwdDqSimt,
+  kBwdDkdvSimt,
+  kNumKernels
+};
+
+const char* const kKernelNames[kNumKernels] = {
+    "rope_pi", "fwd_tc", "fwd_simt", "bwd_rowsum", "bwd_dkdv_tc", "bwd_dq_tc", "bwd_dq_simt",
+    "bwd_dkdv_simt"};
+
+struct Record {
+  int id;
+  cudaEvent_t start, stop;
+};
+
+constexpr size_t kMaxRecords = 8192;
+
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  int dropped = 0;
+  std::vector<Record> pending;
+  std::vector<cudaEvent_t> pool;
+  int launches[kNumKernels] = {};
+  double total_ms[kNumKernels] = {};
+
+  cudaEvent_t get_event() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+  }
+
+  // Folds finished records into the totals; returns the first CUDA error seen.
+  cudaError_t drain() {
+    cudaError_t first = cudaSuccess;
+    for (auto& r : pending) {
+      float ms = 0.f;
+      cudaError_t e = cudaEventSynchronize(r.stop);
+      if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, r.start, r.stop);
+      if (e == cudaSuccess) {
+        launches[r.id] += 1;
+        total_ms[r.id] += ms;
+      } else if (first == cudaSuccess) {
+        first = e;
+      }
+      pool.push_back(r.start);
+      pool.push_back(r.stop);
+    }
+    pending.clear();
+    return first;
+  }
+};
+
+Profiler& profiler() {
+  static Profiler* p = new Profiler();  // never destroyed: events may outlive static teardown
+  return *p;
+}
+
+// Launches `fn` on `st`; when profiling is on, brackets it with events on the same stream.
+template <typename F>
+cudaError_t timed_launch(int id, cudaStream_t st, F fn) {
+  Profiler& pr = profiler();
+  cudaEvent_t a = nullptr, b = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(pr.mu);
+    if (pr.on) {
+      if (pr.pending.size() < kMaxRecords) {
+        a = pr.get_event();
+        b = pr.get_event();
+        if (!a || !b) {
+          if (a) pr.pool.push_back(a);
+          if (b) pr.pool.push_back(b);
+          a = b = nullptr;
+          pr.dropped++;
+        }
+      } else {
+        pr.dropped++;
+      }
+    }
+  }
+  if (a && cudaEventRecord(a, st) != cudaSuccess) return cudaGetLastError();
+  cudaError_t e = fn();
+  if (e != cudaSuccess) return e;
+  if (a) {
+    if (cudaEventRecord(b, st) != cudaSuccess) return cudaGetLastError();
+    std::lock_guard<std::mutex> lk(pr.mu);
+    pr.pending.push_back(Record{id, a, b});
+  }
+  return cudaSuccess;
+}
+
+// ----------------------------------------------------------------------------- arguments
+
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct WsLayout {
+  size_t qr, kr, cs, dsum, status, total;
+};
+
+bool shape_ok(int B, int N, int Hq, int Hkv, int G) {
+  if (B <= 0 || N <= 0 || Hq <= 0 || Hkv <= 0 || G <= 0) return false;
+  if (G > N || N % G != 0 || G % 2 != 0) return false;
+  if (Hq % 2 != 0 || Hkv % 2 != 0 || Hq % Hkv != 0) return false;
+  // every index the kernels form per tensor must fit in 64 bits and rows in 32 bits
+  if ((long long)B * N * Hq > (1LL << 31) - 1) return false;
+  return true;
+}
+
+bool headdim_ok(int d) { return d >= 32 && d <= 256 && d % 32 == 0; }
+
+bool dtype_ok(int dt) { return dt == S2_BF16 || dt == S2_FP32; }
+
+WsLayout ws_layout(int B, int N, int Hq, int Hkv, int d, int dt) {
+  // The status word sits at offset 0 so that s2attn_device_status() finds it without the
+  // shape; the tensors follow, each on a 256-byte boundary.
+  const size_t es = dt == S2_BF16 ? 2 : 4;
+  WsLayout w;
+  w.status = 0;
+  size_t off = kAlign;
+  w.qr = off;
+  off = align_up(off + (size_t)B * Hq * N * d * es);
+  w.kr = off;
+  off = align_up(off + (size_t)B * Hkv * N * d * es);
+  w.cs = off;
+  off = align_up(off + (size_t)N * (d / 2) * sizeof(float2));
+  w.dsum = off;
+  off = align_up(off + (size_t)B * Hq * N * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// The tcgen05 kernels are not built yet: every call takes the CUDA-core kernels.
+bool tc_path(int, int, int) { return false; }
+
+s2_status common_checks(int B, int N, int Hq, int Hkv, int d, int G, int causal, float s,
+                        float base, int dt, void* ws, size_t ws_bytes) {
+  if (!dtype_ok(dt)) return S2_ERR_DTYPE;
+  if (!shape_ok(B, N, Hq, Hkv, G)) return S2_ERR_SHAPE;
+  if (!headdim_ok(d)) return S2_ERR_HEADDIM;
+  if (!(isfinite(s) && s > 0.f) || !(isfinite(base) && base > 0.f) ||
+      (causal != 0 && causal != 1))
+    return S2_ERR_ARG;
+  if (!ws) return S2_ERR_WORKSPACE;
+  if (!aligned16(ws)) return S2_ERR_ALIGN;
+  if (ws_bytes < ws_layout(B, N, Hq, Hkv, d, dt).total) return S2_ERR_WORKSPACE;
+  return S2_OK;
+}
+
+Params make_params(int B, int N, int Hq, int Hkv, int d, int G, int causal, float s, float base,
+                   int dt, void* ws) {
+  Params p{};
+  p.B = B; p.N = N; p.Hq = Hq; p.Hkv = Hkv; p.d = d; p.G = G; p.causal = causal;
+  p.pi_scale = s;
+  p.rope_base = base;
+  p.scale = (float)(1.0 / sqrt((double)d));
+  p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)d));
+  WsLayout w = ws_layout(B, N, Hq, Hkv, d, dt);
+  char* c = static_cast<char*>(ws);
+  p.qr = c + w.qr;
+  p.kr = c + w.kr;
+  p.cs = reinterpret_cast<float2*>(c + w.cs);
+  p.Dsum = reinterpret_cast<float*>(c + w.dsum);
+  p.status = reinterpret_cast<unsigned*>(c + w.status);
+  return p;
+}
+
+s2_status to_status(cudaError_t e) { return e == cudaSuccess ? S2_OK : S2_ERR_CUDA; }
+
+}  // namespace
+}  // namespace s2
+
+using namespace s2;
+
+extern "C" {
+
+size_t s2attn_workspace_bytes(int B, int N, int H_q, int H_kv, int d, int dtype) {
+  if (!dtype_ok(dtype) || !headdim_ok(d)) return 0;
+  if (B <= 0 || N <= 0 || H_q <= 0 || H_kv <= 0 || H_q % 2 || H_kv % 2 || H_q % H_kv) return 0;
+  return ws_layout(B, N, H_q, H_kv, d, dtype).total;
+}
+
+int s2attn_kernel_path(int B, int N, int H_q, int H_kv, int d, int G, int causal, int dtype) {
+  if (!dtype_ok(dtype) || !shape_ok(B, N, H_q, H_kv, G) || !headdim_ok(d) ||
+      (causal != 0 && causal != 1))
+    return -1;
+  return tc_path(d, G, dtype) ? 1 : 0;
+}
+
+s2_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int N, int H_q, int H_kv, int d, int G, int causal, float pi_scale,
+                     float rope_base, int dtype, void* workspace, size_t ws_bytes,
+                     void* cuda_stream) {
+  if (!q || !k || !v || !o || !lse) return S2_ERR_NULL;
+  s2_status st = common_checks(B, N, H_q, H_kv, d, G, causal, pi_scale, rope_base, dtype,
+                               workspace, ws_bytes);
+  if (st != S2_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return S2_ERR_ALIGN;
+  Params p = make_params(B, N, H_q, H_kv, d, G, causal, pi_scale, rope_base, dtype, workspace);
+  p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
+  const bool bf16 = dtype == S2_BF16;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e = timed_launch(kRopePi, s, [&] { return launch_rope_pi(p, bf16, s); });
+  if (e != cudaSuccess) return to_status(e);
+  e = timed_launch(kFwdSimt, s, [&] { return launch_simt_fwd(p, bf16, s); });
+  return to_status(e);
+}
+
+s2_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, int B, int N, int H_q,
+                     int H_kv, int d, int G, int causal, float pi_scale, float rope_base,
+                     int dtype, void* workspace, size_t ws_bytes, void* cuda_stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return S2_ERR_NULL;
+  s2_status st = common_checks(B, N, H_q, H_kv, d, G, causal, pi_scale, rope_base, dtype,
+                               workspace, ws_bytes);
+  if (st != S2_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return S2_ERR_ALIGN;
+  Params p = make_params(B, N, H_q, H_kv, d, G, causal, pi_scale, rope_base, dtype, workspace);
+  p.q = q; p.k = k; p.v = v; p.o = const_cast<void*>(o); p.lse = const_cast<float*>(lse);
+  p.dout = dout; p.dq = dq; p.dk = dk; p.dv = dv;
+  const bool bf16 = dtype == S2_BF16;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e = timed_launch(kRopePi, s, [&] { return launch_rope_pi(p, bf16, s); });
+  if (e == cudaSuccess)
+    e = timed_launch(kBwdRowsum, s, [&] { return launch_bwd_rowsum(p, bf16, s); });
+  if (e != cudaSuccess) return to_status(e);
+  e = timed_launch(kBwdDkdvSimt, s, [&] { return launch_simt_dkdv(p, bf16, s); });
+  if (e == cudaSuccess) e = timed_launch(kBwdDqSimt, s, [&] { return launch_simt_dq(p, bf16, s); });
+  return to_status(e);
+}
+
+s2_status s2attn_device_status(void* workspace, size_t ws_bytes, void* cuda_stream) {
+  if (!workspace) return S2_ERR_NULL;
+  if (ws_bytes < kAlign) return S2_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  unsigned word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return S2_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return S2_ERR_CUDA;
+  if (word != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(word), s) != cudaSuccess) return S2_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return S2_ERR_CUDA;
+    return S2_ERR_DEVICE_TIMEOUT;
+  }
+  return S2_OK;
+}
+
+const char* s2attn_status_string(int status) {
+  switch (status) {
+    case S2_OK: return "ok";
+    case S2_ERR_NULL: return "a required pointer is NULL";
+    case S2_ERR_SHAPE: return "invalid shape (B,N,H_q,H_kv,G > 0; G <= N; N % G == 0; G, H_q, "
+                              "H_kv even; H_q % H_kv == 0)";
+    case S2_ERR_DTYPE: return "unknown dtype";
+    case S2_ERR_HEADDIM: return "head dim d must be a multiple of 32 in [32, 256]";
+    case S2_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+    case S2_ERR_WORKSPACE: return "workspace missing or smaller than s2attn_workspace_bytes()";
+    case S2_ERR_CUDA: return "a CUDA call failed";
+    case S2_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
+    case S2_ERR_ARG: return "invalid argument (pi_scale, rope_base finite and > 0; causal 0/1)";
+    default: return "unknown status";
+  }
+}
+
+s2_status s2attn_profile_enable(int on) {
+  Profiler& pr = profiler();
+  std::lock_guard<std::mutex> lk(pr.mu);
+  cudaError_t e = pr.drain();
+  if (on) {
+    for (int i = 0; i < kNumKernels; i++) {
+      pr.launches[i] = 0;
+      pr.total_ms[i] = 0.0;
+    }
+    pr.dropped = 0;
+  }
+  pr.on = on != 0;
+  return to_status(e);
+}
+
+int s2attn_profile_num_kernels(void) { return kNumKernels; }
+
+s2_status s2attn_profile_query(int kernel_id, const char** name, int* launches,
+                               double* total_ms) {
+  if (kernel_id < 0 || kernel_id >= kNumKernels) return S2_ERR_ARG;
+  Profiler& pr = profiler();
+  std::lock_guard<std::mutex> lk(pr.mu);
+  cudaError_t e = pr.drain();
+  if (name) *name = kKernelNames[kernel_id];
+  if (launches) *launches = pr.launches[kernel_id];
+  if (total_ms) *total_ms = pr.total_ms[kernel_id];
+  return to_status(e);
+}
+
+int s2attn_profile_dropped(void) {
+  Profiler& pr = profiler();
+  std::lock_guard<std::mutex> lk(pr.mu);
+  return pr.dropped;
+}
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+// Shared definitions of the S2-Attn CUDA library: argument block, index maps, conversions.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace s2 {
+
+// Everything a kernel of one call needs. Built once per call on the host, passed by value.
+struct Params {
+  int B, N, Hq, Hkv, d, G, causal;
+  float pi_scale, rope_base;
+  float scale;       // 1 / sqrt(d)
+  float scale_log2;  // log2(e) / sqrt(d): scores go straight to the exp2 domain
+  // caller tensors
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  const void* dout;
+  void* dq;
+  void* dk;
+  void* dv;
+  // workspace views
+  void* qr;         // rotated q, [B][Hq][N][d], original token order
+  void* kr;         // rotated k, [B][Hkv][N][d], original token order
+  float2* cs;       // (cos, sin) of (m / s) * theta_i, [N][d/2]
+  float* Dsum;      // rowsum(dO * O), [B][Hq][N]
+  unsigned* status; // device status word (bit 0: a bounded wait expired)
+};
+
+enum StatusBits : unsigned { kStatusTimeout = 1u };
+
+// Half-group shift: query heads h >= Hq/2 (equivalently kv heads >= Hkv/2) are shifted.
+__host__ __device__ inline bool head_shifted(int h, int H) { return h >= H / 2; }
+
+// Rolled row r -> original token. Rolling by -G/2 puts token (r + G/2) mod N at row r.
+__host__ __device__ inline int src_row(int r, bool shifted, int G, int N) {
+  if (!shifted) return r;
+  int m = r + G / 2;
+  return m >= N ? m - N : m;
+}
+
+template <typename T> __device__ inline float to_f32(T x);
+template <> __device__ inline float to_f32<float>(float x) { return x; }
+template <> __device__ inline float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+template <typename T> __device__ inline T from_f32(float x);
+template <> __device__ inline float from_f32<float>(float x) { return x; }
+template <> __device__ inline __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__device__ inline float warp_sum(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+  return x;
+}
+
+}  // namespace s2

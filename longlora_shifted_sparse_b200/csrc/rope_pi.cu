@@ -1,0 +1,82 @@
+// RoPE + position interpolation stage (HBM-bound).
+//
+// For every token m (original order) the pair (2i, 2i+1) of each q and k head vector is
+// rotated by phi = (m / s) * base^(-2i/d) ("LoRA for Long-Context Adaptation", sections on
+// RoPE and on position interpolation; interleaved pairs as in RoFormer). The rotated
+// tensors are written head-major, [B][H][N][d], still in ORIGINAL token order: the -G/2
+// roll of the shifted heads is never materialised, the attention kernels fold it into
+// their row coordinates.
+//
+// One CTA per token. The d/2 angles of a token are shared by all heads of q and k, so the
+// CTA computes them once in fp64 (sincos of an exact fp64 angle, rounded to fp32) and
+// keeps them in shared memory; the (cos, sin) table is also written to the workspace for
+// the backward's inverse rotation. The data moves in 16-byte vectors.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace s2 {
+
+template <typename T>
+__device__ inline void rotate_vec(const T* __restrict__ src, T* __restrict__ dst,
+                                  const float2* __restrict__ cs_row) {
+  constexpr int V = 16 / sizeof(T);
+  uint4 raw = *reinterpret_cast<const uint4*>(src);
+  const T* x = reinterpret_cast<const T*>(&raw);
+  uint4 out_raw;
+  T* y = reinterpret_cast<T*>(&out_raw);
+#pragma unroll
+  for (int t = 0; t < V / 2; t++) {
+    float2 c = cs_row[t];
+    float x0 = to_f32<T>(x[2 * t]), x1 = to_f32<T>(x[2 * t + 1]);
+    y[2 * t] = from_f32<T>(fmaf(x0, c.x, -x1 * c.y));
+    y[2 * t + 1] = from_f32<T>(fmaf(x0, c.y, x1 * c.x));
+  }
+  *reinterpret_cast<uint4*>(dst) = out_raw;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) rope_pi_kernel(Params p) {
+  extern __shared__ float2 s_cs[];
+  constexpr int V = 16 / sizeof(T);
+  const int half = p.d / 2;
+  const int tok = blockIdx.x;
+  const int b = tok / p.N, n = tok - b * p.N;
+  if (tok == 0 && threadIdx.x == 0) *p.status = 0u;  // each call starts with a clean status
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    double theta = pow((double)p.rope_base, -2.0 * (double)i / (double)p.d);
+    double phi = ((double)n / (double)p.pi_scale) * theta;
+    double sn, c;
+    sincos(phi, &sn, &c);
+    float2 v = make_float2((float)c, (float)sn);
+    s_cs[i] = v;
+    if (b == 0) p.cs[(size_t)n * half + i] = v;
+  }
+  __syncthreads();
+
+  const T* q = static_cast<const T*>(p.q) + (size_t)tok * p.Hq * p.d;
+  const T* k = static_cast<const T*>(p.k) + (size_t)tok * p.Hkv * p.d;
+  T* qr = static_cast<T*>(p.qr);
+  T* kr = static_cast<T*>(p.kr);
+  const int vq = p.Hq * p.d / V, vk = p.Hkv * p.d / V;
+  for (int e = threadIdx.x; e < vq + vk; e += blockDim.x) {
+    const bool is_q = e < vq;
+    const int ee = is_q ? e : e - vq;
+    const int h = ee * V / p.d, c0 = ee * V - h * p.d;
+    const int H = is_q ? p.Hq : p.Hkv;
+    const T* src = (is_q ? q : k) + (size_t)ee * V;
+    T* dst = (is_q ? qr : kr) + (((size_t)b * H + h) * p.N + n) * p.d + c0;
+    rotate_vec<T>(src, dst, s_cs + c0 / 2);
+  }
+}
+
+cudaError_t launch_rope_pi(const Params& p, bool bf16, cudaStream_t st) {
+  dim3 grid(p.B * p.N), block(256);
+  size_t smem = (size_t)(p.d / 2) * sizeof(float2);
+  if (bf16)
+    rope_pi_kernel<__nv_bfloat16><<<grid, block, smem, st>>>(p);
+  else
+    rope_pi_kernel<float><<<grid, block, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace s2

@@ -1,0 +1,259 @@
+// CUDA-core S2-Attn kernels: the fp32 path and every shape the tensor-core path does not
+// take (any even G, d a multiple of 32 up to 256), plus the backward's row-sum preprocess.
+//
+// One warp per row, lanes split the head dimension (lane owns elements lane + 32u). Rows
+// are addressed in rolled coordinates: rolled row r of a shifted head is token
+// (r + G/2) mod N, so the -G/2 roll and the +G/2 roll back are index arithmetic only
+// ("LongLoRA: Efficient 100k Context LLM Fine-Tuning Guide", Implementation, Step 1,
+// steps 3 and 5). Each group is attended on its own with the causal mask on group-local
+// positions; the forward uses the online (running max / running sum) form of the
+// max-subtracted softmax.
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace s2 {
+
+// Dot product of two lane-distributed rows, reduced over the warp (every lane gets it).
+template <int DPL>
+__device__ inline float row_dot(const float (&a)[DPL], const float (&b)[DPL]) {
+  float acc = 0.f;
+#pragma unroll
+  for (int u = 0; u < DPL; u++) acc = fmaf(a[u], b[u], acc);
+  return warp_sum(acc);
+}
+
+template <typename T, int DPL>
+__device__ inline void load_row(const T* __restrict__ row, float (&x)[DPL], int lane) {
+#pragma unroll
+  for (int u = 0; u < DPL; u++) x[u] = to_f32<T>(row[lane + 32 * u]);
+}
+
+// Inverse rotation R(phi)^T of a lane-distributed row at token m (pair partner = lane ^ 1).
+template <int DPL>
+__device__ inline void inverse_rope(float (&x)[DPL], const float2* __restrict__ cs_row, int lane) {
+#pragma unroll
+  for (int u = 0; u < DPL; u++) {
+    const int c = lane + 32 * u;
+    const float partner = __shfl_xor_sync(0xffffffffu, x[u], 1);
+    const float2 t = cs_row[c >> 1];
+    // even c: x0 cos + x1 sin ; odd c: -x0 sin + x1 cos
+    x[u] = (c & 1) ? fmaf(-partner, t.y, x[u] * t.x) : fmaf(x[u], t.x, partner * t.y);
+  }
+}
+
+template <typename T, int DPL>
+__global__ void __launch_bounds__(256) simt_fwd_kernel(Params p) {
+  const int lane = threadIdx.x & 31;
+  const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (warp >= (long)p.B * p.Hq * p.N) return;
+  const int r = (int)(warp % p.N);
+  const int h = (int)((warp / p.N) % p.Hq);
+  const int b = (int)(warp / ((long)p.N * p.Hq));
+  const int kvh = h / (p.Hq / p.Hkv);
+  const bool sh = head_shifted(h, p.Hq);
+  const int g = r / p.G, i = r - g * p.G;
+  const int m = src_row(r, sh, p.G, p.N);
+  const int d = p.d;
+
+  const T* qr = static_cast<const T*>(p.qr);
+  const T* kr = static_cast<const T*>(p.kr);
+  const T* v = static_cast<const T*>(p.v);
+  float qv[DPL], acc[DPL], kv[DPL], vv[DPL];
+  load_row<T, DPL>(qr + (((size_t)b * p.Hq + h) * p.N + m) * d, qv, lane);
+#pragma unroll
+  for (int u = 0; u < DPL; u++) acc[u] = 0.f;
+  float mx = -INFINITY, l = 0.f;
+  const int jend = p.causal ? i : p.G - 1;
+  for (int j = 0; j <= jend; j++) {
+    const int mj = src_row(g * p.G + j, sh, p.G, p.N);
+    load_row<T, DPL>(kr + (((size_t)b * p.Hkv + kvh) * p.N + mj) * d, kv, lane);
+    load_row<T, DPL>(v + (((size_t)b * p.N + mj) * p.Hkv + kvh) * d, vv, lane);
+    const float s = row_dot<DPL>(qv, kv) * p.scale;
+    const float mnew = fmaxf(mx, s);
+    const float alpha = expf(mx - mnew);  // 0 on the first key (mx = -inf)
+    const float pj = expf(s - mnew);
+    l = fmaf(l, alpha, pj);
+#pragma unroll
+    for (int u = 0; u < DPL; u++) acc[u] = fmaf(acc[u], alpha, pj * vv[u]);
+    mx = mnew;
+  }
+  const float inv_l = 1.f / l;
+  T* o = static_cast<T*>(p.o) + (((size_t)b * p.N + m) * p.Hq + h) * d;
+#pragma unroll
+  for (int u = 0; u < DPL; u++) o[lane + 32 * u] = from_f32<T>(acc[u] * inv_l);
+  if (lane == 0) p.lse[((size_t)b * p.Hq + h) * p.N + m] = mx + logf(l);
+}
+
+// D[b][h][m] = sum_c dO[b][m][h][c] * O[b][m][h][c] (fp32), one warp per row.
+template <typename T, int DPL>
+__global__ void __launch_bounds__(256) bwd_rowsum_kernel(Params p) {
+  const int lane = threadIdx.x & 31;
+  const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (warp >= (long)p.B * p.N * p.Hq) return;
+  const int h = (int)(warp % p.Hq);
+  const long bm = warp / p.Hq;
+  const int m = (int)(bm % p.N), b = (int)(bm / p.N);
+  const size_t off = (size_t)warp * p.d;
+  float a[DPL], c[DPL];
+  load_row<T, DPL>(static_cast<const T*>(p.dout) + off, a, lane);
+  load_row<T, DPL>(static_cast<const T*>(p.o) + off, c, lane);
+  const float D = row_dot<DPL>(a, c);
+  if (lane == 0) p.Dsum[((size_t)b * p.Hq + h) * p.N + m] = D;
+}
+
+template <typename T, int DPL>
+__global__ void __launch_bounds__(256) simt_dq_kernel(Params p) {
+  const int lane = threadIdx.x & 31;
+  const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (warp >= (long)p.B * p.Hq * p.N) return;
+  const int r = (int)(warp % p.N);
+  const int h = (int)((warp / p.N) % p.Hq);
+  const int b = (int)(warp / ((long)p.N * p.Hq));
+  const int kvh = h / (p.Hq / p.Hkv);
+  const bool sh = head_shifted(h, p.Hq);
+  const int g = r / p.G, i = r - g * p.G;
+  const int m = src_row(r, sh, p.G, p.N);
+  const int d = p.d;
+
+  const T* qr = static_cast<const T*>(p.qr);
+  const T* kr = static_cast<const T*>(p.kr);
+  const T* v = static_cast<const T*>(p.v);
+  float qv[DPL], dov[DPL], dq[DPL], kv[DPL], vv[DPL];
+  load_row<T, DPL>(qr + (((size_t)b * p.Hq + h) * p.N + m) * d, qv, lane);
+  load_row<T, DPL>(static_cast<const T*>(p.dout) + (((size_t)b * p.N + m) * p.Hq + h) * d, dov,
+                   lane);
+  const float lse = p.lse[((size_t)b * p.Hq + h) * p.N + m];
+  const float Dm = p.Dsum[((size_t)b * p.Hq + h) * p.N + m];
+#pragma unroll
+  for (int u = 0; u < DPL; u++) dq[u] = 0.f;
+  const int jend = p.causal ? i : p.G - 1;
+  for (int j = 0; j <= jend; j++) {
+    const int mj = src_row(g * p.G + j, sh, p.G, p.N);
+    load_row<T, DPL>(kr + (((size_t)b * p.Hkv + kvh) * p.N + mj) * d, kv, lane);
+    load_row<T, DPL>(v + (((size_t)b * p.N + mj) * p.Hkv + kvh) * d, vv, lane);
+    const float s = row_dot<DPL>(qv, kv) * p.scale;
+    const float pr = expf(s - lse);
+    const float dp = row_dot<DPL>(dov, vv);
+    const float ds = pr * (dp - Dm);
+#pragma unroll
+    for (int u = 0; u < DPL; u++) dq[u] = fmaf(ds, kv[u], dq[u]);
+  }
+#pragma unroll
+  for (int u = 0; u < DPL; u++) dq[u] *= p.scale;
+  inverse_rope<DPL>(dq, p.cs + (size_t)m * (d / 2), lane);
+  T* out = static_cast<T*>(p.dq) + (((size_t)b * p.N + m) * p.Hq + h) * d;
+#pragma unroll
+  for (int u = 0; u < DPL; u++) out[lane + 32 * u] = from_f32<T>(dq[u]);
+}
+
+template <typename T, int DPL>
+__global__ void __launch_bounds__(256) simt_dkdv_kernel(Params p) {
+  const int lane = threadIdx.x & 31;
+  const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (warp >= (long)p.B * p.Hkv * p.N) return;
+  const int r = (int)(warp % p.N);
+  const int kvh = (int)((warp / p.N) % p.Hkv);
+  const int b = (int)(warp / ((long)p.N * p.Hkv));
+  const int R = p.Hq / p.Hkv;
+  const bool sh = head_shifted(kvh, p.Hkv);
+  const int g = r / p.G, j = r - g * p.G;
+  const int m = src_row(r, sh, p.G, p.N);
+  const int d = p.d;
+
+  const T* qr = static_cast<const T*>(p.qr);
+  const T* kr = static_cast<const T*>(p.kr);
+  const T* dout = static_cast<const T*>(p.dout);
+  float kv[DPL], vv[DPL], dk[DPL], dv[DPL], qv[DPL], dov[DPL];
+  load_row<T, DPL>(kr + (((size_t)b * p.Hkv + kvh) * p.N + m) * d, kv, lane);
+  load_row<T, DPL>(static_cast<const T*>(p.v) + (((size_t)b * p.N + m) * p.Hkv + kvh) * d, vv,
+                   lane);
+#pragma unroll
+  for (int u = 0; u < DPL; u++) dk[u] = dv[u] = 0.f;
+  const int ibeg = p.causal ? j : 0;
+  for (int rr = 0; rr < R; rr++) {
+    const int h = kvh * R + rr;
+    for (int i = ibeg; i < p.G; i++) {
+      const int mi = src_row(g * p.G + i, sh, p.G, p.N);
+      load_row<T, DPL>(qr + (((size_t)b * p.Hq + h) * p.N + mi) * d, qv, lane);
+      load_row<T, DPL>(dout + (((size_t)b * p.N + mi) * p.Hq + h) * d, dov, lane);
+      const float lse = p.lse[((size_t)b * p.Hq + h) * p.N + mi];
+      const float Dm = p.Dsum[((size_t)b * p.Hq + h) * p.N + mi];
+      const float s = row_dot<DPL>(qv, kv) * p.scale;
+      const float pr = expf(s - lse);
+      const float dp = row_dot<DPL>(dov, vv);
+      const float ds = pr * (dp - Dm);
+#pragma unroll
+      for (int u = 0; u < DPL; u++) {
+        dv[u] = fmaf(pr, dov[u], dv[u]);
+        dk[u] = fmaf(ds, qv[u], dk[u]);
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < DPL; u++) dk[u] *= p.scale;
+  inverse_rope<DPL>(dk, p.cs + (size_t)m * (d / 2), lane);
+  const size_t off = (((size_t)b * p.N + m) * p.Hkv + kvh) * d;
+  T* dko = static_cast<T*>(p.dk) + off;
+  T* dvo = static_cast<T*>(p.dv) + off;
+#pragma unroll
+  for (int u = 0; u < DPL; u++) {
+    dko[lane + 32 * u] = from_f32<T>(dk[u]);
+    dvo[lane + 32 * u] = from_f32<T>(dv[u]);
+  }
+}
+
+namespace {
+constexpr int kWarpsPerBlock = 8;
+
+inline dim3 warp_grid(long rows) {
+  return dim3((unsigned)((rows + kWarpsPerBlock - 1) / kWarpsPerBlock));
+}
+}  // namespace
+
+#define S2_DISPATCH_DPL(KERNEL, T, DPL_RT, GRID, ST, P)                          \
+  switch (DPL_RT) {                                                              \
+    case 1: KERNEL<T, 1><<<GRID, kWarpsPerBlock * 32, 0, ST>>>(P); break;        \
+    case 2: KERNEL<T, 2><<<GRID, kWarpsPerBlock * 32, 0, ST>>>(P); break;        \
+    case 3: KERNEL<T, 3><<<GRID, kWarpsPerBlock * 32, 0, ST>>>(P); break;        \
+    case 4: KERNEL<T, 4><<<GRID, kWarpsPerBlock * 32, 0, ST>>>(P); break;        \
+    case 5: KERNEL<T, 5><<<GRID, kWarpsPerBlock * 32, 0, ST>>>(P); break;        \
+    case 6: KERNEL<T, 6><<<GRID, kWarpsPerBlock * 32, 0, ST>>>(P); break;        \
+    case 7: KERNEL<T, 7><<<GRID, kWarpsPerBlock * 32, 0, ST>>>(P); break;        \
+    case 8: KERNEL<T, 8><<<GRID, kWarpsPerBlock * 32, 0, ST>>>(P); break;        \
+    default: return cudaErrorInvalidValue;                                       \
+  }
+
+#define S2_DISPATCH_TYPE(KERNEL, BF16, GRID, ST, P)                              \
+  if (BF16) {                                                                    \
+    S2_DISPATCH_DPL(KERNEL, __nv_bfloat16, (P).d / 32, GRID, ST, P)              \
+  } else {                                                                       \
+    S2_DISPATCH_DPL(KERNEL, float, (P).d / 32, GRID, ST, P)                      \
+  }
+
+cudaError_t launch_simt_fwd(const Params& p, bool bf16, cudaStream_t st) {
+  dim3 grid = warp_grid((long)p.B * p.Hq * p.N);
+  S2_DISPATCH_TYPE(simt_fwd_kernel, bf16, grid, st, p)
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_rowsum(const Params& p, bool bf16, cudaStream_t st) {
+  dim3 grid = warp_grid((long)p.B * p.Hq * p.N);
+  S2_DISPATCH_TYPE(bwd_rowsum_kernel, bf16, grid, st, p)
+  return cudaGetLastError();
+}
+
+cudaError_t launch_simt_dq(const Params& p, bool bf16, cudaStream_t st) {
+  dim3 grid = warp_grid((long)p.B * p.Hq * p.N);
+  S2_DISPATCH_TYPE(simt_dq_kernel, bf16, grid, st, p)
+  return cudaGetLastError();
+}
+
+cudaError_t launch_simt_dkdv(const Params& p, bool bf16, cudaStream_t st) {
+  dim3 grid = warp_grid((long)p.B * p.Hkv * p.N);
+  S2_DISPATCH_TYPE(simt_dkdv_kernel, bf16, grid, st, p)
+  return cudaGetLastError();
+}
+
+}  // namespace s2

@@ -1,0 +1,202 @@
+"""Thin ctypes binding of libs2attn.so (argument marshalling only; every step runs in the
+library's CUDA kernels).
+
+Two layers:
+* the C ABI under its own names (``s2attn_fwd``, ``s2attn_bwd``, ...), taking raw device
+  pointers and sizes exactly like ``include/s2attn.h``;
+* torch conveniences (``forward``, ``backward``, ``S2AttnFunction``) that allocate outputs
+  and the workspace with torch and pass their pointers and the current CUDA stream.
+
+Importing this module raises ImportError when the library has not been built: there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libs2attn.so")
+
+S2_OK, S2_ERR_NULL, S2_ERR_SHAPE, S2_ERR_DTYPE, S2_ERR_HEADDIM, S2_ERR_ALIGN, \
+    S2_ERR_WORKSPACE, S2_ERR_CUDA, S2_ERR_DEVICE_TIMEOUT, S2_ERR_ARG = range(10)
+S2_BF16, S2_FP32 = 0, 1
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        "libs2attn.so is not built (expected at %s); build it with "
+        "`python -m longlora_shifted_sparse_b200.build`" % LIB_PATH)
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_SHAPE = [_i] * 7 + [_f, _f, _i]
+
+_lib.s2attn_workspace_bytes.argtypes = [_i] * 6
+_lib.s2attn_workspace_bytes.restype = _sz
+_lib.s2attn_fwd.argtypes = [_vp] * 5 + _SHAPE + [_vp, _sz, _vp]
+_lib.s2attn_fwd.restype = _i
+_lib.s2attn_bwd.argtypes = [_vp] * 9 + _SHAPE + [_vp, _sz, _vp]
+_lib.s2attn_bwd.restype = _i
+_lib.s2attn_kernel_path.argtypes = [_i] * 8
+_lib.s2attn_kernel_path.restype = _i
+_lib.s2attn_device_status.argtypes = [_vp, _sz, _vp]
+_lib.s2attn_device_status.restype = _i
+_lib.s2attn_status_string.argtypes = [_i]
+_lib.s2attn_status_string.restype = ctypes.c_char_p
+_lib.s2attn_profile_enable.argtypes = [_i]
+_lib.s2attn_profile_enable.restype = _i
+_lib.s2attn_profile_num_kernels.argtypes = []
+_lib.s2attn_profile_num_kernels.restype = _i
+_lib.s2attn_profile_query.argtypes = [_i, ctypes.POINTER(ctypes.c_char_p),
+                                      ctypes.POINTER(_i), ctypes.POINTER(ctypes.c_double)]
+_lib.s2attn_profile_query.restype = _i
+_lib.s2attn_profile_dropped.argtypes = []
+_lib.s2attn_profile_dropped.restype = _i
+
+# C ABI, same names and argument order as include/s2attn.h
+s2attn_workspace_bytes = _lib.s2attn_workspace_bytes
+s2attn_fwd = _lib.s2attn_fwd
+s2attn_bwd = _lib.s2attn_bwd
+s2attn_kernel_path = _lib.s2attn_kernel_path
+s2attn_device_status = _lib.s2attn_device_status
+s2attn_profile_enable = _lib.s2attn_profile_enable
+s2attn_profile_num_kernels = _lib.s2attn_profile_num_kernels
+s2attn_profile_dropped = _lib.s2attn_profile_dropped
+
+
+def s2attn_status_string(status: int) -> str:
+    return _lib.s2attn_status_string(int(status)).decode()
+
+
+def s2attn_profile_query(kernel_id: int):
+    """(name, launches, total_ms) of one kernel id."""
+    name = ctypes.c_char_p()
+    n = _i()
+    ms = ctypes.c_double()
+    rc = _lib.s2attn_profile_query(kernel_id, ctypes.byref(name), ctypes.byref(n),
+                                   ctypes.byref(ms))
+    check(rc)
+    return name.value.decode(), n.value, ms.value
+
+
+def profile_summary():
+    """{kernel name: (launches, total_ms)} for every kernel that launched."""
+    out = {}
+    for i in range(s2attn_profile_num_kernels()):
+        name, n, ms = s2attn_profile_query(i)
+        if n:
+            out[name] = (n, ms)
+    return out
+
+
+class S2Error(RuntimeError):
+    def __init__(self, status: int):
+        super().__init__("s2attn: %s (status %d)" % (s2attn_status_string(status), status))
+        self.status = status
+
+
+def check(status: int) -> None:
+    if status != S2_OK:
+        raise S2Error(status)
+
+
+# ----------------------------------------------------------------------------- torch layer
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return S2_BF16
+    if t.dtype == torch.float32:
+        return S2_FP32
+    raise TypeError("s2attn supports bfloat16 and float32 tensors, got %s" % t.dtype)
+
+
+def _stream_ptr(device) -> int:
+    import torch
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def workspace(B, N, Hq, Hkv, d, dtype_code, device):
+    import torch
+    nbytes = s2attn_workspace_bytes(B, N, Hq, Hkv, d, dtype_code)
+    if nbytes == 0:
+        raise S2Error(S2_ERR_SHAPE)
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def forward(q, k, v, G: int, pi_scale: float, rope_base: float = 10000.0, causal: bool = True,
+            ws=None, out=None, lse=None):
+    """q [B,N,Hq,d], k/v [B,N,Hkv,d] CUDA tensors -> (o, lse)."""
+    import torch
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    dt = _dtype_code(q)
+    if ws is None:
+        ws = workspace(B, N, Hq, Hkv, d, dt, q.device)
+    o = out if out is not None else torch.empty_like(q)
+    lse = lse if lse is not None else torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    check(s2attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                     B, N, Hq, Hkv, d, G, int(causal), pi_scale, rope_base, dt,
+                     ws.data_ptr(), ws.numel(), _stream_ptr(q.device)))
+    return o, lse
+
+
+def backward(q, k, v, o, lse, dout, G: int, pi_scale: float, rope_base: float = 10000.0,
+             causal: bool = True, ws=None, grads=None):
+    """Returns (dq, dk, dv) for the forward that produced (o, lse)."""
+    import torch
+    B, N, Hq, d = q.shape
+    Hkv = k.shape[2]
+    dt = _dtype_code(q)
+    if ws is None:
+        ws = workspace(B, N, Hq, Hkv, d, dt, q.device)
+    if grads is None:
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+    dq, dk, dv = grads
+    check(s2attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                     dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                     B, N, Hq, Hkv, d, G, int(causal), pi_scale, rope_base, dt,
+                     ws.data_ptr(), ws.numel(), _stream_ptr(q.device)))
+    return dq, dk, dv
+
+
+def device_status(ws) -> int:
+    import torch
+    return s2attn_device_status(ws.data_ptr(), ws.numel(), _stream_ptr(ws.device))
+
+
+def _make_function():
+    import torch
+
+    class S2AttnFunction(torch.autograd.Function):
+        """Autograd wrapper: o = S2Attn(q, k, v); backward through the library's kernels."""
+
+        @staticmethod
+        def forward(ctx, q, k, v, G, pi_scale, rope_base=10000.0, causal=True):
+            q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+            o, lse = forward(q, k, v, G, pi_scale, rope_base, causal)
+            ctx.save_for_backward(q, k, v, o, lse)
+            ctx.args = (G, pi_scale, rope_base, causal)
+            return o
+
+        @staticmethod
+        def backward(ctx, do):
+            q, k, v, o, lse = ctx.saved_tensors
+            G, pi_scale, rope_base, causal = ctx.args
+            dq, dk, dv = backward(q, k, v, o, lse, do.contiguous(), G, pi_scale, rope_base, causal)
+            return dq, dk, dv, None, None, None, None
+
+    return S2AttnFunction
+
+
+_fn = None
+
+
+def s2_attention(q, k, v, G: int, pi_scale: float, rope_base: float = 10000.0,
+                 causal: bool = True):
+    """Differentiable S2-Attn on CUDA tensors."""
+    global _fn
+    if _fn is None:
+        _fn = _make_function()
+    return _fn.apply(q, k, v, G, pi_scale, rope_base, causal)

@@ -46,6 +46,10 @@ def _load():
         lib.s2o_bwd_unit.argtypes = [vp, vp, vp, vp, i] + [i] * 7 + [d, d] + [i, i, i] + [dp, dp, dp]
         lib.s2o_fwd.argtypes = [vp, vp, vp, i] + [i] * 7 + [d, d] + [dp, dp]
         lib.s2o_bwd.argtypes = [vp, vp, vp, vp, i] + [i] * 7 + [d, d] + [dp, dp, dp]
+        lib.s2o_fwd_rows.argtypes = [vp, vp, vp, i] + [i] * 7 + [d, d] + [i, i, i] + \
+            [i, vp, dp, dp]
+        lib.s2o_bwd_rows.argtypes = [vp, vp, vp, vp, i] + [i] * 7 + [d, d] + [i, i, i] + \
+            [i, vp, i, vp, dp, dp, dp]
         lib.s2o_rope.argtypes = [dp, dp, i, vp, i, d, d, i]
         lib.s2o_rope.restype = None
         lib.s2o_max_threads.restype = i
@@ -163,3 +167,39 @@ def unit_rows(N: int, G: int, Hq: int, kvh: int, Hkv: int, g: int) -> np.ndarray
     shifted = kvh * R >= Hq // 2
     r = g * G + np.arange(G)
     return (r + G // 2) % N if shifted else r
+
+
+def fwd_rows(q, k, v, G: int, s: float, b: int, h: int, g: int, rows, base: float = 10000.0,
+             causal: bool = True):
+    """Forward at chosen rolled local rows of query head h, group g: (o [n,d], lse [n])."""
+    (q, dt), (k, _), (v, _) = _in(q), _in(k), _in(v)
+    B, N, Hq, Hkv, d = _dims(q, k)
+    rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+    o = np.empty((rows.size, d), dtype=np.float64)
+    lse = np.empty(rows.size, dtype=np.float64)
+    rc = _load().s2o_fwd_rows(_ptr(q), _ptr(k), _ptr(v), dt, B, N, Hq, Hkv, d, G, int(causal),
+                              float(s), float(base), b, h, g, rows.size, _ptr(rows), _ptr(o),
+                              _ptr(lse))
+    if rc:
+        raise ValueError("oracle fwd_rows rejected the arguments (rc=%d)" % rc)
+    return o, lse
+
+
+def bwd_rows(q, k, v, dout, G: int, s: float, b: int, kvh: int, g: int, qrows, krows,
+             base: float = 10000.0, causal: bool = True):
+    """Backward of unit (b, kvh, g) at chosen rolled local rows:
+    (dq [nq,R,d] for the R query heads of kvh, dk [nk,d], dv [nk,d])."""
+    (q, dt), (k, _), (v, _), (dout, _) = _in(q), _in(k), _in(v), _in(dout)
+    B, N, Hq, Hkv, d = _dims(q, k)
+    R = Hq // Hkv
+    qrows = np.ascontiguousarray(np.asarray(qrows, dtype=np.int32))
+    krows = np.ascontiguousarray(np.asarray(krows, dtype=np.int32))
+    dq = np.empty((qrows.size, R, d), dtype=np.float64)
+    dk = np.empty((krows.size, d), dtype=np.float64)
+    dv = np.empty((krows.size, d), dtype=np.float64)
+    rc = _load().s2o_bwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), dt, B, N, Hq, Hkv, d, G,
+                              int(causal), float(s), float(base), b, kvh, g, qrows.size,
+                              _ptr(qrows), krows.size, _ptr(krows), _ptr(dq), _ptr(dk), _ptr(dv))
+    if rc:
+        raise ValueError("oracle bwd_rows rejected the arguments (rc=%d)" % rc)
+    return dq, dk, dv

@@ -375,6 +375,171 @@ int s2o_bwd(const void* q, const void* k, const void* v, const void* dout, int d
   return err;
 }
 
+/* ------------------------------------------------------------------------------------
+ * Row-sampled evaluation: the same definition evaluated only at chosen rows, so that large
+ * shapes can be checked on sampled outputs. Row indices are rolled local rows of group g.
+ * ---------------------------------------------------------------------------------- */
+
+/* Softmax statistics and output of one query row i (rotated q row qi) against the group's
+ * rotated keys / values: lse and o (length d). sc is a G-length buffer. */
+static void row_forward(const cfg_t* c, const double* qi, const double* kr, const double* vr,
+                        int i, double* sc, double* o, double* lse_out) {
+  int d = c->d, G = c->G;
+  double inv_sqrt_d = 1.0 / sqrt((double)d);
+  int jmax = c->causal ? i : G - 1;
+  double mx = -INFINITY;
+  for (int j = 0; j <= jmax; j++) {
+    sc[j] = dot(qi, kr + (size_t)j * d, d) * inv_sqrt_d;
+    if (sc[j] > mx) mx = sc[j];
+  }
+  double sum = 0.0;
+  for (int j = 0; j <= jmax; j++) sum += exp(sc[j] - mx);
+  double lse = mx + log(sum);
+  for (int e = 0; e < d; e++) o[e] = 0.0;
+  for (int j = 0; j <= jmax; j++) {
+    double p = exp(sc[j] - lse);
+    for (int e = 0; e < d; e++) o[e] += p * vr[(size_t)j * d + e];
+  }
+  *lse_out = lse;
+}
+
+static void load_q_row(const cfg_t* c, const void* x, int dt, int b, int h, long m, double* tmp,
+                       double* out, int rotate) {
+  size_t base = (((size_t)b * c->N + m) * c->Hq + h) * c->d;
+  for (int e = 0; e < c->d; e++) tmp[e] = load(x, dt, base + e);
+  if (rotate)
+    rope(tmp, out, c->d, m, c->s, c->base, 0);
+  else
+    memcpy(out, tmp, (size_t)c->d * sizeof(double));
+}
+
+/* Forward at nrows rolled local rows of query head h in group g:
+ * o_rows [nrows][d], lse_rows [nrows]. */
+int s2o_fwd_rows(const void* q, const void* k, const void* v, int dt, int B, int N, int Hq,
+                 int Hkv, int d, int G, int causal, double s, double base, int b, int h, int g,
+                 int nrows, const int* rows, double* o_rows, double* lse_rows) {
+  cfg_t c;
+  scratch_t w;
+  if (s2o_check(B, N, Hq, Hkv, d, G)) return 1;
+  fill_cfg(&c, B, N, Hq, Hkv, d, G, causal, s, base);
+  int R = Hq / Hkv, kvh = h / R;
+  if (h < 0 || h >= Hq || !unit_args_ok(&c, b, kvh, g)) return 1;
+  for (int t = 0; t < nrows; t++)
+    if (rows[t] < 0 || rows[t] >= G) return 1;
+  if (!scratch_alloc(&w, G, d)) { scratch_free(&w); return 2; }
+  int shifted = shifted_head(&c, h);
+  load_group_kv(&c, k, v, dt, b, kvh, g, shifted, &w);
+#pragma omp parallel
+  {
+    double* sc = malloc((size_t)G * sizeof(double));
+    double* tmp = malloc((size_t)d * sizeof(double));
+    double* qi = malloc((size_t)d * sizeof(double));
+#pragma omp for schedule(dynamic, 4)
+    for (int t = 0; t < nrows; t++) {
+      long m = src_row(&c, (long)g * G + rows[t], shifted);
+      load_q_row(&c, q, dt, b, h, m, tmp, qi, 1);
+      row_forward(&c, qi, w.kr, w.vr, rows[t], sc, o_rows + (size_t)t * d, lse_rows + t);
+    }
+    free(sc); free(tmp); free(qi);
+  }
+  scratch_free(&w);
+  return 0;
+}
+
+/* Backward of unit (b, kvh, g) at sampled rows: dq at nq query rows for all R heads of the
+ * kv head (dq_rows [nq][R][d]) and dk, dv at nk key rows (dk_rows, dv_rows [nk][d]).
+ * The per-row statistics lse_i and D_i = <dO_i, O_i> that every gradient needs are
+ * computed for all G rows first (the oracle's own forward). */
+int s2o_bwd_rows(const void* q, const void* k, const void* v, const void* dout, int dt, int B,
+                 int N, int Hq, int Hkv, int d, int G, int causal, double s, double base, int b,
+                 int kvh, int g, int nq, const int* qrows, int nk, const int* krows,
+                 double* dq_rows, double* dk_rows, double* dv_rows) {
+  cfg_t c;
+  scratch_t w;
+  if (s2o_check(B, N, Hq, Hkv, d, G)) return 1;
+  fill_cfg(&c, B, N, Hq, Hkv, d, G, causal, s, base);
+  if (!unit_args_ok(&c, b, kvh, g)) return 1;
+  for (int t = 0; t < nq; t++)
+    if (qrows[t] < 0 || qrows[t] >= G) return 1;
+  for (int t = 0; t < nk; t++)
+    if (krows[t] < 0 || krows[t] >= G) return 1;
+  if (!scratch_alloc(&w, G, d)) { scratch_free(&w); return 2; }
+  int R = Hq / Hkv;
+  double inv_sqrt_d = 1.0 / sqrt((double)d);
+  int shifted = shifted_head(&c, kvh * R);
+  load_group_kv(&c, k, v, dt, b, kvh, g, shifted, &w);
+  double* dkr = calloc((size_t)(nk > 0 ? nk : 1) * d, sizeof(double));
+  double* dvr = calloc((size_t)(nk > 0 ? nk : 1) * d, sizeof(double));
+  for (int r = 0; r < R; r++) {
+    int h = kvh * R + r;
+    /* statistics of every row of the group */
+#pragma omp parallel
+    {
+      double* sc = malloc((size_t)G * sizeof(double));
+      double* tmp = malloc((size_t)d * sizeof(double));
+      double* orow = malloc((size_t)d * sizeof(double));
+#pragma omp for schedule(dynamic, 16)
+      for (int i = 0; i < G; i++) {
+        long m = src_row(&c, (long)g * G + i, shifted);
+        load_q_row(&c, q, dt, b, h, m, tmp, w.qr + (size_t)i * d, 1);
+        load_q_row(&c, dout, dt, b, h, m, tmp, w.dor + (size_t)i * d, 0);
+        row_forward(&c, w.qr + (size_t)i * d, w.kr, w.vr, i, sc, orow, w.lse + i);
+        w.Drow[i] = dot(w.dor + (size_t)i * d, orow, d);
+      }
+      free(sc); free(tmp); free(orow);
+    }
+    /* dq at the sampled query rows */
+#pragma omp parallel
+    {
+      double* acc = malloc((size_t)d * sizeof(double));
+#pragma omp for schedule(dynamic, 1)
+      for (int t = 0; t < nq; t++) {
+        int i = qrows[t];
+        const double* qi = w.qr + (size_t)i * d;
+        const double* doi = w.dor + (size_t)i * d;
+        int jmax = c.causal ? i : G - 1;
+        for (int e = 0; e < d; e++) acc[e] = 0.0;
+        for (int j = 0; j <= jmax; j++) {
+          const double* kj = w.kr + (size_t)j * d;
+          double p = exp(dot(qi, kj, d) * inv_sqrt_d - w.lse[i]);
+          double ds = p * (dot(doi, w.vr + (size_t)j * d, d) - w.Drow[i]);
+          for (int e = 0; e < d; e++) acc[e] += ds * inv_sqrt_d * kj[e];
+        }
+        long m = src_row(&c, (long)g * G + i, shifted);
+        rope(acc, dq_rows + ((size_t)t * R + r) * d, d, m, c.s, c.base, 1);
+      }
+      free(acc);
+    }
+    /* dk, dv at the sampled key rows (summed over the kv head's query heads) */
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int t = 0; t < nk; t++) {
+      int j = krows[t];
+      const double* kj = w.kr + (size_t)j * d;
+      const double* vj = w.vr + (size_t)j * d;
+      int ibeg = c.causal ? j : 0;
+      for (int i = ibeg; i < G; i++) {
+        const double* qi = w.qr + (size_t)i * d;
+        const double* doi = w.dor + (size_t)i * d;
+        double p = exp(dot(qi, kj, d) * inv_sqrt_d - w.lse[i]);
+        double ds = p * (dot(doi, vj, d) - w.Drow[i]);
+        for (int e = 0; e < d; e++) {
+          dkr[(size_t)t * d + e] += ds * inv_sqrt_d * qi[e];
+          dvr[(size_t)t * d + e] += p * doi[e];
+        }
+      }
+    }
+  }
+  for (int t = 0; t < nk; t++) {
+    long m = src_row(&c, (long)g * G + krows[t], shifted);
+    rope(dkr + (size_t)t * d, dk_rows + (size_t)t * d, d, m, c.s, c.base, 1);
+    memcpy(dv_rows + (size_t)t * d, dvr + (size_t)t * d, (size_t)d * sizeof(double));
+  }
+  free(dkr);
+  free(dvr);
+  scratch_free(&w);
+  return 0;
+}
+
 int s2o_max_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

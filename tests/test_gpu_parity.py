@@ -1,0 +1,197 @@
+"""GPU parity: the library (through its C ABI) against the fp64 oracle on identical seeded
+inputs. Small shapes are compared element by element in full; the LLaMA2-sized workloads
+run at full size in the configuration the bench times and are compared on sampled rows
+(tile edges, the half-group boundary, the wrap group of the shifted heads)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests import gpu_helpers as H
+from workloads import WORKLOADS, Workload
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def s2():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from longlora_shifted_sparse_b200 import s2attn  # raises if the library is missing
+    return s2attn
+
+
+def _run(s2, w, q, k, v, do):
+    tq, tk, tv = (H.to_device(x, w.dtype) for x in (q, k, v))
+    o, lse = s2.forward(tq, tk, tv, w.G, w.pi_scale, w.rope_base, w.causal)
+    grads = None
+    if do is not None:
+        tdo = H.to_device(do, w.dtype)
+        grads = s2.backward(tq, tk, tv, o, lse, tdo, w.G, w.pi_scale, w.rope_base, w.causal)
+    torch.cuda.synchronize()
+    return o, lse, grads
+
+
+def _full_compare(s2, w):
+    q, k, v, do = H.inputs(w, with_dout=w.backward)
+    o, lse, grads = _run(s2, w, q, k, v, do)
+    o_ref, lse_ref = oracle.fwd(q, k, v, w.G, w.pi_scale, w.rope_base, w.causal)
+    H.assert_close_o(H.to_host_f64(o), o_ref, w.dtype)
+    H.assert_close_lse(H.to_host_f64(lse), lse_ref, w.dtype)
+    if grads is not None:
+        refs = oracle.bwd(q, k, v, do, w.G, w.pi_scale, w.rope_base, w.causal)
+        for name, g, r in zip(("dq", "dk", "dv"), grads, refs):
+            H.assert_close_grad(H.to_host_f64(g), r, w.dtype, name)
+
+
+def test_tiny_fp32_workload_full(s2):
+    """The tiny fp32 workload (N=256, H=4, d=64, G=64, s=2), fwd+bwd, every element."""
+    _full_compare(s2, WORKLOADS["tiny_fp32"])
+
+
+SMALL = [
+    # name, B, N, Hq, Hkv, d, G, s, dtype, causal
+    ("bf16_d128_g256", 1, 1024, 4, 4, 128, 256, 2.0, "bf16", True),
+    ("bf16_gqa_b2", 2, 1024, 8, 2, 128, 512, 4.0, "bf16", True),
+    ("bf16_one_group", 1, 512, 4, 4, 128, 512, 1.0, "bf16", True),
+    ("bf16_noncausal", 1, 1024, 4, 4, 128, 256, 2.0, "bf16", False),
+    ("bf16_d64_g64", 1, 512, 4, 4, 64, 64, 2.0, "bf16", True),
+    ("bf16_d32_odd_tiles", 1, 600, 2, 2, 32, 200, 1.0, "bf16", True),
+    ("f32_d128_g96", 1, 384, 4, 2, 128, 96, 3.0, "f32", True),
+    ("f32_d256_noncausal", 1, 128, 2, 2, 256, 32, 1.0, "f32", False),
+    ("f32_g2_minimal", 1, 8, 2, 2, 32, 2, 1.0, "f32", True),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+def test_small_shapes_full(s2, case):
+    name, B, N, Hq, Hkv, d, G, s, dt, causal = case
+    w = Workload(name, B, N, Hq, Hkv, d, G, s, dt, 0.5 if dt == "bf16" else 1.0, True,
+                 seed=100 + SMALL.index(case), causal=causal)
+    _full_compare(s2, w)
+
+
+def _sampled_fwd_check(w, q, k, v, o, lse):
+    ng = w.N // w.G
+    heads = sorted({0, w.Hq // 2 - 1, w.Hq // 2, w.Hq - 1})
+    groups = sorted({0, ng // 2, ng - 1})
+    rows = H.sample_rows(w.G)
+    got_o, got_l, ref_o, ref_l = [], [], [], []
+    for h in heads:
+        kvh = h // (w.Hq // w.Hkv)
+        for g in groups:
+            tok = oracle.unit_rows(w.N, w.G, w.Hq, kvh, w.Hkv, g)[rows]
+            o_r, l_r = oracle.fwd_rows(q, k, v, w.G, w.pi_scale, 0, h, g, rows, w.rope_base,
+                                       w.causal)
+            idx = torch.as_tensor(tok, device=o.device)
+            got_o.append(H.to_host_f64(o[0, idx, h]))
+            got_l.append(H.to_host_f64(lse[0, h, idx]))
+            ref_o.append(o_r)
+            ref_l.append(l_r)
+    H.assert_close_o(np.concatenate(got_o), np.concatenate(ref_o), w.dtype)
+    H.assert_close_lse(np.concatenate(got_l), np.concatenate(ref_l), w.dtype)
+
+
+def _sampled_bwd_check(w, q, k, v, do, grads, units):
+    dq, dk, dv = grads
+    R = w.Hq // w.Hkv
+    rows = H.sample_rows(w.G, extra=4, seed=1)
+    gq, rq, gk, rk, gv, rv = [], [], [], [], [], []
+    for (b, kvh, g) in units:
+        tok = oracle.unit_rows(w.N, w.G, w.Hq, kvh, w.Hkv, g)[rows]
+        dq_r, dk_r, dv_r = oracle.bwd_rows(q, k, v, do, w.G, w.pi_scale, b, kvh, g, rows, rows,
+                                           w.rope_base, w.causal)
+        idx = torch.as_tensor(tok, device=dq.device)
+        gq.append(H.to_host_f64(dq[b, idx, kvh * R:(kvh + 1) * R]))
+        rq.append(dq_r)
+        gk.append(H.to_host_f64(dk[b, idx, kvh]))
+        rk.append(dk_r)
+        gv.append(H.to_host_f64(dv[b, idx, kvh]))
+        rv.append(dv_r)
+    H.assert_close_grad(np.concatenate(gq), np.concatenate(rq), w.dtype, "dq")
+    H.assert_close_grad(np.concatenate(gk), np.concatenate(rk), w.dtype, "dk")
+    H.assert_close_grad(np.concatenate(gv), np.concatenate(rv), w.dtype, "dv")
+
+
+BIG = ["llama2_7b_8k_fwd", "llama2_7b_32k", "llama2_70b_gqa_32k", "llama2_7b_100k"]
+
+
+@pytest.mark.parametrize("name", BIG)
+def test_llama2_workload_sampled(s2, name):
+    """Full-size run; O/LSE on sampled rows of both head halves and first / middle / last
+    (wrap) groups; dq/dk/dv on sampled rows of units in both halves incl. the wrap group."""
+    w = WORKLOADS[name]
+    q, k, v, do = H.inputs(w, with_dout=w.backward)
+    o, lse, grads = _run(s2, w, q, k, v, do)
+    _sampled_fwd_check(w, q, k, v, o, lse)
+    if w.backward:
+        ng = w.N // w.G
+        units = [(0, 0, 0), (0, w.Hkv - 1, ng - 1)]
+        if name != "llama2_7b_100k":
+            units += [(0, w.Hkv // 2, 0), (0, w.Hkv // 2 - 1, ng - 1)]
+        _sampled_bwd_check(w, q, k, v, do, grads, units)
+
+
+def test_outputs_stay_inside_their_buffers(s2):
+    """Canary bands (NaN patterns) around every output are untouched."""
+    w = Workload("canary", 1, 1024, 4, 2, 128, 256, 2.0, "bf16", 0.5, True, seed=7)
+    q, k, v, do = H.inputs(w)
+    tq, tk, tv, tdo = (H.to_device(x, "bf16") for x in (q, k, v, do))
+    pad = 64
+
+    def padded(shape, dtype):
+        n = int(np.prod(shape))
+        buf = torch.empty(n + 2 * pad, dtype=dtype, device="cuda")
+        buf.view(torch.int16 if dtype == torch.bfloat16 else torch.int32).fill_(-1)
+        return buf, buf[pad:pad + n].view(shape)
+
+    ob, o = padded(tq.shape, torch.bfloat16)
+    lb, lse = padded((1, w.Hq, w.N), torch.float32)
+    qb, dq = padded(tq.shape, torch.bfloat16)
+    kb, dk = padded(tk.shape, torch.bfloat16)
+    vb, dv = padded(tv.shape, torch.bfloat16)
+    s2.forward(tq, tk, tv, w.G, w.pi_scale, out=o, lse=lse)
+    s2.backward(tq, tk, tv, o, lse, tdo, w.G, w.pi_scale, grads=(dq, dk, dv))
+    torch.cuda.synchronize()
+    for buf in (ob, lb, qb, kb, vb):
+        ints = buf.view(torch.int16 if buf.dtype == torch.bfloat16 else torch.int32)
+        assert bool((ints[:pad] == -1).all()) and bool((ints[-pad:] == -1).all())
+    assert bool(torch.isfinite(o).all()) and bool(torch.isfinite(dq).all())
+
+
+def test_results_are_deterministic(s2):
+    w = Workload("det", 1, 2048, 8, 2, 128, 512, 4.0, "bf16", 0.5, True, seed=8)
+    q, k, v, do = H.inputs(w)
+    a = _run(s2, w, q, k, v, do)
+    b = _run(s2, w, q, k, v, do)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    for x, y in zip(a[2], b[2]):
+        assert torch.equal(x, y)
+
+
+def test_autograd_function_matches_abi_calls(s2):
+    w = Workload("ag", 1, 512, 4, 4, 64, 128, 2.0, "f32", 1.0, True, seed=9)
+    q, k, v, do = H.inputs(w)
+    tq, tk, tv = (H.to_device(x, "f32").requires_grad_(True) for x in (q, k, v))
+    o = s2.s2_attention(tq, tk, tv, w.G, w.pi_scale)
+    o.backward(H.to_device(do, "f32"))
+    o2, lse2, (dq, dk, dv) = _run(s2, w, q, k, v, do)
+    assert torch.equal(o.detach(), o2)
+    assert torch.equal(tq.grad, dq) and torch.equal(tk.grad, dk) and torch.equal(tv.grad, dv)
+
+
+def test_device_status_and_profiler(s2):
+    w = Workload("prof", 1, 1024, 4, 4, 128, 256, 2.0, "bf16", 0.5, True, seed=10)
+    q, k, v, do = H.inputs(w)
+    tq, tk, tv = (H.to_device(x, "bf16") for x in (q, k, v))
+    ws = s2.workspace(w.B, w.N, w.Hq, w.Hkv, w.d, s2.S2_BF16, tq.device)
+    s2.check(s2.s2attn_profile_enable(1))
+    o, lse = s2.forward(tq, tk, tv, w.G, w.pi_scale, ws=ws)
+    s2.backward(tq, tk, tv, o, lse, H.to_device(do, "bf16"), w.G, w.pi_scale, ws=ws)
+    assert s2.device_status(ws) == s2.S2_OK
+    summary = s2.profile_summary()
+    s2.check(s2.s2attn_profile_enable(0))
+    assert summary["rope_pi"][0] == 2 and summary["bwd_rowsum"][0] == 1
+    assert sum(n for n, _ in summary.values()) == 6
+    assert all(ms > 0 for _, ms in summary.values())

@@ -298,6 +298,29 @@ def test_unit_functions_agree_with_full_functions():
         np.testing.assert_array_equal(dv_u, dv[b, rows, kvh])
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_row_sampled_functions_agree_with_full_functions(causal):
+    N, G, d, Hq, Hkv = 64, 16, 8, 8, 2
+    q, k, v, do = _inputs(16, 2, N, Hq, Hkv, d)
+    o, lse = oracle.fwd(q, k, v, G=G, s=2.0, causal=causal)
+    dq, dk, dv = oracle.bwd(q, k, v, do, G=G, s=2.0, causal=causal)
+    R = Hq // Hkv
+    rows = np.array([0, 1, 7, 15, 3])
+    for b, kvh, g in ((0, 0, 0), (1, 1, N // G - 1), (1, 1, 0)):
+        tok = oracle.unit_rows(N, G, Hq, kvh, Hkv, g)[rows]
+        for r in range(R):
+            h = kvh * R + r
+            o_r, l_r = oracle.fwd_rows(q, k, v, G, 2.0, b, h, g, rows, causal=causal)
+            np.testing.assert_allclose(o_r, o[b, tok, h], rtol=0, atol=1e-14)
+            np.testing.assert_allclose(l_r, lse[b, h, tok], rtol=0, atol=1e-14)
+        dq_r, dk_r, dv_r = oracle.bwd_rows(q, k, v, do, G, 2.0, b, kvh, g, rows, rows[::-1],
+                                           causal=causal)
+        for r in range(R):
+            np.testing.assert_allclose(dq_r[:, r], dq[b, tok, kvh * R + r], atol=1e-13)
+        np.testing.assert_allclose(dk_r, dk[b, tok[::-1], kvh], atol=1e-13)
+        np.testing.assert_allclose(dv_r, dv[b, tok[::-1], kvh], atol=1e-13)
+
+
 def test_oracle_rejects_shapes_the_method_cannot_take():
     assert oracle.check(1, 64, 4, 4, 8, 16)
     assert not oracle.check(1, 60, 4, 4, 8, 16)   # N % G
