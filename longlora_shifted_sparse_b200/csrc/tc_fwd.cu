@@ -1,0 +1,340 @@
+// S2-Attn forward on the 5th-generation tensor cores (tcgen05, TMEM accumulators, TMA).
+//
+// Work item = one 128-row query tile of one (batch, query head, group): rolled rows
+// g*G + qt*128 ... + 127. A shifted head's rolled row r is token (r + G/2) mod N, and
+// because G/2 is a multiple of 128 a tile never straddles the wrap, so the -G/2 roll of q,
+// k, v and the +G/2 roll back of o are just the row coordinate of each TMA load / store
+// ("LongLoRA and Shifted Sparse Attention (S^2-Attn)", definition; "LongLoRA: Efficient
+// 100k Context LLM Fine-Tuning Guide", Implementation, Step 1). Inside the group the
+// query tile attends to key tiles 0..qt (causal: tiles above the diagonal are skipped and
+// the diagonal tile is masked on group-local positions).
+//
+// Roles (192 threads):
+//   warp 0      TMA producer: Q once, then K_j and V_j into two 2-stage rings.
+//   warp 1      MMA issuer (one thread) and TMEM owner: S_j = Q K_j^T into one of two
+//               TMEM score buffers, then O += P_{j-1} V_{j-1} with P read from TMEM.
+//   warps 2..5  softmax: thread = query row = TMEM lane. Reads its S row, keeps the
+//               running max / sum in fp32 (exp2 domain, log2(e)/sqrt(d) folded into one
+//               scale), writes P as bf16 over the S buffer it came from, and rescales
+//               the O accumulator in TMEM only when the running max grows by more than
+//               2^8 (the stale max keeps every P <= 256). Epilogue: O / l -> bf16 at the
+//               token's original row, LSE = ln 2 * (m + log2 l).
+// TMEM: S0 [0,128), S1 [128,256), O [256,384) of a 512-column allocation.
+// Every wait is bounded; on expiry the CTA records it in the status word and drains.
+#include "common.cuh"
+#include "sm100.cuh"
+#include "tc_kernels.h"
+#include "tma_host.h"
+
+namespace s2 {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;
+constexpr int kTile = 128;
+constexpr uint32_t kTileBytes = kTile * kD * 2;    // 32 KB: 128 rows x 128 bf16
+constexpr uint32_t kHalfBytes = kTileBytes / 2;    // one 128 x 64 TMA box
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
+constexpr float kRescaleThreshold = 8.0f;          // log2 units
+
+// dynamic shared memory: Q | K0 K1 | V0 V1, each 32 KB, 1024-byte aligned
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kTileBytes;
+constexpr uint32_t kOffV = 3 * kTileBytes;
+constexpr uint32_t kSmemBytes = 5 * kTileBytes + 1024;
+
+struct FwdBarriers {
+  uint64_t q_full;
+  uint64_t k_full[2], k_empty[2];
+  uint64_t v_full[2], v_empty[2];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_done;
+  uint64_t drain;
+};
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// A or B operand tile (128 rows x 128 bf16, two 64-column SW128 boxes), K-major, k-step kk.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_saddr, int kk) {
+  return smem_desc_sw128(tile_saddr + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
+}
+
+// V tile as the MN-major B operand of O += P V: k-step kk covers kv rows 16kk..16kk+15.
+__device__ __forceinline__ uint64_t v_desc(uint32_t tile_saddr, int kk) {
+  return smem_desc_sw128(tile_saddr + kk * 2048, kHalfBytes, 1024);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_fwd_kernel(const Params p, const __grid_constant__ CUtensorMap tm_q,
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  __shared__ FwdBarriers bars;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = p.G / kTile, ng = p.N / p.G;
+  const int per_qt = p.B * p.Hq * ng;
+  const int qt = T - 1 - (int)(blockIdx.x / per_qt);  // heaviest query tiles first
+  const int rest = (int)(blockIdx.x % per_qt);
+  const int g = rest % ng, bh = rest / ng;
+  const int h = bh % p.Hq, b = bh / p.Hq;
+  const int kvh = h / (p.Hq / p.Hkv);
+  const bool sh = head_shifted(h, p.Hq);
+  const int nkv = p.causal ? qt + 1 : T;
+  const int r0 = g * p.G + qt * kTile;  // rolled row of the tile's first query
+
+  Abort ab{&abort_flag, p.status};
+  if (threadIdx.x == 0) {
+    // a CTA of this launch already gave up: do nothing (outputs are undefined then)
+    abort_flag = *reinterpret_cast<volatile unsigned*>(p.status) != 0u;
+    mbar_init(smem_addr(&bars.q_full), 1);
+    for (int s = 0; s < 2; s++) {
+      mbar_init(smem_addr(&bars.k_full[s]), 1);
+      mbar_init(smem_addr(&bars.k_empty[s]), 1);
+      mbar_init(smem_addr(&bars.v_full[s]), 1);
+      mbar_init(smem_addr(&bars.v_empty[s]), 1);
+      mbar_init(smem_addr(&bars.s_full[s]), 1);
+      mbar_init(smem_addr(&bars.p_full[s]), 128);
+    }
+    mbar_init(smem_addr(&bars.o_done), 1);
+    mbar_init(smem_addr(&bars.drain), 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(smem_addr(&tmem_base_sh), kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  const uint32_t sQ = smem_addr(smem + kOffQ);
+  const bool skip = abort_flag != 0;
+
+  if (skip) {
+    // fall through to the teardown
+  } else if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      const int qrow = (b * p.Hq + h) * p.N + src_row(r0, sh, p.G, p.N);
+      mbar_arrive_expect_tx(smem_addr(&bars.q_full), kTileBytes);
+      tma_load_2d(sQ, &tm_q, smem_addr(&bars.q_full), 0, qrow);
+      tma_load_2d(sQ + kHalfBytes, &tm_q, smem_addr(&bars.q_full), 64, qrow);
+      int issued = 0;
+      for (int j = 0; j < nkv; j++) {
+        const int s = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        const int mk = src_row(g * p.G + j * kTile, sh, p.G, p.N);
+        if (!mbar_wait(smem_addr(&bars.k_empty[s]), ph ^ 1, ab)) break;
+        const uint32_t sK = smem_addr(smem + kOffK + s * kTileBytes);
+        mbar_arrive_expect_tx(smem_addr(&bars.k_full[s]), kTileBytes);
+        tma_load_2d(sK, &tm_k, smem_addr(&bars.k_full[s]), 0, (b * p.Hkv + kvh) * p.N + mk);
+        tma_load_2d(sK + kHalfBytes, &tm_k, smem_addr(&bars.k_full[s]), 64,
+                    (b * p.Hkv + kvh) * p.N + mk);
+        if (!mbar_wait(smem_addr(&bars.v_empty[s]), ph ^ 1, ab)) {
+          issued = 2 * j + 1;
+          break;
+        }
+        const uint32_t sV = smem_addr(smem + kOffV + s * kTileBytes);
+        mbar_arrive_expect_tx(smem_addr(&bars.v_full[s]), kTileBytes);
+        tma_load_3d(sV, &tm_v, smem_addr(&bars.v_full[s]), 0, kvh, b * p.N + mk);
+        tma_load_3d(sV + kHalfBytes, &tm_v, smem_addr(&bars.v_full[s]), 64, kvh, b * p.N + mk);
+        issued = 2 * j + 2;
+      }
+      // Let the last loads in flight land before the CTA can exit. This wait ignores the
+      // abort flag (it is set on this path) but keeps its own time limit.
+      int no_abort = 0;
+      Abort local{&no_abort, p.status};
+      for (int t = issued - 1; t >= 0 && t >= issued - 4; t--) {
+        const int j = t >> 1, s = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        mbar_wait(smem_addr((t & 1) ? &bars.v_full[s] : &bars.k_full[s]), ph, local);
+      }
+      mbar_wait(smem_addr(&bars.q_full), 0, local);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc_qk = idesc_bf16_f32(kTile, kTile, false, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(kTile, kD, false, true);
+      bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
+      tc_fence_after();
+      for (int j = 0; ok && j <= nkv; j++) {
+        if (j < nkv) {
+          const int s = j & 1;
+          const uint32_t ph = (j >> 1) & 1;
+          if (!mbar_wait(smem_addr(&bars.k_full[s]), ph, ab)) break;
+          tc_fence_after();
+          const uint32_t sK = smem_addr(smem + kOffK + s * kTileBytes);
+          const uint32_t dS = tmem + (s ? kColS1 : kColS0);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; kk++)
+            mma_ss(dS, kmajor_desc(sQ, kk), kmajor_desc(sK, kk), idesc_qk, kk > 0);
+          mma_commit(smem_addr(&bars.s_full[s]));
+          mma_commit(smem_addr(&bars.k_empty[s]));
+        }
+        if (j >= 1) {
+          const int jj = j - 1, s = jj & 1;
+          const uint32_t ph = (jj >> 1) & 1;
+          if (!mbar_wait(smem_addr(&bars.p_full[s]), ph, ab)) break;
+          if (!mbar_wait(smem_addr(&bars.v_full[s]), ph, ab)) break;
+          tc_fence_after();
+          const uint32_t sV = smem_addr(smem + kOffV + s * kTileBytes);
+          const uint32_t aP = tmem + (s ? kColS1 : kColS0);
+#pragma unroll
+          for (int kk = 0; kk < kTile / 16; kk++)
+            mma_ts(tmem + kColO, aP + kk * 8, v_desc(sV, kk), idesc_pv, (jj > 0 || kk > 0));
+          mma_commit(smem_addr(&bars.v_empty[s]));
+          mma_commit(smem_addr(&bars.o_done));
+        }
+      }
+      // every MMA issued above has completed before TMEM is released
+      mma_commit(smem_addr(&bars.drain));
+      int no_abort = 0;
+      Abort local{&no_abort, p.status};
+      mbar_wait(smem_addr(&bars.drain), 0, local);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax / epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkv; j++) {
+      const int s = j & 1;
+      const uint32_t ph = (j >> 1) & 1;
+      ok = mbar_wait(smem_addr(&bars.s_full[s]), ph, ab);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t tS = tmem + lane_off + (s ? kColS1 : kColS0);
+      uint32_t r[4][32];
+#pragma unroll
+      for (int ch = 0; ch < 4; ch++) tmem_ld32(tS + ch * 32, r[ch]);
+      tmem_wait_ld();
+      const bool diag = p.causal && j == qt;
+      float mt = -INFINITY;
+#pragma unroll
+      for (int ch = 0; ch < 4; ch++)
+#pragma unroll
+        for (int c = 0; c < 32; c++) {
+          float x = __uint_as_float(r[ch][c]) * sl2;
+          if (diag && ch * 32 + c > row) x = -INFINITY;
+          r[ch][c] = __float_as_uint(x);
+          mt = fmaxf(mt, x);
+        }
+      float alpha = 1.f;
+      bool rescale = false;
+      if (mt > m + kRescaleThreshold) {
+        alpha = fast_exp2(m - mt);  // 0 while m is -inf
+        rescale = j > 0;
+        m = mt;
+      }
+      float rs = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 4; ch++) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int t = 0; t < 16; t++) {
+          const float p0 = fast_exp2(__uint_as_float(r[ch][2 * t]) - m);
+          const float p1 = fast_exp2(__uint_as_float(r[ch][2 * t + 1]) - m);
+          rs += p0 + p1;
+          pk[t] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + ch * 16, pk);
+      }
+      l = l * alpha + rs;
+      tmem_wait_st();
+      if (j > 0) {
+        ok = mbar_wait(smem_addr(&bars.o_done), (j - 1) & 1, ab);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale)) {
+          const uint32_t tO = tmem + lane_off + kColO;
+#pragma unroll
+          for (int ch = 0; ch < 4; ch++) {
+            uint32_t o[32];
+            tmem_ld32(tO + ch * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; c++) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st32(tO + ch * 32, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_addr(&bars.p_full[s]));
+    }
+    if (ok) {
+      ok = mbar_wait(smem_addr(&bars.o_done), (nkv - 1) & 1, ab);
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const int mrow = src_row(r0 + row, sh, p.G, p.N);
+      __nv_bfloat16* orow =
+          static_cast<__nv_bfloat16*>(p.o) + ((size_t)(b * p.N + mrow) * p.Hq + h) * kD;
+      const float inv_l = 1.f / l;
+      const uint32_t tO = tmem + lane_off + kColO;
+#pragma unroll
+      for (int ch = 0; ch < 4; ch++) {
+        uint32_t o[32];
+        tmem_ld32(tO + ch * 32, o);
+        tmem_wait_ld();
+        uint4 pk[4];
+        uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+        for (int t = 0; t < 16; t++)
+          pw[t] = pack_bf16x2(__uint_as_float(o[2 * t]) * inv_l, __uint_as_float(o[2 * t + 1]) * inv_l);
+        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+        for (int t = 0; t < 4; t++) dst[t] = pk[t];
+      }
+      p.lse[((size_t)b * p.Hq + h) * p.N + mrow] = (m + __log2f(l)) * 0.69314718055994531f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_tc_fwd(const Params& p, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  cudaError_t e;
+  if ((e = make_tmap_bf16_2d(&tq, p.qr, kD, (uint64_t)p.B * p.Hq * p.N, kD * 2, 64, kTile)))
+    return e;
+  if ((e = make_tmap_bf16_2d(&tk, p.kr, kD, (uint64_t)p.B * p.Hkv * p.N, kD * 2, 64, kTile)))
+    return e;
+  if ((e = make_tmap_bf16_3d(&tv, p.v, kD, p.Hkv, (uint64_t)p.B * p.N, kD * 2,
+                             (uint64_t)p.Hkv * kD * 2, 64, kTile)))
+    return e;
+  if ((e = cudaFuncSetAttribute(tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)kSmemBytes)))
+    return e;
+  const long tiles = (long)p.B * p.Hq * (p.N / p.G) * (p.G / kTile);
+  tc_fwd_kernel<<<dim3((unsigned)tiles), dim3(kThreads), kSmemBytes, st>>>(p, tq, tk, tv);
+  return cudaGetLastError();
+}
+
+}  // namespace s2
