@@ -93,6 +93,29 @@ S2_API s2_status s2attn_bwd(const void* q, const void* k, const void* v, const v
                      float pi_scale, float rope_base, int dtype,
                      void* workspace, size_t ws_bytes, void* cuda_stream);
 
+/* Bytes of the fixed scratch array that s2attn_fwd_noalloc uses on each device. */
+#define S2ATTN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/* Forward for callers that cannot allocate device memory per call (a plugin whose host
+ * application owns every device allocation, a latency-critical loop that cannot afford
+ * cudaMalloc's implicit synchronisation, a C caller with no allocator). The pages have no
+ * counterpart: this is a deployment variant of s2attn_fwd, not part of the method.
+ * Same arguments, semantics and outputs as s2attn_fwd, minus the workspace: the scratch is
+ * a fixed S2ATTN_NOALLOC_SCRATCH_BYTES array inside the library, which every device that
+ * loads the library holds until the process exits. Neither this call nor the library
+ * allocates memory (no cudaMalloc, cudaFree or allocating library routine).
+ *  - Limit: shapes whose s2attn_workspace_bytes() exceeds S2ATTN_NOALLOC_SCRATCH_BYTES are
+ *    rejected with S2_ERR_WORKSPACE before anything is enqueued.
+ *  - Set-up: the first call on a device looks up the array's device address (with that
+ *    device current) and caches it; make that first call before any stream capture.
+ *  - Sharing: every call on a device uses the same array and leaves its contents behind
+ *    (each call rewrites what it reads, and resets the status word first). Calls whose
+ *    kernels overlap on the GPU (e.g. on two streams) race on the array: serialise them. */
+S2_API s2_status s2attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o,
+                                    float* lse, int B, int N, int H_q, int H_kv, int d, int G,
+                                    int causal, float pi_scale, float rope_base, int dtype,
+                                    void* cuda_stream);
+
 /* Which kernel family s2attn_fwd/s2attn_bwd launch for these arguments:
  * 1 = tcgen05 tensor-core kernels (bf16, d == 128, G % 256 == 0),
  * 0 = CUDA-core kernels (any other valid shape, and every fp32 call), -1 = invalid. */

@@ -332,3 +332,69 @@ int s2attn_profile_dropped(void) {
 }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------- no-allocation forward
+//
+// Some callers must not allocate device memory for a call: a plugin whose host application
+// owns every device allocation, a latency-critical loop that cannot afford cudaMalloc's
+// implicit device synchronisation, or a plain C caller with no allocator at hand. For them
+// s2attn_fwd_noalloc runs the same kernels as s2attn_fwd, with the workspace replaced by a
+// fixed array compiled into this library (allocated by the driver when the library's
+// device code is loaded, held by every device that loads it until the process exits).
+namespace s2 {
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[S2ATTN_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device. In host code the array's
+// name is only a host-side stand-in, so the address is looked up with the device current,
+// once per device, and cached.
+cudaError_t noalloc_scratch_address(void** out) {
+  static std::mutex mu;
+  static std::vector<void*> addr;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  if ((int)addr.size() <= dev) addr.resize(dev + 1, nullptr);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace s2
+
+extern "C" s2_status s2attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o,
+                                        float* lse, int B, int N, int H_q, int H_kv, int d, int G,
+                                        int causal, float pi_scale, float rope_base, int dtype,
+                                        void* cuda_stream) {
+  if (!q || !k || !v || !o || !lse) return S2_ERR_NULL;
+  if (!dtype_ok(dtype)) return S2_ERR_DTYPE;
+  if (!shape_ok(B, N, H_q, H_kv, G)) return S2_ERR_SHAPE;
+  if (!headdim_ok(d)) return S2_ERR_HEADDIM;
+  if (!(isfinite(pi_scale) && pi_scale > 0.f) || !(isfinite(rope_base) && rope_base > 0.f) ||
+      (causal != 0 && causal != 1))
+    return S2_ERR_ARG;
+  if (ws_layout(B, N, H_q, H_kv, d, dtype).total > (size_t)S2ATTN_NOALLOC_SCRATCH_BYTES)
+    return S2_ERR_WORKSPACE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return S2_ERR_ALIGN;
+  void* scratch = nullptr;
+  if (noalloc_scratch_address(&scratch) != cudaSuccess) return S2_ERR_CUDA;
+  // The status word at the start of the scratch is reset by the first kernel of the call;
+  // everything else the kernels read from the scratch is written earlier in the same call.
+  Params p = make_params(B, N, H_q, H_kv, d, G, causal, pi_scale, rope_base, dtype, scratch);
+  p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
+  const bool bf16 = dtype == S2_BF16;
+  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e = timed_launch(kRopePi, s, [&] { return launch_rope_pi(p, bf16, s); });
+  if (e != cudaSuccess) return to_status(e);
+  e = timed_launch(kFwdSimt, s, [&] { return launch_simt_fwd(p, bf16, s); });
+  return to_status(e);
+}

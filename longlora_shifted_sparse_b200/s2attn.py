@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libs2attn.so")
 S2_OK, S2_ERR_NULL, S2_ERR_SHAPE, S2_ERR_DTYPE, S2_ERR_HEADDIM, S2_ERR_ALIGN, \
     S2_ERR_WORKSPACE, S2_ERR_CUDA, S2_ERR_DEVICE_TIMEOUT, S2_ERR_ARG = range(10)
 S2_BF16, S2_FP32 = 0, 1
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # S2ATTN_NOALLOC_SCRATCH_BYTES
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(
@@ -38,6 +39,8 @@ _lib.s2attn_fwd.argtypes = [_vp] * 5 + _SHAPE + [_vp, _sz, _vp]
 _lib.s2attn_fwd.restype = _i
 _lib.s2attn_bwd.argtypes = [_vp] * 9 + _SHAPE + [_vp, _sz, _vp]
 _lib.s2attn_bwd.restype = _i
+_lib.s2attn_fwd_noalloc.argtypes = [_vp] * 5 + _SHAPE + [_vp]
+_lib.s2attn_fwd_noalloc.restype = _i
 _lib.s2attn_kernel_path.argtypes = [_i] * 8
 _lib.s2attn_kernel_path.restype = _i
 _lib.s2attn_device_status.argtypes = [_vp, _sz, _vp]
@@ -58,6 +61,7 @@ _lib.s2attn_profile_dropped.restype = _i
 s2attn_workspace_bytes = _lib.s2attn_workspace_bytes
 s2attn_fwd = _lib.s2attn_fwd
 s2attn_bwd = _lib.s2attn_bwd
+s2attn_fwd_noalloc = _lib.s2attn_fwd_noalloc
 s2attn_kernel_path = _lib.s2attn_kernel_path
 s2attn_device_status = _lib.s2attn_device_status
 s2attn_profile_enable = _lib.s2attn_profile_enable
