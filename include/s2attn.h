@@ -116,7 +116,7 @@ S2_API s2_status s2attn_fwd_noalloc(const void* q, const void* k, const void* v,
                                     int causal, float pi_scale, float rope_base, int dtype,
                                     void* cuda_stream);
 
-/* Which kernel family s2attn_fwd/s2attn_bwd launch for these arguments:
+/* Which kernel family s2attn_fwd launches for these arguments:
  * 1 = tcgen05 tensor-core kernels (bf16, d == 128, G % 256 == 0),
  * 0 = CUDA-core kernels (any other valid shape, and every fp32 call), -1 = invalid. */
 S2_API int s2attn_kernel_path(int B, int N, int H_q, int H_kv, int d, int G, int causal, int dtype);

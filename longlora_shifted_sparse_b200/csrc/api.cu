@@ -9,6 +9,7 @@
 #include "../../include/s2attn.h"
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_kernels.h"
 
 namespace s2 {
 namespace {
@@ -161,8 +162,18 @@ WsLayout ws_layout(int B, int N, int Hq, int Hkv, int d, int dt) {
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
-// The tcgen05 kernels are not built yet: every call takes the CUDA-core kernels.
-bool tc_path(int, int, int) { return false; }
+// tcgen05 kernels: bf16, d == 128, and G/2 a whole number of 128-row tiles (no tile
+// straddles the wrap of the shifted heads).
+bool tc_path(int d, int G, int dt) { return dt == S2_BF16 && d == 128 && G % 256 == 0; }
+
+// RoPE+PI stage, then the forward kernel of the selected family.
+cudaError_t enqueue_forward(const Params& p, int dt, cudaStream_t s) {
+  const bool bf16 = dt == S2_BF16;
+  cudaError_t e = timed_launch(kRopePi, s, [&] { return launch_rope_pi(p, bf16, s); });
+  if (e != cudaSuccess) return e;
+  if (tc_path(p.d, p.G, dt)) return timed_launch(kFwdTc, s, [&] { return launch_tc_fwd(p, s); });
+  return timed_launch(kFwdSimt, s, [&] { return launch_simt_fwd(p, bf16, s); });
+}
 
 s2_status common_checks(int B, int N, int Hq, int Hkv, int d, int G, int causal, float s,
                         float base, int dt, void* ws, size_t ws_bytes) {
@@ -230,12 +241,7 @@ s2_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, float
     return S2_ERR_ALIGN;
   Params p = make_params(B, N, H_q, H_kv, d, G, causal, pi_scale, rope_base, dtype, workspace);
   p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
-  const bool bf16 = dtype == S2_BF16;
-  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-  cudaError_t e = timed_launch(kRopePi, s, [&] { return launch_rope_pi(p, bf16, s); });
-  if (e != cudaSuccess) return to_status(e);
-  e = timed_launch(kFwdSimt, s, [&] { return launch_simt_fwd(p, bf16, s); });
-  return to_status(e);
+  return to_status(enqueue_forward(p, dtype, static_cast<cudaStream_t>(cuda_stream)));
 }
 
 s2_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -391,10 +397,5 @@ extern "C" s2_status s2attn_fwd_noalloc(const void* q, const void* k, const void
   // everything else the kernels read from the scratch is written earlier in the same call.
   Params p = make_params(B, N, H_q, H_kv, d, G, causal, pi_scale, rope_base, dtype, scratch);
   p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
-  const bool bf16 = dtype == S2_BF16;
-  cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-  cudaError_t e = timed_launch(kRopePi, s, [&] { return launch_rope_pi(p, bf16, s); });
-  if (e != cudaSuccess) return to_status(e);
-  e = timed_launch(kFwdSimt, s, [&] { return launch_simt_fwd(p, bf16, s); });
-  return to_status(e);
+  return to_status(enqueue_forward(p, dtype, static_cast<cudaStream_t>(cuda_stream)));
 }

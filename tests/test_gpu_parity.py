@@ -69,6 +69,9 @@ def test_small_shapes_full(s2, case):
     name, B, N, Hq, Hkv, d, G, s, dt, causal = case
     w = Workload(name, B, N, Hq, Hkv, d, G, s, dt, 0.5 if dt == "bf16" else 1.0, True,
                  seed=100 + SMALL.index(case), causal=causal)
+    expect_tc = dt == "bf16" and d == 128 and G % 256 == 0
+    code = s2.S2_BF16 if dt == "bf16" else s2.S2_FP32
+    assert s2.s2attn_kernel_path(B, N, Hq, Hkv, d, G, int(causal), code) == int(expect_tc)
     _full_compare(s2, w)
 
 
@@ -122,6 +125,8 @@ def test_llama2_workload_sampled(s2, name):
     """Full-size run; O/LSE on sampled rows of both head halves and first / middle / last
     (wrap) groups; dq/dk/dv on sampled rows of units in both halves incl. the wrap group."""
     w = WORKLOADS[name]
+    # these shapes must take the tensor-core kernels
+    assert s2.s2attn_kernel_path(w.B, w.N, w.Hq, w.Hkv, w.d, w.G, int(w.causal), s2.S2_BF16) == 1
     q, k, v, do = H.inputs(w, with_dout=w.backward)
     o, lse, grads = _run(s2, w, q, k, v, do)
     _sampled_fwd_check(w, q, k, v, o, lse)
