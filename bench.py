@@ -35,6 +35,27 @@ METRIC = "S2-Attn fwd+bwd TFLOP/s (bf16, 1 B200) and % of dense bf16 tensor-core
 UNIT = "TFLOP/s"
 
 
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own independent batch of the workload."""
+    return seed + 1000 * rank
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(step_flops: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank's counted FLOPs over the slowest rank's step time."""
+    return step_flops * world / (ms_per_step * 1e-3) / 1e12
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -219,7 +240,7 @@ def run_ours(args):
     es = 2 if w.dtype == "bf16" else 4
 
     # seeded host inputs, one independent batch per rank
-    q, k, v, do = synth.s2attn_inputs(w.seed + 1000 * rank, w.B, w.N, w.Hq, w.Hkv, w.d,
+    q, k, v, do = synth.s2attn_inputs(rank_seed(w.seed, rank), w.B, w.N, w.Hq, w.Hkv, w.d,
                                       w.in_scale, w.dtype)
 
     def host_pinned(x):
@@ -275,13 +296,10 @@ def run_ours(args):
     elapsed_ms = e0.elapsed_time(e1)
     if s2.device_status(ws) != s2.S2_OK:
         raise RuntimeError("device status reports an expired wait in the timed region")
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
     ms_per_step = elapsed_ms / args.steps
     step_flops = _counted_step_flops(w)
-    value = step_flops * world / (ms_per_step * 1e-3) / 1e12
+    value = aggregate_tflops(step_flops, world, ms_per_step)
 
     # end to end: pinned host inputs -> device, step, results -> pinned host, every step
     e2e = None
@@ -309,12 +327,8 @@ def run_ours(args):
             e2e_step()
         e1.record(stream)
         barrier()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": step_flops * world / (e2e_ms / args.steps * 1e-3) / 1e12, "unit": UNIT,
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+        e2e = {"value": aggregate_tflops(step_flops, world, e2e_ms / args.steps), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
     peaks = _peaks()
