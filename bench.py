@@ -338,7 +338,9 @@ def run_ours(args):
         bound, work, unit = _kernel_work(name, w, es)
         avg_s = ms / n * 1e-3
         if bound == "tensor":
-            peak = peaks["bf16_sustained"]
+            # burst: the larger (stricter) measured figure; the step is far shorter than the
+            # seconds-long loop the sustained figure comes from (reported beside it)
+            peak = peaks["bf16"]
             achieved = work / avg_s / 1e12
         elif bound == "alu":
             # fp32 FMA pipes: 148 SMs x 128 lanes x 2 FLOP x max SM clock
@@ -349,8 +351,10 @@ def run_ours(args):
             achieved = work / avg_s / 1e9
         roofline = {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak,
                     "unit": unit, "frac": achieved / peak, "traffic": _traffic(name),
-                    "peak_source": peaks["source"] + (" sustained bf16" if bound == "tensor"
-                                                      else ""),
+                    "peak_source": peaks["source"] + (" burst bf16 (cuBLAS 8192^3)"
+                                                      if bound == "tensor" else ""),
+                    "frac_of_sustained": (achieved / peaks["bf16_sustained"]
+                                          if bound == "tensor" else None),
                     "launches": n, "avg_ms": ms / n,
                     "kernels": {k_: {"launches": n_, "total_ms": t_} for k_, (n_, t_) in
                                 prof.items()}}

@@ -116,7 +116,7 @@ S2_API s2_status s2attn_fwd_noalloc(const void* q, const void* k, const void* v,
                                     int causal, float pi_scale, float rope_base, int dtype,
                                     void* cuda_stream);
 
-/* Which kernel family s2attn_fwd launches for these arguments:
+/* Which kernel family s2attn_fwd and s2attn_bwd launch for these arguments:
  * 1 = tcgen05 tensor-core kernels (bf16, d == 128, G % 256 == 0),
  * 0 = CUDA-core kernels (any other valid shape, and every fp32 call), -1 = invalid. */
 S2_API int s2attn_kernel_path(int B, int N, int H_q, int H_kv, int d, int G, int causal, int dtype);
@@ -125,6 +125,14 @@ S2_API int s2attn_kernel_path(int B, int N, int H_q, int H_kv, int d, int G, int
  * used by the last call on it: S2_OK, or S2_ERR_DEVICE_TIMEOUT if a bounded wait in a
  * kernel expired (that kernel's outputs are then undefined). S2_ERR_CUDA on a CUDA error. */
 S2_API s2_status s2attn_device_status(void* workspace, size_t ws_bytes, void* cuda_stream);
+
+/* Self-test of the device-side failure path: enqueues one tiny kernel whose bounded wait
+ * on an mbarrier (which nothing ever arrives on) expires after 50 ms and records the
+ * timeout in the workspace's status word, exactly as an expired wait in the attention
+ * kernels does. Afterwards s2attn_device_status() must report S2_ERR_DEVICE_TIMEOUT and
+ * the CUDA context stays usable. Needs only the first 256 bytes of a workspace. */
+S2_API s2_status s2attn_selftest_wait_timeout(void* workspace, size_t ws_bytes,
+                                              void* cuda_stream);
 
 /* Static, NUL-terminated description of a status code. */
 S2_API const char* s2attn_status_string(int status);

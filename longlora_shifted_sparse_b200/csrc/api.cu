@@ -264,8 +264,14 @@ s2_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o,
   if (e == cudaSuccess)
     e = timed_launch(kBwdRowsum, s, [&] { return launch_bwd_rowsum(p, bf16, s); });
   if (e != cudaSuccess) return to_status(e);
-  e = timed_launch(kBwdDkdvSimt, s, [&] { return launch_simt_dkdv(p, bf16, s); });
-  if (e == cudaSuccess) e = timed_launch(kBwdDqSimt, s, [&] { return launch_simt_dq(p, bf16, s); });
+  if (tc_path(d, G, dtype)) {
+    e = timed_launch(kBwdDkdvTc, s, [&] { return launch_tc_bwd_dkdv(p, s); });
+    if (e == cudaSuccess) e = timed_launch(kBwdDqTc, s, [&] { return launch_tc_bwd_dq(p, s); });
+  } else {
+    e = timed_launch(kBwdDkdvSimt, s, [&] { return launch_simt_dkdv(p, bf16, s); });
+    if (e == cudaSuccess)
+      e = timed_launch(kBwdDqSimt, s, [&] { return launch_simt_dq(p, bf16, s); });
+  }
   return to_status(e);
 }
 
@@ -283,6 +289,15 @@ s2_status s2attn_device_status(void* workspace, size_t ws_bytes, void* cuda_stre
     return S2_ERR_DEVICE_TIMEOUT;
   }
   return S2_OK;
+}
+
+s2_status s2attn_selftest_wait_timeout(void* workspace, size_t ws_bytes, void* cuda_stream) {
+  if (!workspace) return S2_ERR_NULL;
+  if (ws_bytes < kAlign) return S2_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return S2_ERR_ALIGN;
+  return to_status(launch_wait_timeout_selftest(static_cast<unsigned*>(workspace),
+                                                50ull * 1000 * 1000,
+                                                static_cast<cudaStream_t>(cuda_stream)));
 }
 
 const char* s2attn_status_string(int status) {

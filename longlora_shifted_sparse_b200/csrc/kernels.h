@@ -16,4 +16,7 @@ cudaError_t launch_bwd_rowsum(const Params& p, bool bf16, cudaStream_t st);
 cudaError_t launch_simt_dq(const Params& p, bool bf16, cudaStream_t st);
 cudaError_t launch_simt_dkdv(const Params& p, bool bf16, cudaStream_t st);
 
+// Failure-path self-test: a bounded wait that must expire and set *status.
+cudaError_t launch_wait_timeout_selftest(unsigned* status, uint64_t limit_ns, cudaStream_t st);
+
 }  // namespace s2

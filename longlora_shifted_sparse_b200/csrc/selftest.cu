@@ -1,0 +1,36 @@
+// Self-test of the device-side failure path: one CTA waits on an mbarrier that nothing
+// ever arrives on. The bounded wait (the same code every tcgen05 kernel uses) must give up
+// after `limit_ns`, record the timeout in the status word and return, leaving the CUDA
+// context usable. No trap, no fault, no unbounded spin.
+#include "common.cuh"
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace s2 {
+namespace {
+
+using namespace sm100;
+
+__global__ void __launch_bounds__(32, 1) wait_timeout_kernel(unsigned* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_addr(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  Abort ab{&abort_flag, status};
+  mbar_wait(smem_addr(&bar), 0, ab, limit_ns);  // nothing arrives: expires by design
+}
+
+}  // namespace
+
+cudaError_t launch_wait_timeout_selftest(unsigned* status, uint64_t limit_ns, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), st);
+  if (e != cudaSuccess) return e;
+  wait_timeout_kernel<<<1, 32, 0, st>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace s2

@@ -63,7 +63,8 @@ struct Abort {
 // status word), then gives up at its next check.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-__device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, Abort ab) {
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, Abort ab,
+                                                   uint64_t limit_ns) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 0;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -73,7 +74,7 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, Abort
         *ab.flag = 1;
         return false;
       }
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         atomicOr(ab.status, 1u);
         *ab.flag = 1;
         __threadfence_block();
@@ -83,9 +84,10 @@ __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, Abort
   }
 }
 
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, Abort ab) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, Abort ab,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, ab);
+  return mbar_wait_slow(bar, parity, ab, limit_ns);
 }
 
 // ------------------------------------------------------------------------------ TMA

@@ -1,25 +1,29 @@
 // S2-Attn forward on the 5th-generation tensor cores (tcgen05, TMEM accumulators, TMA).
 //
-// Work item = one 128-row query tile of one (batch, query head, group): rolled rows
-// g*G + qt*128 ... + 127. A shifted head's rolled row r is token (r + G/2) mod N, and
-// because G/2 is a multiple of 128 a tile never straddles the wrap, so the -G/2 roll of q,
-// k, v and the +G/2 roll back of o are just the row coordinate of each TMA load / store
-// ("LongLoRA and Shifted Sparse Attention (S^2-Attn)", definition; "LongLoRA: Efficient
-// 100k Context LLM Fine-Tuning Guide", Implementation, Step 1). Inside the group the
-// query tile attends to key tiles 0..qt (causal: tiles above the diagonal are skipped and
-// the diagonal tile is masked on group-local positions).
+// Work item = two consecutive 128-row query tiles (A = 2p, B = 2p+1) of one (batch, query
+// head, group): rolled rows g*G + 256p ... + 255. A shifted head's rolled row r is token
+// (r + G/2) mod N, and because G/2 is a multiple of 128 a tile never straddles the wrap,
+// so the -G/2 roll of q, k, v and the +G/2 roll back of o are just the row coordinate of
+// each TMA load / store ("LongLoRA and Shifted Sparse Attention (S^2-Attn)", definition;
+// "LongLoRA: Efficient 100k Context LLM Fine-Tuning Guide", Implementation, Step 1).
+// Inside the group each query tile attends to key tiles 0..its own index (causal: tiles
+// above the diagonal are skipped, the diagonal tile is masked on group-local positions).
 //
-// Roles (192 threads):
-//   warp 0      TMA producer: Q once, then K_j and V_j into two 2-stage rings.
-//   warp 1      MMA issuer (one thread) and TMEM owner: S_j = Q K_j^T into one of two
-//               TMEM score buffers, then O += P_{j-1} V_{j-1} with P read from TMEM.
-//   warps 2..5  softmax: thread = query row = TMEM lane. Reads its S row, keeps the
-//               running max / sum in fp32 (exp2 domain, log2(e)/sqrt(d) folded into one
-//               scale), writes P as bf16 over the S buffer it came from, and rescales
-//               the O accumulator in TMEM only when the running max grows by more than
-//               2^8 (the stale max keeps every P <= 256). Epilogue: O / l -> bf16 at the
-//               token's original row, LSE = ln 2 * (m + log2 l).
-// TMEM: S0 [0,128), S1 [128,256), O [256,384) of a 512-column allocation.
+// Roles (384 threads):
+//   warp 0       TMA producer: Q_A and Q_B once, then K_j, V_j into two 2-stage rings
+//                (each K/V tile serves both query tiles).
+//   warp 1       MMA issuer (one thread) and TMEM owner. Order per key tile j:
+//                PV_A(j-1), QK_A(j), PV_B(j-1), QK_B(j): while the tensor cores work on
+//                one tile, the other tile's softmax runs (ping-pong).
+//   warps 4..7   softmax of tile A; warps 8..11 softmax of tile B. Thread = query row =
+//                TMEM lane. Pass 1 reads the row of S and takes its max; pass 2 reads it
+//                again and writes P = exp2(S log2(e)/sqrt(d) - m) as bf16 over S. The O
+//                accumulator (TMEM) is rescaled only when the running max grows by more
+//                than 2^8; the stale max keeps every P <= 256 and l uses the same max.
+//                When S_t(j) has landed, PV_t(j-1) has completed (commit order), so the
+//                rescale needs no extra wait. Epilogue: O / l -> bf16 at the token's
+//                original row, LSE = ln 2 * (m + log2 l).
+// TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
 // Every wait is bounded; on expiry the CTA records it in the status word and drains.
 #include "common.cuh"
 #include "sm100.cuh"
@@ -35,23 +39,21 @@ constexpr int kD = 128;
 constexpr int kTile = 128;
 constexpr uint32_t kTileBytes = kTile * kD * 2;    // 32 KB: 128 rows x 128 bf16
 constexpr uint32_t kHalfBytes = kTileBytes / 2;    // one 128 x 64 TMA box
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
 
-// dynamic shared memory: Q | K0 K1 | V0 V1, each 32 KB, 1024-byte aligned
+// dynamic shared memory: Q_A Q_B | K0 K1 | V0 V1, each 32 KB, 1024-byte aligned
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kTileBytes;
-constexpr uint32_t kOffV = 3 * kTileBytes;
-constexpr uint32_t kSmemBytes = 5 * kTileBytes + 1024;
+constexpr uint32_t kOffK = 2 * kTileBytes;
+constexpr uint32_t kOffV = 4 * kTileBytes;
+constexpr uint32_t kSmemBytes = 6 * kTileBytes + 1024;
 
 struct FwdBarriers {
   uint64_t q_full;
   uint64_t k_full[2], k_empty[2];
   uint64_t v_full[2], v_empty[2];
-  uint64_t s_full[2], p_full[2];
-  uint64_t o_done;
+  uint64_t s_full[2], p_full[2], o_final[2];  // index: query tile A = 0, B = 1
   uint64_t drain;
 };
 
@@ -83,15 +85,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.G / kTile, ng = p.N / p.G;
-  const int per_qt = p.B * p.Hq * ng;
-  const int qt = T - 1 - (int)(blockIdx.x / per_qt);  // heaviest query tiles first
-  const int rest = (int)(blockIdx.x % per_qt);
+  const int per_pair = p.B * p.Hq * ng;
+  const int pr = T / 2 - 1 - (int)(blockIdx.x / per_pair);  // heaviest pairs first
+  const int rest = (int)(blockIdx.x % per_pair);
   const int g = rest % ng, bh = rest / ng;
   const int h = bh % p.Hq, b = bh / p.Hq;
   const int kvh = h / (p.Hq / p.Hkv);
   const bool sh = head_shifted(h, p.Hq);
-  const int nkv = p.causal ? qt + 1 : T;
-  const int r0 = g * p.G + qt * kTile;  // rolled row of the tile's first query
+  const int qt0 = 2 * pr;                                  // tile A; tile B = qt0 + 1
+  const int nA = p.causal ? qt0 + 1 : T;                   // key tiles of tile A
+  const int nB = p.causal ? qt0 + 2 : T;                   // key tiles of tile B (>= nA)
+  const int r0 = g * p.G + qt0 * kTile;                    // rolled row of tile A's row 0
 
   Abort ab{&abort_flag, p.status};
   if (threadIdx.x == 0) {
@@ -105,8 +109,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_addr(&bars.v_empty[s]), 1);
       mbar_init(smem_addr(&bars.s_full[s]), 1);
       mbar_init(smem_addr(&bars.p_full[s]), 128);
+      mbar_init(smem_addr(&bars.o_final[s]), 1);
     }
-    mbar_init(smem_addr(&bars.o_done), 1);
     mbar_init(smem_addr(&bars.drain), 1);
     fence_barrier_init();
   }
@@ -126,12 +130,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      const int qrow = (b * p.Hq + h) * p.N + src_row(r0, sh, p.G, p.N);
-      mbar_arrive_expect_tx(smem_addr(&bars.q_full), kTileBytes);
-      tma_load_2d(sQ, &tm_q, smem_addr(&bars.q_full), 0, qrow);
-      tma_load_2d(sQ + kHalfBytes, &tm_q, smem_addr(&bars.q_full), 64, qrow);
+      const uint32_t qb = smem_addr(&bars.q_full);
+      mbar_arrive_expect_tx(qb, 2 * kTileBytes);
+      for (int t = 0; t < 2; t++) {
+        const int qrow = (b * p.Hq + h) * p.N + src_row(r0 + t * kTile, sh, p.G, p.N);
+        tma_load_2d(sQ + t * kTileBytes, &tm_q, qb, 0, qrow);
+        tma_load_2d(sQ + t * kTileBytes + kHalfBytes, &tm_q, qb, 64, qrow);
+      }
       int issued = 0;
-      for (int j = 0; j < nkv; j++) {
+      for (int j = 0; j < nB; j++) {
         const int s = j & 1;
         const uint32_t ph = (j >> 1) & 1;
         const int mk = src_row(g * p.G + j * kTile, sh, p.G, p.N);
@@ -160,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = (j >> 1) & 1;
         mbar_wait(smem_addr((t & 1) ? &bars.v_full[s] : &bars.k_full[s]), ph, local);
       }
-      mbar_wait(smem_addr(&bars.q_full), 0, local);
+      mbar_wait(qb, 0, local);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -169,34 +176,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_pv = idesc_bf16_f32(kTile, kD, false, true);
       bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
       tc_fence_after();
-      for (int j = 0; ok && j <= nkv; j++) {
-        if (j < nkv) {
-          const int s = j & 1;
-          const uint32_t ph = (j >> 1) & 1;
-          if (!mbar_wait(smem_addr(&bars.k_full[s]), ph, ab)) break;
-          tc_fence_after();
-          const uint32_t sK = smem_addr(smem + kOffK + s * kTileBytes);
-          const uint32_t dS = tmem + (s ? kColS1 : kColS0);
-#pragma unroll
-          for (int kk = 0; kk < kD / 16; kk++)
-            mma_ss(dS, kmajor_desc(sQ, kk), kmajor_desc(sK, kk), idesc_qk, kk > 0);
-          mma_commit(smem_addr(&bars.s_full[s]));
-          mma_commit(smem_addr(&bars.k_empty[s]));
-        }
+      for (int j = 0; ok && j <= nB; j++) {
+        const int jj = j - 1;
         if (j >= 1) {
-          const int jj = j - 1, s = jj & 1;
-          const uint32_t ph = (jj >> 1) & 1;
-          if (!mbar_wait(smem_addr(&bars.p_full[s]), ph, ab)) break;
-          if (!mbar_wait(smem_addr(&bars.v_full[s]), ph, ab)) break;
-          tc_fence_after();
-          const uint32_t sV = smem_addr(smem + kOffV + s * kTileBytes);
-          const uint32_t aP = tmem + (s ? kColS1 : kColS0);
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; kk++)
-            mma_ts(tmem + kColO, aP + kk * 8, v_desc(sV, kk), idesc_pv, (jj > 0 || kk > 0));
-          mma_commit(smem_addr(&bars.v_empty[s]));
-          mma_commit(smem_addr(&bars.o_done));
+          if (!mbar_wait(smem_addr(&bars.v_full[jj & 1]), (jj >> 1) & 1, ab)) break;
         }
+        if (j < nB) {
+          if (!mbar_wait(smem_addr(&bars.k_full[j & 1]), (j >> 1) & 1, ab)) break;
+        }
+        tc_fence_after();
+        const uint32_t sK = smem_addr(smem + kOffK + (j & 1) * kTileBytes);
+        const uint32_t sV = smem_addr(smem + kOffV + (jj & 1) * kTileBytes);
+#pragma unroll
+        for (int t = 0; t < 2; t++) {
+          const int nt = t ? nB : nA;
+          const uint32_t tS = tmem + t * 128, tO = tmem + 256 + t * 128;
+          if (j >= 1 && jj < nt) {
+            if (!mbar_wait(smem_addr(&bars.p_full[t]), jj & 1, ab)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kTile / 16; kk++)
+              mma_ts(tO, tS + kk * 8, v_desc(sV, kk), idesc_pv, (jj > 0 || kk > 0));
+            if (jj == nt - 1) mma_commit(smem_addr(&bars.o_final[t]));
+          }
+          if (j < nt) {
+            const uint32_t sQt = sQ + t * kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < kD / 16; kk++)
+              mma_ss(tS, kmajor_desc(sQt, kk), kmajor_desc(sK, kk), idesc_qk, kk > 0);
+            mma_commit(smem_addr(&bars.s_full[t]));
+          }
+        }
+        if (!ok) break;
+        if (j >= 1) mma_commit(smem_addr(&bars.v_empty[jj & 1]));
+        if (j < nB) mma_commit(smem_addr(&bars.k_empty[j & 1]));
       }
       // every MMA issued above has completed before TMEM is released
       mma_commit(smem_addr(&bars.drain));
@@ -204,37 +217,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       Abort local{&no_abort, p.status};
       mbar_wait(smem_addr(&bars.drain), 0, local);
     }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------------ softmax / epilogue
+    const int t = (warp - 4) >> 2;  // query tile of this warpgroup
+    const int qt = qt0 + t;
+    const int n = t ? nB : nA;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + 256 + t * 128;
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nkv; j++) {
-      const int s = j & 1;
-      const uint32_t ph = (j >> 1) & 1;
-      ok = mbar_wait(smem_addr(&bars.s_full[s]), ph, ab);
+    for (int j = 0; j < n; j++) {
+      ok = mbar_wait(smem_addr(&bars.s_full[t]), j & 1, ab);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t tS = tmem + lane_off + (s ? kColS1 : kColS0);
-      uint32_t r[4][32];
-#pragma unroll
-      for (int ch = 0; ch < 4; ch++) tmem_ld32(tS + ch * 32, r[ch]);
-      tmem_wait_ld();
       const bool diag = p.causal && j == qt;
-      float mt = -INFINITY;
+      // pass 1: row max of the raw scores
+      float mraw = -INFINITY;
 #pragma unroll
-      for (int ch = 0; ch < 4; ch++)
+      for (int ch = 0; ch < 4; ch++) {
+        uint32_t x[32];
+        tmem_ld32(tS + ch * 32, x);
+        tmem_wait_ld();
+        if (diag) {
 #pragma unroll
-        for (int c = 0; c < 32; c++) {
-          float x = __uint_as_float(r[ch][c]) * sl2;
-          if (diag && ch * 32 + c > row) x = -INFINITY;
-          r[ch][c] = __float_as_uint(x);
-          mt = fmaxf(mt, x);
+          for (int c = 0; c < 32; c++)
+            if (ch * 32 + c <= row) mraw = fmaxf(mraw, __uint_as_float(x[c]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; c++) mraw = fmaxf(mraw, __uint_as_float(x[c]));
         }
+      }
+      const float mt = mraw * sl2;
       float alpha = 1.f;
       bool rescale = false;
       if (mt > m + kRescaleThreshold) {
@@ -242,55 +260,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         rescale = j > 0;
         m = mt;
       }
+      if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+        for (int ch = 0; ch < 4; ch++) {
+          uint32_t o[32];
+          tmem_ld32(tO + ch * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; c++) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          tmem_st32(tO + ch * 32, o);
+        }
+      }
+      // pass 2: P = exp2(S * sl2 - m) as bf16 over the scores already consumed
+      const float nm = -m;
       float rs = 0.f;
 #pragma unroll
       for (int ch = 0; ch < 4; ch++) {
+        uint32_t x[32];
+        tmem_ld32(tS + ch * 32, x);
+        tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
-        for (int t = 0; t < 16; t++) {
-          const float p0 = fast_exp2(__uint_as_float(r[ch][2 * t]) - m);
-          const float p1 = fast_exp2(__uint_as_float(r[ch][2 * t + 1]) - m);
+        for (int c2 = 0; c2 < 16; c2++) {
+          float p0 = fast_exp2(fmaf(__uint_as_float(x[2 * c2]), sl2, nm));
+          float p1 = fast_exp2(fmaf(__uint_as_float(x[2 * c2 + 1]), sl2, nm));
+          if (diag) {
+            if (ch * 32 + 2 * c2 > row) p0 = 0.f;
+            if (ch * 32 + 2 * c2 + 1 > row) p1 = 0.f;
+          }
           rs += p0 + p1;
-          pk[t] = pack_bf16x2(p0, p1);
+          pk[c2] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + ch * 16, pk);
       }
       l = l * alpha + rs;
       tmem_wait_st();
-      if (j > 0) {
-        ok = mbar_wait(smem_addr(&bars.o_done), (j - 1) & 1, ab);
-        __syncwarp();
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
-          const uint32_t tO = tmem + lane_off + kColO;
-#pragma unroll
-          for (int ch = 0; ch < 4; ch++) {
-            uint32_t o[32];
-            tmem_ld32(tO + ch * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int c = 0; c < 32; c++) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(tO + ch * 32, o);
-          }
-          tmem_wait_st();
-        }
-      }
       tc_fence_before();
-      mbar_arrive(smem_addr(&bars.p_full[s]));
+      mbar_arrive(smem_addr(&bars.p_full[t]));
     }
     if (ok) {
-      ok = mbar_wait(smem_addr(&bars.o_done), (nkv - 1) & 1, ab);
+      ok = mbar_wait(smem_addr(&bars.o_final[t]), 0, ab);
       __syncwarp();
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
       tc_fence_after();
-      const int mrow = src_row(r0 + row, sh, p.G, p.N);
+      const int mrow = src_row(r0 + t * kTile + row, sh, p.G, p.N);
       __nv_bfloat16* orow =
           static_cast<__nv_bfloat16*>(p.o) + ((size_t)(b * p.N + mrow) * p.Hq + h) * kD;
       const float inv_l = 1.f / l;
-      const uint32_t tO = tmem + lane_off + kColO;
 #pragma unroll
       for (int ch = 0; ch < 4; ch++) {
         uint32_t o[32];
@@ -299,11 +317,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint4 pk[4];
         uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
-        for (int t = 0; t < 16; t++)
-          pw[t] = pack_bf16x2(__uint_as_float(o[2 * t]) * inv_l, __uint_as_float(o[2 * t + 1]) * inv_l);
+        for (int c2 = 0; c2 < 16; c2++)
+          pw[c2] = pack_bf16x2(__uint_as_float(o[2 * c2]) * inv_l,
+                               __uint_as_float(o[2 * c2 + 1]) * inv_l);
         uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
-        for (int t = 0; t < 4; t++) dst[t] = pk[t];
+        for (int c4 = 0; c4 < 4; c4++) dst[c4] = pk[c4];
       }
       p.lse[((size_t)b * p.Hq + h) * p.N + mrow] = (m + __log2f(l)) * 0.69314718055994531f;
     }
@@ -332,8 +351,8 @@ cudaError_t launch_tc_fwd(const Params& p, cudaStream_t st) {
   if ((e = cudaFuncSetAttribute(tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kSmemBytes)))
     return e;
-  const long tiles = (long)p.B * p.Hq * (p.N / p.G) * (p.G / kTile);
-  tc_fwd_kernel<<<dim3((unsigned)tiles), dim3(kThreads), kSmemBytes, st>>>(p, tq, tk, tv);
+  const long pairs = (long)p.B * p.Hq * (p.N / p.G) * (p.G / kTile / 2);
+  tc_fwd_kernel<<<dim3((unsigned)pairs), dim3(kThreads), kSmemBytes, st>>>(p, tq, tk, tv);
   return cudaGetLastError();
 }
 

@@ -10,5 +10,7 @@
 namespace s2 {
 
 cudaError_t launch_tc_fwd(const Params& p, cudaStream_t st);
+cudaError_t launch_tc_bwd_dkdv(const Params& p, cudaStream_t st);
+cudaError_t launch_tc_bwd_dq(const Params& p, cudaStream_t st);
 
 }  // namespace s2

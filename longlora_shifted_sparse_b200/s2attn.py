@@ -43,6 +43,8 @@ _lib.s2attn_fwd_noalloc.argtypes = [_vp] * 5 + _SHAPE + [_vp]
 _lib.s2attn_fwd_noalloc.restype = _i
 _lib.s2attn_kernel_path.argtypes = [_i] * 8
 _lib.s2attn_kernel_path.restype = _i
+_lib.s2attn_selftest_wait_timeout.argtypes = [_vp, _sz, _vp]
+_lib.s2attn_selftest_wait_timeout.restype = _i
 _lib.s2attn_device_status.argtypes = [_vp, _sz, _vp]
 _lib.s2attn_device_status.restype = _i
 _lib.s2attn_status_string.argtypes = [_i]
@@ -64,6 +66,7 @@ s2attn_bwd = _lib.s2attn_bwd
 s2attn_fwd_noalloc = _lib.s2attn_fwd_noalloc
 s2attn_kernel_path = _lib.s2attn_kernel_path
 s2attn_device_status = _lib.s2attn_device_status
+s2attn_selftest_wait_timeout = _lib.s2attn_selftest_wait_timeout
 s2attn_profile_enable = _lib.s2attn_profile_enable
 s2attn_profile_num_kernels = _lib.s2attn_profile_num_kernels
 s2attn_profile_dropped = _lib.s2attn_profile_dropped

@@ -105,6 +105,9 @@ def test_bwd_rejects_bad_arguments(lib, kw, code):
 def test_device_status_rejects_null(lib):
     assert lib.s2attn_device_status(None, 4096, None) == lib.S2_ERR_NULL
     assert lib.s2attn_device_status(P, 8, None) == lib.S2_ERR_WORKSPACE
+    assert lib.s2attn_selftest_wait_timeout(None, 4096, None) == lib.S2_ERR_NULL
+    assert lib.s2attn_selftest_wait_timeout(P, 8, None) == lib.S2_ERR_WORKSPACE
+    assert lib.s2attn_selftest_wait_timeout(P + 4, 4096, None) == lib.S2_ERR_ALIGN
 
 
 def test_profiler_host_side(lib):

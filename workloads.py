@@ -35,6 +35,8 @@ WORKLOADS = {
         Workload("llama2_7b_32k", 1, 32768, 32, 32, 128, 8192, 8.0, "bf16", 0.5, True, 2),
         Workload("llama2_7b_100k", 1, 102400, 32, 32, 128, 25600, 25.0, "bf16", 0.5, True, 3),
         Workload("llama2_70b_gqa_32k", 1, 32768, 64, 8, 128, 8192, 8.0, "bf16", 0.5, True, 4),
+        # a smaller case of the same shape family for ncu captures (q is 134 MB > L2)
+        Workload("llama2_7b_16k", 1, 16384, 32, 32, 128, 4096, 4.0, "bf16", 0.5, True, 5),
     ]
 }
 
