@@ -10,22 +10,29 @@
 // rotated back, dq = R(phi)^T dq~, dk = R(phi)^T dk~ ("LoRA for Long-Context Adaptation",
 // RoPE and position-interpolation sections), using the workspace's (cos, sin) table.
 //
-// dK/dV pass: one CTA per 128-row key tile (b, kv head, group, kt), heaviest tiles first.
-//   For every query head of the kv head and every query tile it >= kt (causal):
-//     S^T  = K Q^T      (SS MMA, TMEM cols [0,128))      thread = key row = TMEM lane
-//     dP^T = V dO^T     (SS MMA, TMEM cols [128,256))
-//     P^T  = exp2(S^T log2(e)/sqrt(d) - LSE_i log2(e)), written as bf16 over S^T
-//     dS^T = P^T * (dP^T - D_i), written as bf16 over dP^T
-//     dV  += P^T dO     (TS MMA, TMEM cols [256,384))
-//     dK  += dS^T Q     (TS MMA, TMEM cols [384,512))
-//   The GQA sum over query heads happens in the TMEM accumulators (no atomics).
+// Both passes walk the other side of the group in 64-row half tiles u = 0, 1, 2, ... with
+// two TMEM score buffers, so the tensor cores compute half u+1 while the per-row math of
+// half u runs. MMA issue order per half: scores of u+1, then the gradient MMAs of u.
+//
+// dK/dV pass: one CTA per 128-row key tile (b, kv head, group, kt). For every query head of
+// the kv head and every query tile it >= kt (causal), in two 64-row halves:
+//     S^T  = K Q_h^T     (SS MMA, N = 64)             thread = key row = TMEM lane
+//     dP^T = V dO_h^T    (SS MMA, N = 64)
+//     P^T  = exp2(S^T log2(e)/sqrt(d) - LSE_i log2(e)) -> bf16 over S^T
+//     dS^T = P^T * (dP^T - D_i)                        -> bf16 over dP^T
+//     dV  += P^T dO_h    (TS MMA, K = 64)
+//     dK  += dS^T Q_h    (TS MMA, K = 64)
+//   TMEM: S^T_0 [0,64) dP^T_0 [64,128) S^T_1 [128,192) dP^T_1 [192,256) dV [256,384)
+//   dK [384,512). The GQA sum over query heads happens in the TMEM accumulators.
 //   Epilogue: dk = R^T (dK / sqrt(d)), dv = dV, bf16, at the key tokens' original rows.
-// dQ pass: one CTA per 128-row query tile (b, head, group, qt), heaviest first.
-//   For every key tile j <= qt: S = Q K^T, dP = dO V^T (SS MMAs), dS = P * (dP - D) written
-//   as bf16 over S (thread = query row), dQ += dS K (TS MMA).
+// dQ pass: one CTA per 128-row query tile (b, head, group, qt). For every key tile j <= qt,
+//   in two 64-row halves: S = Q K_h^T, dP = dO V_h^T (SS MMAs, N = 64); dS = P (dP - D)
+//   -> bf16 over S (thread = query row); dQ += dS K_h (TS MMA, K = 64).
+//   TMEM: S_0 [0,64) dP_0 [64,128) S_1 [128,192) dP_1 [192,256) dQ [256,384).
 //   Epilogue: dq = R^T (dQ / sqrt(d)), bf16, at the query tokens' original rows.
-// Roles as in the forward: warp 0 TMA producer, warp 1 MMA issuer and TMEM owner, warps
-// 2..5 the per-row math. Every wait is bounded (see sm100.cuh).
+// CTAs are launched head-group-major so that the CTAs running together share the tiles
+// they stream (L2 reuse). Roles as in the forward: warp 0 TMA producer, warp 1 MMA issuer
+// and TMEM owner, warps 2..5 the per-row math. Every wait is bounded (see sm100.cuh).
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tc_kernels.h"
@@ -38,8 +45,9 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kTile = 128;
+constexpr int kHalf = 64;                          // rows per half tile
 constexpr uint32_t kTileBytes = kTile * kD * 2;
-constexpr uint32_t kHalfBytes = kTileBytes / 2;
+constexpr uint32_t kBoxBytes = kTileBytes / 2;     // one 128-row x 64-column TMA box
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -50,13 +58,16 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_saddr, int kk) {
-  return smem_desc_sw128(tile_saddr + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
+// K-major operand starting at row `row0` (multiple of 8) of a 128 x 128 tile, k-step kk.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_saddr, int kk, int row0 = 0) {
+  return smem_desc_sw128(tile_saddr + (kk >> 2) * kBoxBytes + (kk & 3) * 32 + row0 * 128, 16,
+                         1024);
 }
 
-// tile as an MN-major B operand: k-step kk covers tile rows 16kk..16kk+15, N = d.
-__device__ __forceinline__ uint64_t mn_desc(uint32_t tile_saddr, int kk) {
-  return smem_desc_sw128(tile_saddr + kk * 2048, kHalfBytes, 1024);
+// Tile rows as an MN-major B operand (K = rows, N = d): k-step kk covers rows
+// row0 + 16kk .. row0 + 16kk + 15.
+__device__ __forceinline__ uint64_t mn_desc(uint32_t tile_saddr, int kk, int row0 = 0) {
+  return smem_desc_sw128(tile_saddr + (row0 + kk * 16) * 128, kBoxBytes, 1024);
 }
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
@@ -101,7 +112,8 @@ constexpr uint32_t kKVSmem = 6 * kTileBytes + 2048 + 1024;
 struct DkdvBarriers {
   uint64_t kv_full;
   uint64_t q_full[2], q_empty[2];
-  uint64_t sdp_full, p_ready, ds_ready, acc_done, drain;
+  uint64_t sdp_full[2], p_ready[2], ds_ready[2];
+  uint64_t acc_done, drain;
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -117,15 +129,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.G / kTile, ng = p.N / p.G, R = p.Hq / p.Hkv;
-  const int per_kt = p.B * p.Hkv * ng;
-  const int kt = (int)(blockIdx.x / per_kt);  // kt = 0 has the most query tiles
-  const int rest = (int)(blockIdx.x % per_kt);
-  const int g = rest % ng, bk = rest / ng;
+  // head-group-major: the key tiles of one (b, kv head, group) run together, heaviest first
+  const int kt = (int)(blockIdx.x % T);
+  const int bkg = (int)(blockIdx.x / T);
+  const int g = bkg % ng, bk = bkg / ng;
   const int kvh = bk % p.Hkv, b = bk / p.Hkv;
   const bool sh = head_shifted(kvh, p.Hkv);
   const int it0 = p.causal ? kt : 0;
   const int nq = T - it0;         // query tiles per query head
-  const int npairs = R * nq;      // (query head, query tile) pairs
+  const int ntiles = R * nq;      // (query head, query tile) pairs
+  const int nsteps = 2 * ntiles;  // 64-row halves
   const int mk0 = src_row(g * p.G + kt * kTile, sh, p.G, p.N);
 
   Abort ab{&abort_flag, p.status};
@@ -135,10 +148,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; s++) {
       mbar_init(smem_addr(&bars.q_full[s]), 1);
       mbar_init(smem_addr(&bars.q_empty[s]), 1);
+      mbar_init(smem_addr(&bars.sdp_full[s]), 1);
+      mbar_init(smem_addr(&bars.p_ready[s]), 128);
+      mbar_init(smem_addr(&bars.ds_ready[s]), 128);
     }
-    mbar_init(smem_addr(&bars.sdp_full), 1);
-    mbar_init(smem_addr(&bars.p_ready), 128);
-    mbar_init(smem_addr(&bars.ds_ready), 128);
     mbar_init(smem_addr(&bars.acc_done), 1);
     mbar_init(smem_addr(&bars.drain), 1);
     fence_barrier_init();
@@ -148,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t colST = 0, colDPT = 128, colDV = 256, colDK = 384;
+  const uint32_t colDV = 256, colDK = 384;
   const uint32_t sK = smem_addr(smem + kKVOffK), sV = smem_addr(smem + kKVOffV);
   const bool skip = abort_flag != 0;
 
@@ -164,11 +177,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(kvb, 2 * kTileBytes);
       const int krow = (b * p.Hkv + kvh) * p.N + mk0;
       tma_load_2d(sK, &tm_k, kvb, 0, krow);
-      tma_load_2d(sK + kHalfBytes, &tm_k, kvb, 64, krow);
+      tma_load_2d(sK + kBoxBytes, &tm_k, kvb, 64, krow);
       tma_load_3d(sV, &tm_v, kvb, 0, kvh, b * p.N + mk0);
-      tma_load_3d(sV + kHalfBytes, &tm_v, kvb, 64, kvh, b * p.N + mk0);
+      tma_load_3d(sV + kBoxBytes, &tm_v, kvb, 64, kvh, b * p.N + mk0);
       int issued = 0;
-      for (int n = 0; n < npairs; n++) {
+      for (int n = 0; n < ntiles; n++) {
         const int s = n & 1;
         const uint32_t ph = (n >> 1) & 1;
         const int h = kvh * R + n / nq;
@@ -181,9 +194,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(qb, 2 * kTileBytes + 1024);
         const int qrow = (b * p.Hq + h) * p.N + mq0;
         tma_load_2d(sQ, &tm_q, qb, 0, qrow);
-        tma_load_2d(sQ + kHalfBytes, &tm_q, qb, 64, qrow);
+        tma_load_2d(sQ + kBoxBytes, &tm_q, qb, 64, qrow);
         tma_load_3d(sDO, &tm_do, qb, 0, h, b * p.N + mq0);
-        tma_load_3d(sDO + kHalfBytes, &tm_do, qb, 64, h, b * p.N + mq0);
+        tma_load_3d(sDO + kBoxBytes, &tm_do, qb, 64, h, b * p.N + mq0);
         const size_t lrow = ((size_t)b * p.Hq + h) * p.N + mq0;
         bulk_load(smem_addr(smem + kKVOffLse + s * 512), p.lse + lrow, 512, qb);
         bulk_load(smem_addr(smem + kKVOffD + s * 512), p.Dsum + lrow, 512, qb);
@@ -198,35 +211,49 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
+      const uint32_t idesc_s = idesc_bf16_f32(kTile, kHalf, false, false);
       const uint32_t idesc_g = idesc_bf16_f32(kTile, kD, false, true);
       bool ok = mbar_wait(smem_addr(&bars.kv_full), 0, ab);
-      tc_fence_after();
-      for (int n = 0; ok && n < npairs; n++) {
-        const int s = n & 1;
-        const uint32_t ph = (n >> 1) & 1;
-        if (!mbar_wait(smem_addr(&bars.q_full[s]), ph, ab)) break;
+      // scores of half u into buffer u & 1 (waits for its query tile on the first half)
+      auto issue_scores = [&](int u) -> bool {
+        const int n = u >> 1, hf = u & 1, s = n & 1;
+        if (hf == 0 && !mbar_wait(smem_addr(&bars.q_full[s]), (n >> 1) & 1, ab)) return false;
         tc_fence_after();
         const uint32_t sQ = smem_addr(smem + kKVOffStage + s * 2 * kTileBytes);
         const uint32_t sDO = sQ + kTileBytes;
+        const uint32_t cST = (u & 1) * 128, cDPT = cST + 64;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; kk++)
-          mma_ss(tmem + colST, kmajor_desc(sK, kk), kmajor_desc(sQ, kk), idesc_s, kk > 0);
+          mma_ss(tmem + cST, kmajor_desc(sK, kk), kmajor_desc(sQ, kk, hf * kHalf), idesc_s, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; kk++)
-          mma_ss(tmem + colDPT, kmajor_desc(sV, kk), kmajor_desc(sDO, kk), idesc_s, kk > 0);
-        mma_commit(smem_addr(&bars.sdp_full));
-        if (!mbar_wait(smem_addr(&bars.p_ready), n & 1, ab)) break;
+          mma_ss(tmem + cDPT, kmajor_desc(sV, kk), kmajor_desc(sDO, kk, hf * kHalf), idesc_s,
+                 kk > 0);
+        mma_commit(smem_addr(&bars.sdp_full[u & 1]));
+        return true;
+      };
+      tc_fence_after();
+      if (ok && nsteps > 0) ok = issue_scores(0);
+      for (int u = 0; ok && u < nsteps; u++) {
+        if (u + 1 < nsteps && !issue_scores(u + 1)) break;
+        const int n = u >> 1, hf = u & 1, s = n & 1, bb = u & 1;
+        const uint32_t ph = (u >> 1) & 1;
+        const uint32_t sQ = smem_addr(smem + kKVOffStage + s * 2 * kTileBytes);
+        const uint32_t sDO = sQ + kTileBytes;
+        const uint32_t cST = bb * 128, cDPT = cST + 64;
+        if (!mbar_wait(smem_addr(&bars.p_ready[bb]), ph, ab)) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; kk++)
-          mma_ts(tmem + colDV, tmem + colST + kk * 8, mn_desc(sDO, kk), idesc_g, (n > 0 || kk > 0));
-        if (!mbar_wait(smem_addr(&bars.ds_ready), n & 1, ab)) break;
+        for (int kk = 0; kk < kHalf / 16; kk++)
+          mma_ts(tmem + colDV, tmem + cST + kk * 8, mn_desc(sDO, kk, hf * kHalf), idesc_g,
+                 (u > 0 || kk > 0));
+        if (!mbar_wait(smem_addr(&bars.ds_ready[bb]), ph, ab)) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; kk++)
-          mma_ts(tmem + colDK, tmem + colDPT + kk * 8, mn_desc(sQ, kk), idesc_g, (n > 0 || kk > 0));
-        mma_commit(smem_addr(&bars.q_empty[s]));
+        for (int kk = 0; kk < kHalf / 16; kk++)
+          mma_ts(tmem + colDK, tmem + cDPT + kk * 8, mn_desc(sQ, kk, hf * kHalf), idesc_g,
+                 (u > 0 || kk > 0));
+        if (hf == 1) mma_commit(smem_addr(&bars.q_empty[s]));
       }
       mma_commit(smem_addr(&bars.acc_done));
       mma_commit(smem_addr(&bars.drain));
@@ -241,41 +268,42 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float sl2 = p.scale_log2;
     bool ok = true;
-    for (int n = 0; n < npairs; n++) {
-      const int s = n & 1;
+    for (int u = 0; u < nsteps; u++) {
+      const int n = u >> 1, hf = u & 1, s = n & 1, bb = u & 1;
       const int it = it0 + n % nq;
-      ok = mbar_wait(smem_addr(&bars.sdp_full), n & 1, ab);
+      ok = mbar_wait(smem_addr(&bars.sdp_full[bb]), (u >> 1) & 1, ab);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      const float* lse_s = reinterpret_cast<const float*>(smem + kKVOffLse + s * 512);
-      const float* d_s = reinterpret_cast<const float*>(smem + kKVOffD + s * 512);
+      const float* lse_s = reinterpret_cast<const float*>(smem + kKVOffLse + s * 512) + hf * kHalf;
+      const float* d_s = reinterpret_cast<const float*>(smem + kKVOffD + s * 512) + hf * kHalf;
       const bool diag = p.causal && it == kt;
-      float pr[128];
+      const uint32_t tST = tmem + lane_off + bb * 128, tDPT = tST + 64;
+      float pr[kHalf];
 #pragma unroll
-      for (int ch = 0; ch < 4; ch++) {
+      for (int ch = 0; ch < 2; ch++) {
         uint32_t x[32];
-        tmem_ld32(tmem + lane_off + colST + ch * 32, x);
+        tmem_ld32(tST + ch * 32, x);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 32; c++) {
-          const int i = ch * 32 + c;  // query row inside its tile
+          const int i = ch * 32 + c;  // query row inside the half
           float v = fast_exp2(fmaf(__uint_as_float(x[c]), sl2, -lse_s[i] * kLog2e));
-          if (diag && i < row) v = 0.f;
+          if (diag && hf * kHalf + i < row) v = 0.f;
           pr[i] = v;
         }
 #pragma unroll
         for (int t = 0; t < 16; t++) pk[t] = pack_bf16x2(pr[ch * 32 + 2 * t], pr[ch * 32 + 2 * t + 1]);
-        tmem_st16(tmem + lane_off + colST + ch * 16, pk);
+        tmem_st16(tST + ch * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_addr(&bars.p_ready));
+      mbar_arrive(smem_addr(&bars.p_ready[bb]));
 #pragma unroll
-      for (int ch = 0; ch < 4; ch++) {
+      for (int ch = 0; ch < 2; ch++) {
         uint32_t x[32];
-        tmem_ld32(tmem + lane_off + colDPT + ch * 32, x);
+        tmem_ld32(tDPT + ch * 32, x);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
@@ -285,11 +313,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float d1 = pr[i + 1] * (__uint_as_float(x[2 * t + 1]) - d_s[i + 1]);
           pk[t] = pack_bf16x2(d0, d1);
         }
-        tmem_st16(tmem + lane_off + colDPT + ch * 16, pk);
+        tmem_st16(tDPT + ch * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_addr(&bars.ds_ready));
+      mbar_arrive(smem_addr(&bars.ds_ready[bb]));
     }
     if (ok) {
       ok = mbar_wait(smem_addr(&bars.acc_done), 0, ab);
@@ -342,7 +370,8 @@ constexpr uint32_t kQSmem = 6 * kTileBytes + 1024;
 struct DqBarriers {
   uint64_t q_full;
   uint64_t kv_full[2], kv_empty[2];
-  uint64_t sdp_full, ds_ready, acc_done, drain;
+  uint64_t sdp_full[2], ds_ready[2];
+  uint64_t acc_done, drain;
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -357,15 +386,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int T = p.G / kTile, ng = p.N / p.G;
-  const int per_qt = p.B * p.Hq * ng;
-  const int qt = T - 1 - (int)(blockIdx.x / per_qt);
-  const int rest = (int)(blockIdx.x % per_qt);
-  const int g = rest % ng, bh = rest / ng;
-  const int h = bh % p.Hq, b = bh / p.Hq;
-  const int kvh = h / (p.Hq / p.Hkv);
+  const int T = p.G / kTile, ng = p.N / p.G, R = p.Hq / p.Hkv;
+  // head-group-major: the query tiles of all query heads of one (b, kv head, group) run
+  // together (they share K and V), heaviest query tiles first
+  const int per_kg = T * R;
+  const int inner = (int)(blockIdx.x % per_kg);
+  const int bkg = (int)(blockIdx.x / per_kg);
+  const int qt = T - 1 - inner / R;
+  const int g = bkg % ng, bk = bkg / ng;
+  const int kvh = bk % p.Hkv, b = bk / p.Hkv;
+  const int h = kvh * R + inner % R;
   const bool sh = head_shifted(h, p.Hq);
   const int nkv = p.causal ? qt + 1 : T;
+  const int nsteps = 2 * nkv;
   const int mq0 = src_row(g * p.G + qt * kTile, sh, p.G, p.N);
 
   Abort ab{&abort_flag, p.status};
@@ -375,9 +408,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < 2; s++) {
       mbar_init(smem_addr(&bars.kv_full[s]), 1);
       mbar_init(smem_addr(&bars.kv_empty[s]), 1);
+      mbar_init(smem_addr(&bars.sdp_full[s]), 1);
+      mbar_init(smem_addr(&bars.ds_ready[s]), 128);
     }
-    mbar_init(smem_addr(&bars.sdp_full), 1);
-    mbar_init(smem_addr(&bars.ds_ready), 128);
     mbar_init(smem_addr(&bars.acc_done), 1);
     mbar_init(smem_addr(&bars.drain), 1);
     fence_barrier_init();
@@ -387,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t colS = 0, colDP = 128, colDQ = 256;
+  const uint32_t colDQ = 256;
   const uint32_t sQ = smem_addr(smem + kQOffQ), sDO = smem_addr(smem + kQOffDO);
   const bool skip = abort_flag != 0;
 
@@ -402,9 +435,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_arrive_expect_tx(qb, 2 * kTileBytes);
       const int qrow = (b * p.Hq + h) * p.N + mq0;
       tma_load_2d(sQ, &tm_q, qb, 0, qrow);
-      tma_load_2d(sQ + kHalfBytes, &tm_q, qb, 64, qrow);
+      tma_load_2d(sQ + kBoxBytes, &tm_q, qb, 64, qrow);
       tma_load_3d(sDO, &tm_do, qb, 0, h, b * p.N + mq0);
-      tma_load_3d(sDO + kHalfBytes, &tm_do, qb, 64, h, b * p.N + mq0);
+      tma_load_3d(sDO + kBoxBytes, &tm_do, qb, 64, h, b * p.N + mq0);
       int issued = 0;
       for (int j = 0; j < nkv; j++) {
         const int s = j & 1;
@@ -417,9 +450,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(kb, 2 * kTileBytes);
         const int krow = (b * p.Hkv + kvh) * p.N + mk;
         tma_load_2d(sKs, &tm_k, kb, 0, krow);
-        tma_load_2d(sKs + kHalfBytes, &tm_k, kb, 64, krow);
+        tma_load_2d(sKs + kBoxBytes, &tm_k, kb, 64, krow);
         tma_load_3d(sVs, &tm_v, kb, 0, kvh, b * p.N + mk);
-        tma_load_3d(sVs + kHalfBytes, &tm_v, kb, 64, kvh, b * p.N + mk);
+        tma_load_3d(sVs + kBoxBytes, &tm_v, kb, 64, kvh, b * p.N + mk);
         issued = j + 1;
       }
       int no_abort = 0;
@@ -430,30 +463,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
+      const uint32_t idesc_s = idesc_bf16_f32(kTile, kHalf, false, false);
       const uint32_t idesc_g = idesc_bf16_f32(kTile, kD, false, true);
       bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
-      tc_fence_after();
-      for (int j = 0; ok && j < nkv; j++) {
-        const int s = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(smem_addr(&bars.kv_full[s]), ph, ab)) break;
+      auto issue_scores = [&](int u) -> bool {
+        const int j = u >> 1, hf = u & 1, s = j & 1;
+        if (hf == 0 && !mbar_wait(smem_addr(&bars.kv_full[s]), (j >> 1) & 1, ab)) return false;
         tc_fence_after();
         const uint32_t sKs = smem_addr(smem + kQOffStage + s * 2 * kTileBytes);
         const uint32_t sVs = sKs + kTileBytes;
+        const uint32_t cS = (u & 1) * 128, cDP = cS + 64;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; kk++)
-          mma_ss(tmem + colS, kmajor_desc(sQ, kk), kmajor_desc(sKs, kk), idesc_s, kk > 0);
+          mma_ss(tmem + cS, kmajor_desc(sQ, kk), kmajor_desc(sKs, kk, hf * kHalf), idesc_s, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; kk++)
-          mma_ss(tmem + colDP, kmajor_desc(sDO, kk), kmajor_desc(sVs, kk), idesc_s, kk > 0);
-        mma_commit(smem_addr(&bars.sdp_full));
-        if (!mbar_wait(smem_addr(&bars.ds_ready), j & 1, ab)) break;
+          mma_ss(tmem + cDP, kmajor_desc(sDO, kk), kmajor_desc(sVs, kk, hf * kHalf), idesc_s,
+                 kk > 0);
+        mma_commit(smem_addr(&bars.sdp_full[u & 1]));
+        return true;
+      };
+      tc_fence_after();
+      if (ok && nsteps > 0) ok = issue_scores(0);
+      for (int u = 0; ok && u < nsteps; u++) {
+        if (u + 1 < nsteps && !issue_scores(u + 1)) break;
+        const int j = u >> 1, hf = u & 1, s = j & 1, bb = u & 1;
+        const uint32_t sKs = smem_addr(smem + kQOffStage + s * 2 * kTileBytes);
+        if (!mbar_wait(smem_addr(&bars.ds_ready[bb]), (u >> 1) & 1, ab)) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; kk++)
-          mma_ts(tmem + colDQ, tmem + colS + kk * 8, mn_desc(sKs, kk), idesc_g, (j > 0 || kk > 0));
-        mma_commit(smem_addr(&bars.kv_empty[s]));
+        for (int kk = 0; kk < kHalf / 16; kk++)
+          mma_ts(tmem + colDQ, tmem + bb * 128 + kk * 8, mn_desc(sKs, kk, hf * kHalf), idesc_g,
+                 (u > 0 || kk > 0));
+        if (hf == 1) mma_commit(smem_addr(&bars.kv_empty[s]));
       }
       mma_commit(smem_addr(&bars.acc_done));
       mma_commit(smem_addr(&bars.drain));
@@ -471,22 +513,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float Dm = p.Dsum[lrow];
     const float sl2 = p.scale_log2;
     bool ok = true;
-    for (int j = 0; j < nkv; j++) {
-      ok = mbar_wait(smem_addr(&bars.sdp_full), j & 1, ab);
+    for (int u = 0; u < nsteps; u++) {
+      const int j = u >> 1, hf = u & 1, bb = u & 1;
+      ok = mbar_wait(smem_addr(&bars.sdp_full[bb]), (u >> 1) & 1, ab);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       const bool diag = p.causal && j == qt;
+      const uint32_t tS = tmem + lane_off + bb * 128, tDP = tS + 64;
 #pragma unroll
-      for (int ch = 0; ch < 4; ch++) {
+      for (int ch = 0; ch < 2; ch++) {
         uint32_t xs[32], xd[32];
-        tmem_ld32(tmem + lane_off + colS + ch * 32, xs);
-        tmem_ld32(tmem + lane_off + colDP + ch * 32, xd);
+        tmem_ld32(tS + ch * 32, xs);
+        tmem_ld32(tDP + ch * 32, xd);
         tmem_wait_ld();
         uint32_t pk[16];
 #pragma unroll
         for (int t = 0; t < 16; t++) {
-          const int c0 = ch * 32 + 2 * t;  // key column inside its tile
+          const int c0 = hf * kHalf + ch * 32 + 2 * t;  // key column inside its tile
           float p0 = fast_exp2(fmaf(__uint_as_float(xs[2 * t]), sl2, nlse2));
           float p1 = fast_exp2(fmaf(__uint_as_float(xs[2 * t + 1]), sl2, nlse2));
           if (diag && c0 > row) p0 = 0.f;
@@ -494,11 +538,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           pk[t] = pack_bf16x2(p0 * (__uint_as_float(xd[2 * t]) - Dm),
                               p1 * (__uint_as_float(xd[2 * t + 1]) - Dm));
         }
-        tmem_st16(tmem + lane_off + colS + ch * 16, pk);
+        tmem_st16(tS + ch * 16, pk);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_addr(&bars.ds_ready));
+      mbar_arrive(smem_addr(&bars.ds_ready[bb]));
     }
     if (ok) {
       ok = mbar_wait(smem_addr(&bars.acc_done), 0, ab);
