@@ -300,6 +300,12 @@ s2_status s2attn_selftest_wait_timeout(void* workspace, size_t ws_bytes, void* c
                                                 static_cast<cudaStream_t>(cuda_stream)));
 }
 
+s2_status s2attn_selftest_exp2(const float* x, float* y, int n, void* cuda_stream) {
+  if (!x || !y) return S2_ERR_NULL;
+  if (n <= 0) return S2_ERR_ARG;
+  return to_status(launch_exp2_poly_selftest(x, y, n, static_cast<cudaStream_t>(cuda_stream)));
+}
+
 const char* s2attn_status_string(int status) {
   switch (status) {
     case S2_OK: return "ok";

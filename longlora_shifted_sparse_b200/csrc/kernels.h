@@ -19,4 +19,7 @@ cudaError_t launch_simt_dkdv(const Params& p, bool bf16, cudaStream_t st);
 // Failure-path self-test: a bounded wait that must expire and set *status.
 cudaError_t launch_wait_timeout_selftest(unsigned* status, uint64_t limit_ns, cudaStream_t st);
 
+// Elementwise y = 2^x with the FMA-pipe polynomial the softmax uses (for testing it).
+cudaError_t launch_exp2_poly_selftest(const float* x, float* y, int n, cudaStream_t st);
+
 }  // namespace s2

@@ -3,6 +3,7 @@
 // after `limit_ns`, record the timeout in the status word and return, leaving the CUDA
 // context usable. No trap, no fault, no unbounded spin.
 #include "common.cuh"
+#include "fastmath.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -24,7 +25,17 @@ __global__ void __launch_bounds__(32, 1) wait_timeout_kernel(unsigned* status, u
   mbar_wait(smem_addr(&bar), 0, ab, limit_ns);  // nothing arrives: expires by design
 }
 
+__global__ void exp2_poly_kernel(const float* x, float* y, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    y[i] = exp2_poly(x[i]);
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_poly_selftest(const float* x, float* y, int n, cudaStream_t st) {
+  exp2_poly_kernel<<<(n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024, 256, 0, st>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_wait_timeout_selftest(unsigned* status, uint64_t limit_ns, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(unsigned), st);

@@ -10,29 +10,32 @@
 // rotated back, dq = R(phi)^T dq~, dk = R(phi)^T dk~ ("LoRA for Long-Context Adaptation",
 // RoPE and position-interpolation sections), using the workspace's (cos, sin) table.
 //
-// Both passes walk the other side of the group in 64-row half tiles u = 0, 1, 2, ... with
-// two TMEM score buffers, so the tensor cores compute half u+1 while the per-row math of
-// half u runs. MMA issue order per half: scores of u+1, then the gradient MMAs of u.
+// Keeping the tensor cores busy. Per pair of 128-row tiles both passes run three or four
+// 128 x 128 x 128 MMAs and one round of per-row math that depends on two of them. The
+// math warps first load the score tile (S, or S^T) into registers and release it at once,
+// so the next pair's score MMA can run while they compute; they write the bf16 operands
+// of the gradient MMAs (P^T and dS^T, or dS) over the dP tile after loading it. The MMA
+// queue therefore always holds work: gradient MMAs of pair n, dP of pair n+1, scores of
+// pair n+2 (issued last, so it never delays the MMAs the next math phase waits for).
+// Eight math warps share the rows (two per TMEM lane quarter, 64 columns each).
 //
 // dK/dV pass: one CTA per 128-row key tile (b, kv head, group, kt). For every query head of
-// the kv head and every query tile it >= kt (causal), in two 64-row halves:
-//     S^T  = K Q_h^T     (SS MMA, N = 64)             thread = key row = TMEM lane
-//     dP^T = V dO_h^T    (SS MMA, N = 64)
-//     P^T  = exp2(S^T log2(e)/sqrt(d) - LSE_i log2(e)) -> bf16 over S^T
-//     dS^T = P^T * (dP^T - D_i)                        -> bf16 over dP^T
-//     dV  += P^T dO_h    (TS MMA, K = 64)
-//     dK  += dS^T Q_h    (TS MMA, K = 64)
-//   TMEM: S^T_0 [0,64) dP^T_0 [64,128) S^T_1 [128,192) dP^T_1 [192,256) dV [256,384)
-//   dK [384,512). The GQA sum over query heads happens in the TMEM accumulators.
+// the kv head and every query tile it >= kt (causal):
+//     S^T  = K Q^T       (SS MMA)             TMEM [0,128)     thread = key row = lane
+//     dP^T = V dO^T      (SS MMA)             TMEM [128,256)
+//     P^T  = exp2(S^T log2(e)/sqrt(d) - LSE_i log2(e)), dS^T = P^T (dP^T - D_i), both bf16,
+//            written over dP^T: per 32 query rows, P^T in 16 columns and dS^T in the next 16
+//     dV  += P^T dO      (TS MMA)             TMEM [256,384)
+//     dK  += dS^T Q      (TS MMA)             TMEM [384,512)
+//   The GQA sum over query heads happens in the TMEM accumulators (no atomics).
 //   Epilogue: dk = R^T (dK / sqrt(d)), dv = dV, bf16, at the key tokens' original rows.
-// dQ pass: one CTA per 128-row query tile (b, head, group, qt). For every key tile j <= qt,
-//   in two 64-row halves: S = Q K_h^T, dP = dO V_h^T (SS MMAs, N = 64); dS = P (dP - D)
-//   -> bf16 over S (thread = query row); dQ += dS K_h (TS MMA, K = 64).
-//   TMEM: S_0 [0,64) dP_0 [64,128) S_1 [128,192) dP_1 [192,256) dQ [256,384).
+// dQ pass: one CTA per 128-row query tile (b, head, group, qt). For every key tile j <= qt:
+//   S = Q K^T (TMEM [0,128)), dP = dO V^T ([128,256)), dS = P (dP - D) bf16 over dP
+//   (the first 32 of each math warp's 64 columns), dQ += dS K (TS MMA, [256,384)).
 //   Epilogue: dq = R^T (dQ / sqrt(d)), bf16, at the query tokens' original rows.
 // CTAs are launched head-group-major so that the CTAs running together share the tiles
-// they stream (L2 reuse). Roles as in the forward: warp 0 TMA producer, warp 1 MMA issuer
-// and TMEM owner, warps 2..5 the per-row math. Every wait is bounded (see sm100.cuh).
+// they stream (L2 reuse). Roles: warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
+// warps 4..11 the per-row math. Every wait is bounded (see sm100.cuh).
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tc_kernels.h"
@@ -45,10 +48,10 @@ using namespace sm100;
 
 constexpr int kD = 128;
 constexpr int kTile = 128;
-constexpr int kHalf = 64;                          // rows per half tile
 constexpr uint32_t kTileBytes = kTile * kD * 2;
 constexpr uint32_t kBoxBytes = kTileBytes / 2;     // one 128-row x 64-column TMA box
-constexpr int kThreads = 192;
+constexpr int kThreads = 384;
+constexpr int kMathThreads = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -58,25 +61,23 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// K-major operand starting at row `row0` (multiple of 8) of a 128 x 128 tile, k-step kk.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_saddr, int kk, int row0 = 0) {
-  return smem_desc_sw128(tile_saddr + (kk >> 2) * kBoxBytes + (kk & 3) * 32 + row0 * 128, 16,
-                         1024);
+// K-major operand (128 rows x 128 bf16 in two 64-column SW128 boxes), k-step kk.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_saddr, int kk) {
+  return smem_desc_sw128(tile_saddr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
 }
 
-// Tile rows as an MN-major B operand (K = rows, N = d): k-step kk covers rows
-// row0 + 16kk .. row0 + 16kk + 15.
-__device__ __forceinline__ uint64_t mn_desc(uint32_t tile_saddr, int kk, int row0 = 0) {
-  return smem_desc_sw128(tile_saddr + (row0 + kk * 16) * 128, kBoxBytes, 1024);
+// Tile rows as an MN-major B operand (K = rows, N = d): k-step kk covers rows 16kk..16kk+15.
+__device__ __forceinline__ uint64_t mn_desc(uint32_t tile_saddr, int kk) {
+  return smem_desc_sw128(tile_saddr + kk * 2048, kBoxBytes, 1024);
 }
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-          "r"(dst),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-      : "memory");
+// TMEM column of the bf16 A operand for k-step kk (16 K rows = 8 packed columns). Each
+// math warp owns 64 K rows (columns c0 = 0 or 64 of the tile) and writes them chunk by
+// chunk (32 K rows each) into the 32 fp32 columns it has just read:
+//   dQ pass: dS at region + c0 + 16 * chunk .. + 16          -> packed_col(region, kk, 16)
+//   dK/dV:   P^T at region + c0 + 32 * chunk, dS^T 16 later  -> packed_col(region, kk, 32)
+__device__ __forceinline__ uint32_t packed_col(uint32_t region, int kk, int chunk_stride) {
+  return region + (kk >> 2) * 64 + ((kk >> 1) & 1) * chunk_stride + (kk & 1) * 8;
 }
 
 // Rotates a chunk of 32 consecutive fp32 columns (16 channel pairs starting at pair p0)
@@ -99,20 +100,27 @@ __device__ __forceinline__ void scale_pack(const uint32_t (&x)[32], float scale,
     w[t] = pack_bf16x2(__uint_as_float(x[2 * t]) * scale, __uint_as_float(x[2 * t + 1]) * scale);
 }
 
+__device__ __forceinline__ void store_row64(__nv_bfloat16* dst, const uint4 (&a)[4]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int t = 0; t < 4; t++) d4[t] = a[t];
+}
+
 // ================================================================================ dK / dV
 
-// smem: K | V | stage 0: Q, dO | stage 1: Q, dO | LSE[2][128] | D[2][128]
+// smem: K | V | Q stages 0..2 | dO stages 0..1
+constexpr int kQStages = 3, kDOStages = 2;
 constexpr uint32_t kKVOffK = 0;
 constexpr uint32_t kKVOffV = kTileBytes;
-constexpr uint32_t kKVOffStage = 2 * kTileBytes;   // + s * 2 * kTileBytes: Q then dO
-constexpr uint32_t kKVOffLse = 6 * kTileBytes;     // + s * 512
-constexpr uint32_t kKVOffD = 6 * kTileBytes + 1024;
-constexpr uint32_t kKVSmem = 6 * kTileBytes + 2048 + 1024;
+constexpr uint32_t kKVOffQ = 2 * kTileBytes;
+constexpr uint32_t kKVOffDO = (2 + kQStages) * kTileBytes;
+constexpr uint32_t kKVSmem = (2 + kQStages + kDOStages) * kTileBytes + 1024;
 
 struct DkdvBarriers {
   uint64_t kv_full;
-  uint64_t q_full[2], q_empty[2];
-  uint64_t sdp_full[2], p_ready[2], ds_ready[2];
+  uint64_t q_full[kQStages], q_empty[kQStages];
+  uint64_t do_full[kDOStages], do_empty[kDOStages];
+  uint64_t st_full, st_consumed, dpt_full, pds_ready;
   uint64_t acc_done, drain;
 };
 
@@ -136,22 +144,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kvh = bk % p.Hkv, b = bk / p.Hkv;
   const bool sh = head_shifted(kvh, p.Hkv);
   const int it0 = p.causal ? kt : 0;
-  const int nq = T - it0;         // query tiles per query head
-  const int ntiles = R * nq;      // (query head, query tile) pairs
-  const int nsteps = 2 * ntiles;  // 64-row halves
+  const int nq = T - it0;      // query tiles per query head
+  const int np = R * nq;       // (query head, query tile) pairs
   const int mk0 = src_row(g * p.G + kt * kTile, sh, p.G, p.N);
 
   Abort ab{&abort_flag, p.status};
   if (threadIdx.x == 0) {
     abort_flag = *reinterpret_cast<volatile unsigned*>(p.status) != 0u;
     mbar_init(smem_addr(&bars.kv_full), 1);
-    for (int s = 0; s < 2; s++) {
+    for (int s = 0; s < kQStages; s++) {
       mbar_init(smem_addr(&bars.q_full[s]), 1);
       mbar_init(smem_addr(&bars.q_empty[s]), 1);
-      mbar_init(smem_addr(&bars.sdp_full[s]), 1);
-      mbar_init(smem_addr(&bars.p_ready[s]), 128);
-      mbar_init(smem_addr(&bars.ds_ready[s]), 128);
     }
+    for (int s = 0; s < kDOStages; s++) {
+      mbar_init(smem_addr(&bars.do_full[s]), 1);
+      mbar_init(smem_addr(&bars.do_empty[s]), 1);
+    }
+    mbar_init(smem_addr(&bars.st_full), 1);
+    mbar_init(smem_addr(&bars.st_consumed), kMathThreads);
+    mbar_init(smem_addr(&bars.dpt_full), 1);
+    mbar_init(smem_addr(&bars.pds_ready), kMathThreads);
     mbar_init(smem_addr(&bars.acc_done), 1);
     mbar_init(smem_addr(&bars.drain), 1);
     fence_barrier_init();
@@ -161,9 +173,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t colDV = 256, colDK = 384;
+  const uint32_t colST = 0, colDPT = 128, colDV = 256, colDK = 384;
   const uint32_t sK = smem_addr(smem + kKVOffK), sV = smem_addr(smem + kKVOffV);
   const bool skip = abort_flag != 0;
+
+  // pair n -> query head, query tile
+  auto pair_q = [&](int n, int& h, int& mq0) {
+    h = kvh * R + n / nq;
+    mq0 = src_row(g * p.G + (it0 + n % nq) * kTile, sh, p.G, p.N);
+  };
 
   if (skip) {
   } else if (warp == 0) {
@@ -180,80 +198,92 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_2d(sK + kBoxBytes, &tm_k, kvb, 64, krow);
       tma_load_3d(sV, &tm_v, kvb, 0, kvh, b * p.N + mk0);
       tma_load_3d(sV + kBoxBytes, &tm_v, kvb, 64, kvh, b * p.N + mk0);
-      int issued = 0;
-      for (int n = 0; n < ntiles; n++) {
-        const int s = n & 1;
-        const uint32_t ph = (n >> 1) & 1;
-        const int h = kvh * R + n / nq;
-        const int it = it0 + n % nq;
-        const int mq0 = src_row(g * p.G + it * kTile, sh, p.G, p.N);
-        if (!mbar_wait(smem_addr(&bars.q_empty[s]), ph ^ 1, ab)) break;
-        const uint32_t qb = smem_addr(&bars.q_full[s]);
-        const uint32_t sQ = smem_addr(smem + kKVOffStage + s * 2 * kTileBytes);
-        const uint32_t sDO = sQ + kTileBytes;
-        mbar_arrive_expect_tx(qb, 2 * kTileBytes + 1024);
+      int nq_issued = 0, ndo_issued = 0;
+      for (int n = 0; n < np; n++) {
+        int h, mq0;
+        pair_q(n, h, mq0);
+        const int sq = n % kQStages, sd = n % kDOStages;
+        if (!mbar_wait(smem_addr(&bars.q_empty[sq]), ((n / kQStages) & 1) ^ 1, ab)) break;
+        const uint32_t qb = smem_addr(&bars.q_full[sq]);
+        const uint32_t sQ = smem_addr(smem + kKVOffQ + sq * kTileBytes);
+        mbar_arrive_expect_tx(qb, kTileBytes);
         const int qrow = (b * p.Hq + h) * p.N + mq0;
         tma_load_2d(sQ, &tm_q, qb, 0, qrow);
         tma_load_2d(sQ + kBoxBytes, &tm_q, qb, 64, qrow);
-        tma_load_3d(sDO, &tm_do, qb, 0, h, b * p.N + mq0);
-        tma_load_3d(sDO + kBoxBytes, &tm_do, qb, 64, h, b * p.N + mq0);
-        const size_t lrow = ((size_t)b * p.Hq + h) * p.N + mq0;
-        bulk_load(smem_addr(smem + kKVOffLse + s * 512), p.lse + lrow, 512, qb);
-        bulk_load(smem_addr(smem + kKVOffD + s * 512), p.Dsum + lrow, 512, qb);
-        issued = n + 1;
+        nq_issued = n + 1;
+        if (!mbar_wait(smem_addr(&bars.do_empty[sd]), ((n / kDOStages) & 1) ^ 1, ab)) break;
+        const uint32_t db = smem_addr(&bars.do_full[sd]);
+        const uint32_t sDO = smem_addr(smem + kKVOffDO + sd * kTileBytes);
+        mbar_arrive_expect_tx(db, kTileBytes);
+        tma_load_3d(sDO, &tm_do, db, 0, h, b * p.N + mq0);
+        tma_load_3d(sDO + kBoxBytes, &tm_do, db, 64, h, b * p.N + mq0);
+        ndo_issued = n + 1;
       }
       int no_abort = 0;
       Abort local{&no_abort, p.status};
-      for (int n = issued - 1; n >= 0 && n >= issued - 2; n--)
-        mbar_wait(smem_addr(&bars.q_full[n & 1]), (n >> 1) & 1, local);
+      for (int n = nq_issued - 1; n >= 0 && n >= nq_issued - kQStages; n--)
+        mbar_wait(smem_addr(&bars.q_full[n % kQStages]), (n / kQStages) & 1, local);
+      for (int n = ndo_issued - 1; n >= 0 && n >= ndo_issued - kDOStages; n--)
+        mbar_wait(smem_addr(&bars.do_full[n % kDOStages]), (n / kDOStages) & 1, local);
       mbar_wait(kvb, 0, local);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(kTile, kHalf, false, false);
+      const uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
       const uint32_t idesc_g = idesc_bf16_f32(kTile, kD, false, true);
-      bool ok = mbar_wait(smem_addr(&bars.kv_full), 0, ab);
-      // scores of half u into buffer u & 1 (waits for its query tile on the first half)
-      auto issue_scores = [&](int u) -> bool {
-        const int n = u >> 1, hf = u & 1, s = n & 1;
-        if (hf == 0 && !mbar_wait(smem_addr(&bars.q_full[s]), (n >> 1) & 1, ab)) return false;
+      auto issue_st = [&](int n) -> bool {  // S^T(n) = K Q_n^T
+        const int sq = n % kQStages;
+        if (!mbar_wait(smem_addr(&bars.q_full[sq]), (n / kQStages) & 1, ab)) return false;
         tc_fence_after();
-        const uint32_t sQ = smem_addr(smem + kKVOffStage + s * 2 * kTileBytes);
-        const uint32_t sDO = sQ + kTileBytes;
-        const uint32_t cST = (u & 1) * 128, cDPT = cST + 64;
+        const uint32_t sQ = smem_addr(smem + kKVOffQ + sq * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; kk++)
-          mma_ss(tmem + cST, kmajor_desc(sK, kk), kmajor_desc(sQ, kk, hf * kHalf), idesc_s, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; kk++)
-          mma_ss(tmem + cDPT, kmajor_desc(sV, kk), kmajor_desc(sDO, kk, hf * kHalf), idesc_s,
-                 kk > 0);
-        mma_commit(smem_addr(&bars.sdp_full[u & 1]));
+          mma_ss(tmem + colST, kmajor_desc(sK, kk), kmajor_desc(sQ, kk), idesc_s, kk > 0);
+        mma_commit(smem_addr(&bars.st_full));
         return true;
       };
+      auto issue_dpt = [&](int n) -> bool {  // dP^T(n) = V dO_n^T
+        const int sd = n % kDOStages;
+        if (!mbar_wait(smem_addr(&bars.do_full[sd]), (n / kDOStages) & 1, ab)) return false;
+        tc_fence_after();
+        const uint32_t sDO = smem_addr(smem + kKVOffDO + sd * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; kk++)
+          mma_ss(tmem + colDPT, kmajor_desc(sV, kk), kmajor_desc(sDO, kk), idesc_s, kk > 0);
+        mma_commit(smem_addr(&bars.dpt_full));
+        return true;
+      };
+      // issue order: S^T(0) dP^T(0) S^T(1) | dV(0) dK(0) dP^T(1) S^T(2) | dV(1) ...
+      // After the math warps publish P^T, dS^T of pair n the gradient MMAs of n and dP^T of
+      // n+1 go first (the next math phase waits for them); S^T of n+2 then fills the tensor
+      // pipe while the math warps work on pair n+1.
+      bool ok = mbar_wait(smem_addr(&bars.kv_full), 0, ab);
       tc_fence_after();
-      if (ok && nsteps > 0) ok = issue_scores(0);
-      for (int u = 0; ok && u < nsteps; u++) {
-        if (u + 1 < nsteps && !issue_scores(u + 1)) break;
-        const int n = u >> 1, hf = u & 1, s = n & 1, bb = u & 1;
-        const uint32_t ph = (u >> 1) & 1;
-        const uint32_t sQ = smem_addr(smem + kKVOffStage + s * 2 * kTileBytes);
-        const uint32_t sDO = sQ + kTileBytes;
-        const uint32_t cST = bb * 128, cDPT = cST + 64;
-        if (!mbar_wait(smem_addr(&bars.p_ready[bb]), ph, ab)) break;
+      if (ok && np > 0) ok = issue_st(0) && issue_dpt(0);
+      if (ok && np > 1) ok = mbar_wait(smem_addr(&bars.st_consumed), 0, ab) && issue_st(1);
+      for (int n = 0; ok && n < np; n++) {
+        const uint32_t ph = n & 1;
+        if (!mbar_wait(smem_addr(&bars.pds_ready), ph, ab)) break;
         tc_fence_after();
+        const uint32_t sQ = smem_addr(smem + kKVOffQ + (n % kQStages) * kTileBytes);
+        const uint32_t sDO = smem_addr(smem + kKVOffDO + (n % kDOStages) * kTileBytes);
 #pragma unroll
-        for (int kk = 0; kk < kHalf / 16; kk++)
-          mma_ts(tmem + colDV, tmem + cST + kk * 8, mn_desc(sDO, kk, hf * kHalf), idesc_g,
-                 (u > 0 || kk > 0));
-        if (!mbar_wait(smem_addr(&bars.ds_ready[bb]), ph, ab)) break;
-        tc_fence_after();
+        for (int kk = 0; kk < kTile / 16; kk++)
+          mma_ts(tmem + colDV, tmem + packed_col(colDPT, kk, 32), mn_desc(sDO, kk), idesc_g,
+                 (n > 0 || kk > 0));
+        mma_commit(smem_addr(&bars.do_empty[n % kDOStages]));
 #pragma unroll
-        for (int kk = 0; kk < kHalf / 16; kk++)
-          mma_ts(tmem + colDK, tmem + cDPT + kk * 8, mn_desc(sQ, kk, hf * kHalf), idesc_g,
-                 (u > 0 || kk > 0));
-        if (hf == 1) mma_commit(smem_addr(&bars.q_empty[s]));
+        for (int kk = 0; kk < kTile / 16; kk++)
+          mma_ts(tmem + colDK, tmem + packed_col(colDPT + 16, kk, 32), mn_desc(sQ, kk), idesc_g,
+                 (n > 0 || kk > 0));
+        mma_commit(smem_addr(&bars.q_empty[n % kQStages]));
+        if (n + 1 < np && !issue_dpt(n + 1)) break;
+        // S^T(n+2) once the math warps hold S^T(n+1) in registers
+        if (n + 2 < np) {
+          if (!mbar_wait(smem_addr(&bars.st_consumed), (n + 1) & 1, ab)) break;
+          if (!issue_st(n + 2)) break;
+        }
       }
       mma_commit(smem_addr(&bars.acc_done));
       mma_commit(smem_addr(&bars.drain));
@@ -261,63 +291,85 @@ __global__ void __launch_bounds__(kThreads, 1)
       Abort local{&no_abort, p.status};
       mbar_wait(smem_addr(&bars.drain), 0, local);
     }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------------ per key row math
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;  // key row inside the tile
+    const int c0 = ((warp - 4) >> 2) * 64;  // this warp's 64 query columns of the tile
+    const int row = quarter * 32 + lane;    // key row inside the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tST = tmem + lane_off + colST + c0;
+    const uint32_t tDPT = tmem + lane_off + colDPT + c0;
     const float sl2 = p.scale_log2;
+    // LSE and D of this warp's 64 query rows: lane l holds rows c0 + l and c0 + 32 + l;
+    // loaded one pair ahead and broadcast with shuffles
+    auto load_ld = [&](int n, float (&l2)[2], float (&dd)[2]) {
+      int h, mq0;
+      pair_q(n, h, mq0);
+      const size_t base = ((size_t)b * p.Hq + h) * p.N + mq0 + c0 + lane;
+      l2[0] = -__ldg(p.lse + base) * kLog2e;
+      l2[1] = -__ldg(p.lse + base + 32) * kLog2e;
+      dd[0] = __ldg(p.Dsum + base);
+      dd[1] = __ldg(p.Dsum + base + 32);
+    };
+    float nl2[2], dsum[2], nl2_next[2] = {0.f, 0.f}, dsum_next[2] = {0.f, 0.f};
+    if (np > 0) load_ld(0, nl2, dsum);
     bool ok = true;
-    for (int u = 0; u < nsteps; u++) {
-      const int n = u >> 1, hf = u & 1, s = n & 1, bb = u & 1;
+    for (int n = 0; n < np; n++) {
+      if (n + 1 < np) load_ld(n + 1, nl2_next, dsum_next);
       const int it = it0 + n % nq;
-      ok = mbar_wait(smem_addr(&bars.sdp_full[bb]), (u >> 1) & 1, ab);
+      const bool diag = p.causal && it == kt;
+      ok = mbar_wait(smem_addr(&bars.st_full), n & 1, ab);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
-      const float* lse_s = reinterpret_cast<const float*>(smem + kKVOffLse + s * 512) + hf * kHalf;
-      const float* d_s = reinterpret_cast<const float*>(smem + kKVOffD + s * 512) + hf * kHalf;
-      const bool diag = p.causal && it == kt;
-      const uint32_t tST = tmem + lane_off + bb * 128, tDPT = tST + 64;
-      float pr[kHalf];
-#pragma unroll
-      for (int ch = 0; ch < 2; ch++) {
-        uint32_t x[32];
-        tmem_ld32(tST + ch * 32, x);
+      float pr[64];
+      {
+        uint32_t x0[32], x1[32];
+        tmem_ld32(tST, x0);
+        tmem_ld32(tST + 32, x1);
         tmem_wait_ld();
-        uint32_t pk[16];
+        tc_fence_before();
+        mbar_arrive(smem_addr(&bars.st_consumed));  // S^T may now be overwritten
 #pragma unroll
-        for (int c = 0; c < 32; c++) {
-          const int i = ch * 32 + c;  // query row inside the half
-          float v = fast_exp2(fmaf(__uint_as_float(x[c]), sl2, -lse_s[i] * kLog2e));
-          if (diag && hf * kHalf + i < row) v = 0.f;
-          pr[i] = v;
+        for (int c = 0; c < 64; c++) {
+          const float l = __shfl_sync(0xffffffffu, nl2[c >> 5], c & 31);
+          const float st = __uint_as_float(c < 32 ? x0[c] : x1[c - 32]);
+          float v = fast_exp2(fmaf(st, sl2, l));
+          if (diag && c0 + c < row) v = 0.f;  // query row c0+c before key row: masked
+          pr[c] = v;
         }
+      }
+      ok = mbar_wait(smem_addr(&bars.dpt_full), n & 1, ab);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      {
+        uint32_t x0[32], x1[32];
+        tmem_ld32(tDPT, x0);
+        tmem_ld32(tDPT + 32, x1);
+        tmem_wait_ld();
 #pragma unroll
-        for (int t = 0; t < 16; t++) pk[t] = pack_bf16x2(pr[ch * 32 + 2 * t], pr[ch * 32 + 2 * t + 1]);
-        tmem_st16(tST + ch * 16, pk);
+        for (int ch = 0; ch < 2; ch++) {
+          uint32_t pp[16], pd[16];
+#pragma unroll
+          for (int t = 0; t < 16; t++) {
+            const int c = ch * 32 + 2 * t;
+            const float d0 = __shfl_sync(0xffffffffu, dsum[ch], 2 * t);
+            const float d1 = __shfl_sync(0xffffffffu, dsum[ch], 2 * t + 1);
+            const float dp0 = __uint_as_float(ch ? x1[2 * t] : x0[2 * t]);
+            const float dp1 = __uint_as_float(ch ? x1[2 * t + 1] : x0[2 * t + 1]);
+            pp[t] = pack_bf16x2(pr[c], pr[c + 1]);
+            pd[t] = pack_bf16x2(pr[c] * (dp0 - d0), pr[c + 1] * (dp1 - d1));
+          }
+          tmem_st16(tDPT + ch * 32, pp);       // P^T of these 32 query rows
+          tmem_st16(tDPT + ch * 32 + 16, pd);  // dS^T
+        }
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_addr(&bars.p_ready[bb]));
-#pragma unroll
-      for (int ch = 0; ch < 2; ch++) {
-        uint32_t x[32];
-        tmem_ld32(tDPT + ch * 32, x);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int t = 0; t < 16; t++) {
-          const int i = ch * 32 + 2 * t;
-          const float d0 = pr[i] * (__uint_as_float(x[2 * t]) - d_s[i]);
-          const float d1 = pr[i + 1] * (__uint_as_float(x[2 * t + 1]) - d_s[i + 1]);
-          pk[t] = pack_bf16x2(d0, d1);
-        }
-        tmem_st16(tDPT + ch * 16, pk);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(smem_addr(&bars.ds_ready[bb]));
+      mbar_arrive(smem_addr(&bars.pds_ready));
+      nl2[0] = nl2_next[0]; nl2[1] = nl2_next[1];
+      dsum[0] = dsum_next[0]; dsum[1] = dsum_next[1];
     }
     if (ok) {
       ok = mbar_wait(smem_addr(&bars.acc_done), 0, ab);
@@ -327,26 +379,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       tc_fence_after();
       const int m = src_row(g * p.G + kt * kTile + row, sh, p.G, p.N);
-      const size_t off = ((size_t)(b * p.N + m) * p.Hkv + kvh) * kD;
-      __nv_bfloat16* dk = static_cast<__nv_bfloat16*>(p.dk) + off;
-      __nv_bfloat16* dv = static_cast<__nv_bfloat16*>(p.dv) + off;
+      const size_t off = ((size_t)(b * p.N + m) * p.Hkv + kvh) * kD + c0;
       const float2* cs_row = p.cs + (size_t)m * (kD / 2);
 #pragma unroll
-      for (int ch = 0; ch < 4; ch++) {
+      for (int ch = 0; ch < 2; ch++) {
         uint32_t x[32];
         uint4 o[4];
-        tmem_ld32(tmem + lane_off + colDK + ch * 32, x);
+        tmem_ld32(tmem + lane_off + colDK + c0 + ch * 32, x);
         tmem_wait_ld();
-        unrotate_pack(x, cs_row, ch * 16, p.scale, o);
-        uint4* dst = reinterpret_cast<uint4*>(dk + ch * 32);
-#pragma unroll
-        for (int t = 0; t < 4; t++) dst[t] = o[t];
-        tmem_ld32(tmem + lane_off + colDV + ch * 32, x);
+        unrotate_pack(x, cs_row, (c0 + ch * 32) / 2, p.scale, o);
+        store_row64(static_cast<__nv_bfloat16*>(p.dk) + off + ch * 32, o);
+        tmem_ld32(tmem + lane_off + colDV + c0 + ch * 32, x);
         tmem_wait_ld();
         scale_pack(x, 1.f, o);
-        dst = reinterpret_cast<uint4*>(dv + ch * 32);
-#pragma unroll
-        for (int t = 0; t < 4; t++) dst[t] = o[t];
+        store_row64(static_cast<__nv_bfloat16*>(p.dv) + off + ch * 32, o);
       }
     }
   }
@@ -361,16 +407,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ================================================================================ dQ
 
-// smem: Q | dO | stage 0: K, V | stage 1: K, V
+// smem: Q | dO | K stages 0..2 | V stages 0..1
+constexpr int kKStages = 3, kVStages = 2;
 constexpr uint32_t kQOffQ = 0;
 constexpr uint32_t kQOffDO = kTileBytes;
-constexpr uint32_t kQOffStage = 2 * kTileBytes;  // + s * 2 * kTileBytes: K then V
-constexpr uint32_t kQSmem = 6 * kTileBytes + 1024;
+constexpr uint32_t kQOffK = 2 * kTileBytes;
+constexpr uint32_t kQOffV = (2 + kKStages) * kTileBytes;
+constexpr uint32_t kQSmem = (2 + kKStages + kVStages) * kTileBytes + 1024;
 
 struct DqBarriers {
   uint64_t q_full;
-  uint64_t kv_full[2], kv_empty[2];
-  uint64_t sdp_full[2], ds_ready[2];
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full, s_consumed, dp_full, ds_ready;
   uint64_t acc_done, drain;
 };
 
@@ -398,19 +447,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int h = kvh * R + inner % R;
   const bool sh = head_shifted(h, p.Hq);
   const int nkv = p.causal ? qt + 1 : T;
-  const int nsteps = 2 * nkv;
   const int mq0 = src_row(g * p.G + qt * kTile, sh, p.G, p.N);
 
   Abort ab{&abort_flag, p.status};
   if (threadIdx.x == 0) {
     abort_flag = *reinterpret_cast<volatile unsigned*>(p.status) != 0u;
     mbar_init(smem_addr(&bars.q_full), 1);
-    for (int s = 0; s < 2; s++) {
-      mbar_init(smem_addr(&bars.kv_full[s]), 1);
-      mbar_init(smem_addr(&bars.kv_empty[s]), 1);
-      mbar_init(smem_addr(&bars.sdp_full[s]), 1);
-      mbar_init(smem_addr(&bars.ds_ready[s]), 128);
+    for (int s = 0; s < kKStages; s++) {
+      mbar_init(smem_addr(&bars.k_full[s]), 1);
+      mbar_init(smem_addr(&bars.k_empty[s]), 1);
     }
+    for (int s = 0; s < kVStages; s++) {
+      mbar_init(smem_addr(&bars.v_full[s]), 1);
+      mbar_init(smem_addr(&bars.v_empty[s]), 1);
+    }
+    mbar_init(smem_addr(&bars.s_full), 1);
+    mbar_init(smem_addr(&bars.s_consumed), kMathThreads);
+    mbar_init(smem_addr(&bars.dp_full), 1);
+    mbar_init(smem_addr(&bars.ds_ready), kMathThreads);
     mbar_init(smem_addr(&bars.acc_done), 1);
     mbar_init(smem_addr(&bars.drain), 1);
     fence_barrier_init();
@@ -420,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t colDQ = 256;
+  const uint32_t colS = 0, colDP = 128, colDQ = 256;
   const uint32_t sQ = smem_addr(smem + kQOffQ), sDO = smem_addr(smem + kQOffDO);
   const bool skip = abort_flag != 0;
 
@@ -438,64 +492,82 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_2d(sQ + kBoxBytes, &tm_q, qb, 64, qrow);
       tma_load_3d(sDO, &tm_do, qb, 0, h, b * p.N + mq0);
       tma_load_3d(sDO + kBoxBytes, &tm_do, qb, 64, h, b * p.N + mq0);
-      int issued = 0;
+      int nk_issued = 0, nv_issued = 0;
       for (int j = 0; j < nkv; j++) {
-        const int s = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
         const int mk = src_row(g * p.G + j * kTile, sh, p.G, p.N);
-        if (!mbar_wait(smem_addr(&bars.kv_empty[s]), ph ^ 1, ab)) break;
-        const uint32_t kb = smem_addr(&bars.kv_full[s]);
-        const uint32_t sKs = smem_addr(smem + kQOffStage + s * 2 * kTileBytes);
-        const uint32_t sVs = sKs + kTileBytes;
-        mbar_arrive_expect_tx(kb, 2 * kTileBytes);
         const int krow = (b * p.Hkv + kvh) * p.N + mk;
+        const int sk = j % kKStages, sv = j % kVStages;
+        if (!mbar_wait(smem_addr(&bars.k_empty[sk]), ((j / kKStages) & 1) ^ 1, ab)) break;
+        const uint32_t kb = smem_addr(&bars.k_full[sk]);
+        const uint32_t sKs = smem_addr(smem + kQOffK + sk * kTileBytes);
+        mbar_arrive_expect_tx(kb, kTileBytes);
         tma_load_2d(sKs, &tm_k, kb, 0, krow);
         tma_load_2d(sKs + kBoxBytes, &tm_k, kb, 64, krow);
-        tma_load_3d(sVs, &tm_v, kb, 0, kvh, b * p.N + mk);
-        tma_load_3d(sVs + kBoxBytes, &tm_v, kb, 64, kvh, b * p.N + mk);
-        issued = j + 1;
+        nk_issued = j + 1;
+        if (!mbar_wait(smem_addr(&bars.v_empty[sv]), ((j / kVStages) & 1) ^ 1, ab)) break;
+        const uint32_t vb = smem_addr(&bars.v_full[sv]);
+        const uint32_t sVs = smem_addr(smem + kQOffV + sv * kTileBytes);
+        mbar_arrive_expect_tx(vb, kTileBytes);
+        tma_load_3d(sVs, &tm_v, vb, 0, kvh, b * p.N + mk);
+        tma_load_3d(sVs + kBoxBytes, &tm_v, vb, 64, kvh, b * p.N + mk);
+        nv_issued = j + 1;
       }
       int no_abort = 0;
       Abort local{&no_abort, p.status};
-      for (int j = issued - 1; j >= 0 && j >= issued - 2; j--)
-        mbar_wait(smem_addr(&bars.kv_full[j & 1]), (j >> 1) & 1, local);
+      for (int j = nk_issued - 1; j >= 0 && j >= nk_issued - kKStages; j--)
+        mbar_wait(smem_addr(&bars.k_full[j % kKStages]), (j / kKStages) & 1, local);
+      for (int j = nv_issued - 1; j >= 0 && j >= nv_issued - kVStages; j--)
+        mbar_wait(smem_addr(&bars.v_full[j % kVStages]), (j / kVStages) & 1, local);
       mbar_wait(qb, 0, local);
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(kTile, kHalf, false, false);
+      const uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
       const uint32_t idesc_g = idesc_bf16_f32(kTile, kD, false, true);
-      bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
-      auto issue_scores = [&](int u) -> bool {
-        const int j = u >> 1, hf = u & 1, s = j & 1;
-        if (hf == 0 && !mbar_wait(smem_addr(&bars.kv_full[s]), (j >> 1) & 1, ab)) return false;
+      auto issue_s = [&](int j) -> bool {  // S(j) = Q K_j^T
+        const int sk = j % kKStages;
+        if (!mbar_wait(smem_addr(&bars.k_full[sk]), (j / kKStages) & 1, ab)) return false;
         tc_fence_after();
-        const uint32_t sKs = smem_addr(smem + kQOffStage + s * 2 * kTileBytes);
-        const uint32_t sVs = sKs + kTileBytes;
-        const uint32_t cS = (u & 1) * 128, cDP = cS + 64;
+        const uint32_t sKs = smem_addr(smem + kQOffK + sk * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; kk++)
-          mma_ss(tmem + cS, kmajor_desc(sQ, kk), kmajor_desc(sKs, kk, hf * kHalf), idesc_s, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; kk++)
-          mma_ss(tmem + cDP, kmajor_desc(sDO, kk), kmajor_desc(sVs, kk, hf * kHalf), idesc_s,
-                 kk > 0);
-        mma_commit(smem_addr(&bars.sdp_full[u & 1]));
+          mma_ss(tmem + colS, kmajor_desc(sQ, kk), kmajor_desc(sKs, kk), idesc_s, kk > 0);
+        mma_commit(smem_addr(&bars.s_full));
         return true;
       };
-      tc_fence_after();
-      if (ok && nsteps > 0) ok = issue_scores(0);
-      for (int u = 0; ok && u < nsteps; u++) {
-        if (u + 1 < nsteps && !issue_scores(u + 1)) break;
-        const int j = u >> 1, hf = u & 1, s = j & 1, bb = u & 1;
-        const uint32_t sKs = smem_addr(smem + kQOffStage + s * 2 * kTileBytes);
-        if (!mbar_wait(smem_addr(&bars.ds_ready[bb]), (u >> 1) & 1, ab)) break;
+      auto issue_dp = [&](int j) -> bool {  // dP(j) = dO V_j^T
+        const int sv = j % kVStages;
+        if (!mbar_wait(smem_addr(&bars.v_full[sv]), (j / kVStages) & 1, ab)) return false;
         tc_fence_after();
+        const uint32_t sVs = smem_addr(smem + kQOffV + sv * kTileBytes);
 #pragma unroll
-        for (int kk = 0; kk < kHalf / 16; kk++)
-          mma_ts(tmem + colDQ, tmem + bb * 128 + kk * 8, mn_desc(sKs, kk, hf * kHalf), idesc_g,
-                 (u > 0 || kk > 0));
-        if (hf == 1) mma_commit(smem_addr(&bars.kv_empty[s]));
+        for (int kk = 0; kk < kD / 16; kk++)
+          mma_ss(tmem + colDP, kmajor_desc(sDO, kk), kmajor_desc(sVs, kk), idesc_s, kk > 0);
+        mma_commit(smem_addr(&bars.dp_full));
+        mma_commit(smem_addr(&bars.v_empty[sv]));
+        return true;
+      };
+      // issue order: S(0) dP(0) S(1) | dQ(0) dP(1) S(2) | dQ(1) dP(2) S(3) | ...
+      // (see the dK/dV pass: the MMAs the next math phase waits for go first)
+      bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
+      tc_fence_after();
+      if (ok) ok = issue_s(0) && issue_dp(0);
+      if (ok && nkv > 1) ok = mbar_wait(smem_addr(&bars.s_consumed), 0, ab) && issue_s(1);
+      for (int j = 0; ok && j < nkv; j++) {
+        const uint32_t ph = j & 1;
+        if (!mbar_wait(smem_addr(&bars.ds_ready), ph, ab)) break;
+        tc_fence_after();
+        const uint32_t sKs = smem_addr(smem + kQOffK + (j % kKStages) * kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; kk++)
+          mma_ts(tmem + colDQ, tmem + packed_col(colDP, kk, 16), mn_desc(sKs, kk), idesc_g,
+                 (j > 0 || kk > 0));
+        mma_commit(smem_addr(&bars.k_empty[j % kKStages]));
+        if (j + 1 < nkv && !issue_dp(j + 1)) break;
+        if (j + 2 < nkv) {
+          if (!mbar_wait(smem_addr(&bars.s_consumed), (j + 1) & 1, ab)) break;
+          if (!issue_s(j + 2)) break;
+        }
       }
       mma_commit(smem_addr(&bars.acc_done));
       mma_commit(smem_addr(&bars.drain));
@@ -503,46 +575,65 @@ __global__ void __launch_bounds__(kThreads, 1)
       Abort local{&no_abort, p.status};
       mbar_wait(smem_addr(&bars.drain), 0, local);
     }
-  } else {
+  } else if (warp >= 4) {
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;  // query row inside the tile
+    const int c0 = ((warp - 4) >> 2) * 64;  // this warp's 64 key columns of the tile
+    const int row = quarter * 32 + lane;    // query row inside the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + colS + c0;
+    const uint32_t tDP = tmem + lane_off + colDP + c0;
     const int m = src_row(g * p.G + qt * kTile + row, sh, p.G, p.N);
     const size_t lrow = ((size_t)b * p.Hq + h) * p.N + m;
     const float nlse2 = -p.lse[lrow] * kLog2e;
     const float Dm = p.Dsum[lrow];
     const float sl2 = p.scale_log2;
     bool ok = true;
-    for (int u = 0; u < nsteps; u++) {
-      const int j = u >> 1, hf = u & 1, bb = u & 1;
-      ok = mbar_wait(smem_addr(&bars.sdp_full[bb]), (u >> 1) & 1, ab);
+    for (int j = 0; j < nkv; j++) {
+      ok = mbar_wait(smem_addr(&bars.s_full), j & 1, ab);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       const bool diag = p.causal && j == qt;
-      const uint32_t tS = tmem + lane_off + bb * 128, tDP = tS + 64;
-#pragma unroll
-      for (int ch = 0; ch < 2; ch++) {
-        uint32_t xs[32], xd[32];
-        tmem_ld32(tS + ch * 32, xs);
-        tmem_ld32(tDP + ch * 32, xd);
+      float pr[64];
+      {
+        uint32_t x0[32], x1[32];
+        tmem_ld32(tS, x0);
+        tmem_ld32(tS + 32, x1);
         tmem_wait_ld();
-        uint32_t pk[16];
+        tc_fence_before();
+        mbar_arrive(smem_addr(&bars.s_consumed));  // S may now be overwritten
 #pragma unroll
-        for (int t = 0; t < 16; t++) {
-          const int c0 = hf * kHalf + ch * 32 + 2 * t;  // key column inside its tile
-          float p0 = fast_exp2(fmaf(__uint_as_float(xs[2 * t]), sl2, nlse2));
-          float p1 = fast_exp2(fmaf(__uint_as_float(xs[2 * t + 1]), sl2, nlse2));
-          if (diag && c0 > row) p0 = 0.f;
-          if (diag && c0 + 1 > row) p1 = 0.f;
-          pk[t] = pack_bf16x2(p0 * (__uint_as_float(xd[2 * t]) - Dm),
-                              p1 * (__uint_as_float(xd[2 * t + 1]) - Dm));
+        for (int c = 0; c < 64; c++) {
+          float v = fast_exp2(fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, nlse2));
+          if (diag && c0 + c > row) v = 0.f;  // key column after the query row: masked
+          pr[c] = v;
         }
-        tmem_st16(tS + ch * 16, pk);
+      }
+      ok = mbar_wait(smem_addr(&bars.dp_full), j & 1, ab);
+      __syncwarp();
+      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+      tc_fence_after();
+      {
+        uint32_t x0[32], x1[32];
+        tmem_ld32(tDP, x0);
+        tmem_ld32(tDP + 32, x1);
+        tmem_wait_ld();
+#pragma unroll
+        for (int ch = 0; ch < 2; ch++) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int t = 0; t < 16; t++) {
+            const int c = ch * 32 + 2 * t;
+            const float dp0 = __uint_as_float(ch ? x1[2 * t] : x0[2 * t]);
+            const float dp1 = __uint_as_float(ch ? x1[2 * t + 1] : x0[2 * t + 1]);
+            pk[t] = pack_bf16x2(pr[c] * (dp0 - Dm), pr[c + 1] * (dp1 - Dm));
+          }
+          tmem_st16(tDP + ch * 16, pk);  // dS of these 64 key columns, over dP already read
+        }
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_addr(&bars.ds_ready[bb]));
+      mbar_arrive(smem_addr(&bars.ds_ready));
     }
     if (ok) {
       ok = mbar_wait(smem_addr(&bars.acc_done), 0, ab);
@@ -551,18 +642,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(p.dq) + ((size_t)(b * p.N + m) * p.Hq + h) * kD;
+      __nv_bfloat16* dq =
+          static_cast<__nv_bfloat16*>(p.dq) + ((size_t)(b * p.N + m) * p.Hq + h) * kD + c0;
       const float2* cs_row = p.cs + (size_t)m * (kD / 2);
 #pragma unroll
-      for (int ch = 0; ch < 4; ch++) {
+      for (int ch = 0; ch < 2; ch++) {
         uint32_t x[32];
         uint4 o[4];
-        tmem_ld32(tmem + lane_off + colDQ + ch * 32, x);
+        tmem_ld32(tmem + lane_off + colDQ + c0 + ch * 32, x);
         tmem_wait_ld();
-        unrotate_pack(x, cs_row, ch * 16, p.scale, o);
-        uint4* dst = reinterpret_cast<uint4*>(dq + ch * 32);
-#pragma unroll
-        for (int t = 0; t < 4; t++) dst[t] = o[t];
+        unrotate_pack(x, cs_row, (c0 + ch * 32) / 2, p.scale, o);
+        store_row64(dq + ch * 32, o);
       }
     }
   }

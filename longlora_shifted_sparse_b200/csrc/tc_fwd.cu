@@ -24,8 +24,11 @@
 //                rescale needs no extra wait. Epilogue: O / l -> bf16 at the token's
 //                original row, LSE = ln 2 * (m + log2 l).
 // TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
+// CTAs are launched head-group-major (all tile pairs of the query heads that share one kv
+// head and group, heaviest first), so concurrently running CTAs reuse K and V from L2.
 // Every wait is bounded; on expiry the CTA records it in the status word and drains.
 #include "common.cuh"
+#include "fastmath.cuh"
 #include "sm100.cuh"
 #include "tc_kernels.h"
 #include "tma_host.h"
@@ -42,6 +45,17 @@ constexpr uint32_t kHalfBytes = kTileBytes / 2;    // one 128 x 64 TMA box
 constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
+
+// Column pairs (bit c2 of a 16-bit mask, per 32-column chunk) whose exponentials go to the
+// FMA-pipe exp2 instead of the MUFU unit. At d = 128 the MUFU needs as many cycles per key
+// tile as the tensor cores, but with two softmax warps per scheduler the softmax is bound
+// by instruction latency, not by the MUFU: on a B200 moving 25% / 37.5% / 50% of the
+// exponentials to the FMA pipe slowed the 32k forward from 2.32 ms to 2.52 / 2.84 / 3.10 ms.
+// So every exponential stays on the MUFU unless a build overrides this mask.
+#ifndef S2_FWD_POLY_MASK
+#define S2_FWD_POLY_MASK 0x0000u
+#endif
+constexpr unsigned kPolyMask = S2_FWD_POLY_MASK;
 
 // dynamic shared memory: Q_A Q_B | K0 K1 | V0 V1, each 32 KB, 1024-byte aligned
 constexpr uint32_t kOffQ = 0;
@@ -84,13 +98,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int T = p.G / kTile, ng = p.N / p.G;
-  const int per_pair = p.B * p.Hq * ng;
-  const int pr = T / 2 - 1 - (int)(blockIdx.x / per_pair);  // heaviest pairs first
-  const int rest = (int)(blockIdx.x % per_pair);
-  const int g = rest % ng, bh = rest / ng;
-  const int h = bh % p.Hq, b = bh / p.Hq;
-  const int kvh = h / (p.Hq / p.Hkv);
+  const int T = p.G / kTile, ng = p.N / p.G, R = p.Hq / p.Hkv;
+  // head-group-major: the tile pairs of all query heads of one (b, kv head, group) run
+  // together (they stream the same K and V through L2), heaviest pairs first
+  const int per_kg = (T / 2) * R;
+  const int inner = (int)(blockIdx.x % per_kg);
+  const int bkg = (int)(blockIdx.x / per_kg);
+  const int pr = T / 2 - 1 - inner / R;
+  const int g = bkg % ng, bk = bkg / ng;
+  const int kvh = bk % p.Hkv, b = bk / p.Hkv;
+  const int h = kvh * R + inner % R;
   const bool sh = head_shifted(h, p.Hq);
   const int qt0 = 2 * pr;                                  // tile A; tile B = qt0 + 1
   const int nA = p.causal ? qt0 + 1 : T;                   // key tiles of tile A
@@ -282,8 +299,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int c2 = 0; c2 < 16; c2++) {
-          float p0 = fast_exp2(fmaf(__uint_as_float(x[2 * c2]), sl2, nm));
-          float p1 = fast_exp2(fmaf(__uint_as_float(x[2 * c2 + 1]), sl2, nm));
+          const float a0 = fmaf(__uint_as_float(x[2 * c2]), sl2, nm);
+          const float a1 = fmaf(__uint_as_float(x[2 * c2 + 1]), sl2, nm);
+          float p0, p1;
+          if ((kPolyMask >> c2) & 1u) {
+            p0 = exp2_poly(a0);
+            p1 = exp2_poly(a1);
+          } else {
+            p0 = fast_exp2(a0);
+            p1 = fast_exp2(a1);
+          }
           if (diag) {
             if (ch * 32 + 2 * c2 > row) p0 = 0.f;
             if (ch * 32 + 2 * c2 + 1 > row) p1 = 0.f;

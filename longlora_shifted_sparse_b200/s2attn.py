@@ -45,6 +45,8 @@ _lib.s2attn_kernel_path.argtypes = [_i] * 8
 _lib.s2attn_kernel_path.restype = _i
 _lib.s2attn_selftest_wait_timeout.argtypes = [_vp, _sz, _vp]
 _lib.s2attn_selftest_wait_timeout.restype = _i
+_lib.s2attn_selftest_exp2.argtypes = [_vp, _vp, _i, _vp]
+_lib.s2attn_selftest_exp2.restype = _i
 _lib.s2attn_device_status.argtypes = [_vp, _sz, _vp]
 _lib.s2attn_device_status.restype = _i
 _lib.s2attn_status_string.argtypes = [_i]
@@ -67,6 +69,7 @@ s2attn_fwd_noalloc = _lib.s2attn_fwd_noalloc
 s2attn_kernel_path = _lib.s2attn_kernel_path
 s2attn_device_status = _lib.s2attn_device_status
 s2attn_selftest_wait_timeout = _lib.s2attn_selftest_wait_timeout
+s2attn_selftest_exp2 = _lib.s2attn_selftest_exp2
 s2attn_profile_enable = _lib.s2attn_profile_enable
 s2attn_profile_num_kernels = _lib.s2attn_profile_num_kernels
 s2attn_profile_dropped = _lib.s2attn_profile_dropped

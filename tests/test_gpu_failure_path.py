@@ -32,3 +32,18 @@ def test_expired_wait_is_reported_and_context_survives(s2):
     o, lse = s2.forward(tq, tk, tv, w.G, w.pi_scale, ws=ws)
     assert s2.device_status(ws) == s2.S2_OK
     assert bool(torch.isfinite(o).all()) and bool(torch.isfinite(lse).all())
+
+
+def test_fma_pipe_exp2_matches_exp2(s2):
+    """The polynomial exp2 that takes part of the softmax's exponentials off the MUFU unit
+    agrees with exp2 to a relative 1e-4 over the range the softmax feeds it."""
+    x = np.concatenate([np.linspace(-125.0, 8.0, 200001), np.arange(-125, 9, dtype=np.float64),
+                        np.arange(-125, 9) + 0.5]).astype(np.float32)
+    tx = torch.from_numpy(x).cuda()
+    ty = torch.empty_like(tx)
+    assert s2.s2attn_selftest_exp2(tx.data_ptr(), ty.data_ptr(), tx.numel(),
+                                   torch.cuda.current_stream().cuda_stream) == s2.S2_OK
+    torch.cuda.synchronize()
+    ref = np.exp2(x.astype(np.float64))
+    rel = np.abs(ty.cpu().numpy().astype(np.float64) - ref) / ref
+    assert rel.max() < 1e-4, rel.max()
