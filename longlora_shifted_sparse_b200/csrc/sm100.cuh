@@ -63,6 +63,10 @@ struct Abort {
 // status word), then gives up at its next check.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// kRegion gives each register budget of a kernel that splits its registers (setmaxnreg) its
+// own copy of the out-of-line slow path: a function called from two budgets cannot be
+// allocated for both.
+template <int kRegion = 0>
 static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, Abort ab,
                                                    uint64_t limit_ns) {
   const uint64_t t0 = global_timer_ns();
@@ -84,10 +88,11 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity
   }
 }
 
+template <int kRegion = 0>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, Abort ab,
                                           uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow(bar, parity, ab, limit_ns);
+  return mbar_wait_slow<kRegion>(bar, parity, ab, limit_ns);
 }
 
 // ------------------------------------------------------------------------------ TMA
@@ -184,6 +189,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
+// Warp-collective TMEM load of 16 consecutive 32-bit columns per lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -244,6 +260,23 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   d |= (uint64_t)1u << 46;  // version
   d |= (uint64_t)2u << 61;  // swizzle: 128B
   return d;
+}
+
+// Named barrier over `nthreads` threads (whole warps) that also returns the AND of `pred`
+// across them, so every participant takes the same branch afterwards.
+__device__ __forceinline__ bool named_bar_and(uint32_t id, uint32_t nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

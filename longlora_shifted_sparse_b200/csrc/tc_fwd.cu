@@ -9,20 +9,25 @@
 // Inside the group each query tile attends to key tiles 0..its own index (causal: tiles
 // above the diagonal are skipped, the diagonal tile is masked on group-local positions).
 //
-// Roles (384 threads):
+// Roles (640 threads, five warpgroups):
 //   warp 0       TMA producer: Q_A and Q_B once, then K_j, V_j into two 2-stage rings
 //                (each K/V tile serves both query tiles).
 //   warp 1       MMA issuer (one thread) and TMEM owner. Order per key tile j:
 //                PV_A(j-1), QK_A(j), PV_B(j-1), QK_B(j): while the tensor cores work on
 //                one tile, the other tile's softmax runs (ping-pong).
-//   warps 4..7   softmax of tile A; warps 8..11 softmax of tile B. Thread = query row =
-//                TMEM lane. Pass 1 reads the row of S and takes its max; pass 2 reads it
-//                again and writes P = exp2(S log2(e)/sqrt(d) - m) as bf16 over S. The O
-//                accumulator (TMEM) is rescaled only when the running max grows by more
-//                than 2^8; the stale max keeps every P <= 256 and l uses the same max.
-//                When S_t(j) has landed, PV_t(j-1) has completed (commit order), so the
-//                rescale needs no extra wait. Epilogue: O / l -> bf16 at the token's
-//                original row, LSE = ln 2 * (m + log2 l).
+//   warps 2, 3   idle (they complete warpgroup 0, whose registers go to the softmax).
+//   warps 4..11  softmax of tile A; warps 12..19 softmax of tile B. A query row (= TMEM
+//                lane) is shared by two warps, one per 64-column half of S: each loads its
+//                half once, takes the partial max, swaps it with its partner through shared
+//                memory (a 64-thread named barrier), and writes P = exp2(S log2(e)/sqrt(d)
+//                - m) as bf16 over the first 32 columns of its half. Four softmax warps per
+//                scheduler hide the TMEM-load and MUFU latencies that bound a one-warp-per-
+//                row softmax. The O accumulator (TMEM) is rescaled only when the running max
+//                grows by more than 2^8; the stale max keeps every P <= 256 and l uses the
+//                same max. When S_t(j) has landed, PV_t(j-1) has completed (commit order),
+//                so the rescale needs no extra wait. Epilogue: each half stores its 64
+//                columns of O / l (l = sum of both partial sums) as bf16 at the token's
+//                original row; LSE = ln 2 * (m + log2 l).
 // TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
 // CTAs are launched head-group-major (all tile pairs of the query heads that share one kv
 // head and group, heaviest first), so concurrently running CTAs reuse K and V from L2.
@@ -42,7 +47,16 @@ constexpr int kD = 128;
 constexpr int kTile = 128;
 constexpr uint32_t kTileBytes = kTile * kD * 2;    // 32 KB: 128 rows x 128 bf16
 constexpr uint32_t kHalfBytes = kTileBytes / 2;    // one 128 x 64 TMA box
-constexpr int kThreads = 384;
+// 20 warps: TMA, MMA, two idle, 16 softmax warps. Five warps share one scheduler's 64K-byte
+// register file, so a launch hands each thread 96 registers. Warpgroup 0 then drops to
+// kRegsOther and the four softmax warpgroups rise to kRegsSoftmax (setmaxnreg), enough to
+// hold their 64 scores per row without spilling. The split must fit the launch allocation
+// (an increase beyond it would wait forever), which the launcher checks before every launch.
+constexpr int kThreads = 640;
+constexpr int kRegsOther = 64, kRegsSoftmax = 104;
+static_assert(128 * kRegsOther + (kThreads - 128) * kRegsSoftmax <= kThreads * 96,
+              "register split exceeds the launch allocation");
+constexpr int kSoftmaxThreadsPerTile = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
 
@@ -96,6 +110,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ FwdBarriers bars;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
+  // row-max exchange between the two warps that share a row: [parity][tile][half][row]
+  __shared__ float xmax[2][2][2][kTile];
+  __shared__ float xsum[2][kTile];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.G / kTile, ng = p.N / p.G, R = p.Hq / p.Hkv;
@@ -125,7 +142,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_addr(&bars.v_full[s]), 1);
       mbar_init(smem_addr(&bars.v_empty[s]), 1);
       mbar_init(smem_addr(&bars.s_full[s]), 1);
-      mbar_init(smem_addr(&bars.p_full[s]), 128);
+      mbar_init(smem_addr(&bars.p_full[s]), kSoftmaxThreadsPerTile);
       mbar_init(smem_addr(&bars.o_final[s]), 1);
     }
     mbar_init(smem_addr(&bars.drain), 1);
@@ -139,217 +156,239 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sQ = smem_addr(smem + kOffQ);
   const bool skip = abort_flag != 0;
 
-  if (skip) {
-    // fall through to the teardown
-  } else if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      const uint32_t qb = smem_addr(&bars.q_full);
-      mbar_arrive_expect_tx(qb, 2 * kTileBytes);
-      for (int t = 0; t < 2; t++) {
-        const int qrow = (b * p.Hq + h) * p.N + src_row(r0 + t * kTile, sh, p.G, p.N);
-        tma_load_2d(sQ + t * kTileBytes, &tm_q, qb, 0, qrow);
-        tma_load_2d(sQ + t * kTileBytes + kHalfBytes, &tm_q, qb, 64, qrow);
-      }
-      int issued = 0;
-      for (int j = 0; j < nB; j++) {
-        const int s = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        const int mk = src_row(g * p.G + j * kTile, sh, p.G, p.N);
-        if (!mbar_wait(smem_addr(&bars.k_empty[s]), ph ^ 1, ab)) break;
-        const uint32_t sK = smem_addr(smem + kOffK + s * kTileBytes);
-        mbar_arrive_expect_tx(smem_addr(&bars.k_full[s]), kTileBytes);
-        tma_load_2d(sK, &tm_k, smem_addr(&bars.k_full[s]), 0, (b * p.Hkv + kvh) * p.N + mk);
-        tma_load_2d(sK + kHalfBytes, &tm_k, smem_addr(&bars.k_full[s]), 64,
-                    (b * p.Hkv + kvh) * p.N + mk);
-        if (!mbar_wait(smem_addr(&bars.v_empty[s]), ph ^ 1, ab)) {
-          issued = 2 * j + 1;
-          break;
-        }
-        const uint32_t sV = smem_addr(smem + kOffV + s * kTileBytes);
-        mbar_arrive_expect_tx(smem_addr(&bars.v_full[s]), kTileBytes);
-        tma_load_3d(sV, &tm_v, smem_addr(&bars.v_full[s]), 0, kvh, b * p.N + mk);
-        tma_load_3d(sV + kHalfBytes, &tm_v, smem_addr(&bars.v_full[s]), 64, kvh, b * p.N + mk);
-        issued = 2 * j + 2;
-      }
-      // Let the last loads in flight land before the CTA can exit. This wait ignores the
-      // abort flag (it is set on this path) but keeps its own time limit.
-      int no_abort = 0;
-      Abort local{&no_abort, p.status};
-      for (int t = issued - 1; t >= 0 && t >= issued - 4; t--) {
-        const int j = t >> 1, s = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        mbar_wait(smem_addr((t & 1) ? &bars.v_full[s] : &bars.k_full[s]), ph, local);
-      }
-      mbar_wait(qb, 0, local);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_qk = idesc_bf16_f32(kTile, kTile, false, false);
-      const uint32_t idesc_pv = idesc_bf16_f32(kTile, kD, false, true);
-      bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
-      tc_fence_after();
-      for (int j = 0; ok && j <= nB; j++) {
-        const int jj = j - 1;
-        if (j >= 1) {
-          if (!mbar_wait(smem_addr(&bars.v_full[jj & 1]), (jj >> 1) & 1, ab)) break;
-        }
-        if (j < nB) {
-          if (!mbar_wait(smem_addr(&bars.k_full[j & 1]), (j >> 1) & 1, ab)) break;
-        }
-        tc_fence_after();
-        const uint32_t sK = smem_addr(smem + kOffK + (j & 1) * kTileBytes);
-        const uint32_t sV = smem_addr(smem + kOffV + (jj & 1) * kTileBytes);
-#pragma unroll
+  if (warp < 4) {
+    // warpgroup 0 (TMA producer, MMA issuer, two idle warps) gives registers away
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+    if (!skip && warp == 0) {
+      // ------------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        const uint32_t qb = smem_addr(&bars.q_full);
+        mbar_arrive_expect_tx(qb, 2 * kTileBytes);
         for (int t = 0; t < 2; t++) {
-          const int nt = t ? nB : nA;
-          const uint32_t tS = tmem + t * 128, tO = tmem + 256 + t * 128;
-          if (j >= 1 && jj < nt) {
-            if (!mbar_wait(smem_addr(&bars.p_full[t]), jj & 1, ab)) { ok = false; break; }
-            tc_fence_after();
-#pragma unroll
-            for (int kk = 0; kk < kTile / 16; kk++)
-              mma_ts(tO, tS + kk * 8, v_desc(sV, kk), idesc_pv, (jj > 0 || kk > 0));
-            if (jj == nt - 1) mma_commit(smem_addr(&bars.o_final[t]));
-          }
-          if (j < nt) {
-            const uint32_t sQt = sQ + t * kTileBytes;
-#pragma unroll
-            for (int kk = 0; kk < kD / 16; kk++)
-              mma_ss(tS, kmajor_desc(sQt, kk), kmajor_desc(sK, kk), idesc_qk, kk > 0);
-            mma_commit(smem_addr(&bars.s_full[t]));
-          }
+          const int qrow = (b * p.Hq + h) * p.N + src_row(r0 + t * kTile, sh, p.G, p.N);
+          tma_load_2d(sQ + t * kTileBytes, &tm_q, qb, 0, qrow);
+          tma_load_2d(sQ + t * kTileBytes + kHalfBytes, &tm_q, qb, 64, qrow);
         }
-        if (!ok) break;
-        if (j >= 1) mma_commit(smem_addr(&bars.v_empty[jj & 1]));
-        if (j < nB) mma_commit(smem_addr(&bars.k_empty[j & 1]));
+        int issued = 0;
+        for (int j = 0; j < nB; j++) {
+          const int s = j & 1;
+          const uint32_t ph = (j >> 1) & 1;
+          const int mk = src_row(g * p.G + j * kTile, sh, p.G, p.N);
+          if (!mbar_wait(smem_addr(&bars.k_empty[s]), ph ^ 1, ab)) break;
+          const uint32_t sK = smem_addr(smem + kOffK + s * kTileBytes);
+          mbar_arrive_expect_tx(smem_addr(&bars.k_full[s]), kTileBytes);
+          tma_load_2d(sK, &tm_k, smem_addr(&bars.k_full[s]), 0, (b * p.Hkv + kvh) * p.N + mk);
+          tma_load_2d(sK + kHalfBytes, &tm_k, smem_addr(&bars.k_full[s]), 64,
+                      (b * p.Hkv + kvh) * p.N + mk);
+          if (!mbar_wait(smem_addr(&bars.v_empty[s]), ph ^ 1, ab)) {
+            issued = 2 * j + 1;
+            break;
+          }
+          const uint32_t sV = smem_addr(smem + kOffV + s * kTileBytes);
+          mbar_arrive_expect_tx(smem_addr(&bars.v_full[s]), kTileBytes);
+          tma_load_3d(sV, &tm_v, smem_addr(&bars.v_full[s]), 0, kvh, b * p.N + mk);
+          tma_load_3d(sV + kHalfBytes, &tm_v, smem_addr(&bars.v_full[s]), 64, kvh, b * p.N + mk);
+          issued = 2 * j + 2;
+        }
+        // Let the last loads in flight land before the CTA can exit. This wait ignores the
+        // abort flag (it is set on this path) but keeps its own time limit.
+        int no_abort = 0;
+        Abort local{&no_abort, p.status};
+        for (int t = issued - 1; t >= 0 && t >= issued - 4; t--) {
+          const int j = t >> 1, s = j & 1;
+          const uint32_t ph = (j >> 1) & 1;
+          mbar_wait(smem_addr((t & 1) ? &bars.v_full[s] : &bars.k_full[s]), ph, local);
+        }
+        mbar_wait(qb, 0, local);
       }
-      // every MMA issued above has completed before TMEM is released
-      mma_commit(smem_addr(&bars.drain));
-      int no_abort = 0;
-      Abort local{&no_abort, p.status};
-      mbar_wait(smem_addr(&bars.drain), 0, local);
+    } else if (!skip && warp == 1) {
+      // ------------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint32_t idesc_qk = idesc_bf16_f32(kTile, kTile, false, false);
+        const uint32_t idesc_pv = idesc_bf16_f32(kTile, kD, false, true);
+        bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
+        tc_fence_after();
+        for (int j = 0; ok && j <= nB; j++) {
+          const int jj = j - 1;
+          if (j >= 1) {
+            if (!mbar_wait(smem_addr(&bars.v_full[jj & 1]), (jj >> 1) & 1, ab)) break;
+          }
+          if (j < nB) {
+            if (!mbar_wait(smem_addr(&bars.k_full[j & 1]), (j >> 1) & 1, ab)) break;
+          }
+          tc_fence_after();
+          const uint32_t sK = smem_addr(smem + kOffK + (j & 1) * kTileBytes);
+          const uint32_t sV = smem_addr(smem + kOffV + (jj & 1) * kTileBytes);
+  #pragma unroll
+          for (int t = 0; t < 2; t++) {
+            const int nt = t ? nB : nA;
+            const uint32_t tS = tmem + t * 128, tO = tmem + 256 + t * 128;
+            if (j >= 1 && jj < nt) {
+              if (!mbar_wait(smem_addr(&bars.p_full[t]), jj & 1, ab)) { ok = false; break; }
+              tc_fence_after();
+  #pragma unroll
+              for (int kk = 0; kk < kTile / 16; kk++)  // P of key rows 64h.. at column 64h
+                mma_ts(tO, tS + (kk >> 2) * 64 + (kk & 3) * 8, v_desc(sV, kk), idesc_pv,
+                       (jj > 0 || kk > 0));
+              if (jj == nt - 1) mma_commit(smem_addr(&bars.o_final[t]));
+            }
+            if (j < nt) {
+              const uint32_t sQt = sQ + t * kTileBytes;
+  #pragma unroll
+              for (int kk = 0; kk < kD / 16; kk++)
+                mma_ss(tS, kmajor_desc(sQt, kk), kmajor_desc(sK, kk), idesc_qk, kk > 0);
+              mma_commit(smem_addr(&bars.s_full[t]));
+            }
+          }
+          if (!ok) break;
+          if (j >= 1) mma_commit(smem_addr(&bars.v_empty[jj & 1]));
+          if (j < nB) mma_commit(smem_addr(&bars.k_empty[j & 1]));
+        }
+        // every MMA issued above has completed before TMEM is released
+        mma_commit(smem_addr(&bars.drain));
+        int no_abort = 0;
+        Abort local{&no_abort, p.status};
+        mbar_wait(smem_addr(&bars.drain), 0, local);
+      }
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------------ softmax / epilogue
-    const int t = (warp - 4) >> 2;  // query tile of this warpgroup
-    const int qt = qt0 + t;
-    const int n = t ? nB : nA;
-    const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + t * 128;
-    const uint32_t tO = tmem + lane_off + 256 + t * 128;
-    const float sl2 = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n; j++) {
-      ok = mbar_wait(smem_addr(&bars.s_full[t]), j & 1, ab);
-      __syncwarp();
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-      const bool diag = p.causal && j == qt;
-      // pass 1: row max of the raw scores
-      float mraw = -INFINITY;
-#pragma unroll
-      for (int ch = 0; ch < 4; ch++) {
-        uint32_t x[32];
-        tmem_ld32(tS + ch * 32, x);
-        tmem_wait_ld();
-        if (diag) {
-#pragma unroll
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    if (!skip) {
+      // ------------------------------------------------------------------ softmax / epilogue
+        // warps 4..11 tile A, 12..19 tile B; within a tile the first four warps take key columns
+      // 0..63 and the next four 64..127 of the same rows (lane quarter = warp % 4)
+      const int t = (warp - 4) >> 3;        // query tile
+      const int half = ((warp - 4) >> 2) & 1;
+      const int c0 = half * 64;             // this warp's 64 columns of S, P and O
+      const int qt = qt0 + t;
+      const int n = t ? nB : nA;
+      const int quarter = warp & 3;
+      const int row = quarter * 32 + lane;
+      const uint32_t bar_id = 1 + t * 4 + quarter;  // named barrier of the two warps of a row
+      const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+      const uint32_t tS = tmem + lane_off + t * 128 + c0;
+      const uint32_t tO = tmem + lane_off + 256 + t * 128 + c0;
+      const float sl2 = p.scale_log2;
+      float m = -INFINITY, l = 0.f;   // running max (shared by both halves) and partial sum
+      bool ok = true;
+      for (int j = 0; j < n; j++) {
+        ok = mbar_wait<1>(smem_addr(&bars.s_full[t]), j & 1, ab);
+        __syncwarp();
+        ok = __all_sync(0xffffffffu, ok);
+        tc_fence_after();
+        const bool diag = p.causal && j == qt;
+        uint32_t x0[32], x1[32];
+        float mraw = -INFINITY;
+        if (ok) {
+          tmem_ld32(tS, x0);
+          tmem_ld32(tS + 32, x1);
+          tmem_wait_ld();
+          if (diag) {  // keys after the query (group-local positions) get -inf, so P = 0 there
+            const uint32_t ninf = 0xff800000u;
+  #pragma unroll
+            for (int c = 0; c < 32; c++) {
+              x0[c] = c0 + c <= row ? x0[c] : ninf;
+              x1[c] = c0 + 32 + c <= row ? x1[c] : ninf;
+            }
+          }
+  #pragma unroll
           for (int c = 0; c < 32; c++)
-            if (ch * 32 + c <= row) mraw = fmaxf(mraw, __uint_as_float(x[c]));
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; c++) mraw = fmaxf(mraw, __uint_as_float(x[c]));
+            mraw = fmaxf(mraw, fmaxf(__uint_as_float(x0[c]), __uint_as_float(x1[c])));
         }
+        xmax[j & 1][t][half][row] = mraw;
+        // both warps of the row leave the loop together if either gave up
+        ok = named_bar_and(bar_id, 64, ok);
+        if (!ok) break;
+        mraw = fmaxf(mraw, xmax[j & 1][t][half ^ 1][row]);
+        const float mt = mraw * sl2;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (mt > m + kRescaleThreshold) {
+          alpha = fast_exp2(m - mt);  // 0 while m is -inf
+          rescale = j > 0;
+          m = mt;
+        }
+        // P = exp2(S * sl2 - m) as bf16 over the first 32 of this warp's 64 columns of S
+        const float nm = -m;
+        float rs = 0.f;
+  #pragma unroll
+        for (int ch = 0; ch < 2; ch++) {
+          uint32_t pk[16];
+  #pragma unroll
+          for (int c2 = 0; c2 < 16; c2++) {
+            const float s0 = __uint_as_float(ch ? x1[2 * c2] : x0[2 * c2]);
+            const float s1 = __uint_as_float(ch ? x1[2 * c2 + 1] : x0[2 * c2 + 1]);
+            const float a0 = fmaf(s0, sl2, nm);
+            const float a1 = fmaf(s1, sl2, nm);
+            float p0, p1;
+            if ((kPolyMask >> c2) & 1u) {
+              p0 = exp2_poly(a0);
+              p1 = exp2_poly(a1);
+            } else {
+              p0 = fast_exp2(a0);
+              p1 = fast_exp2(a1);
+            }
+            rs += p0 + p1;
+            pk[c2] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + ch * 16, pk);
+        }
+        l = l * alpha + rs;
+        // O rescale of this warp's 64 columns; PV of the previous key tile has completed
+        // (S_t(j) landed after it), and PV of this one waits for p_full below
+        if (__any_sync(0xffffffffu, rescale)) {
+  #pragma unroll
+          for (int ch = 0; ch < 4; ch++) {
+            uint32_t o[16];
+            tmem_ld16(tO + ch * 16, o);
+            tmem_wait_ld();
+  #pragma unroll
+            for (int c = 0; c < 16; c++) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st16(tO + ch * 16, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_addr(&bars.p_full[t]));
       }
-      const float mt = mraw * sl2;
-      float alpha = 1.f;
-      bool rescale = false;
-      if (mt > m + kRescaleThreshold) {
-        alpha = fast_exp2(m - mt);  // 0 while m is -inf
-        rescale = j > 0;
-        m = mt;
+      if (ok) {
+        ok = mbar_wait<1>(smem_addr(&bars.o_final[t]), 0, ab);
+        __syncwarp();
+        ok = __all_sync(0xffffffffu, ok);
       }
-      if (__any_sync(0xffffffffu, rescale)) {
-#pragma unroll
-        for (int ch = 0; ch < 4; ch++) {
+      // total row sum = both halves' partial sums (every path reaches this barrier)
+      if (half == 1) xsum[t][row] = l;
+      named_bar_sync(bar_id, 64);
+      if (half == 0) xsum[t][row] += l;
+      named_bar_sync(bar_id, 64);
+      const float ltot = xsum[t][row];
+      if (ok) {
+        tc_fence_after();
+        const int mrow = src_row(r0 + t * kTile + row, sh, p.G, p.N);
+        __nv_bfloat16* orow =
+            static_cast<__nv_bfloat16*>(p.o) + ((size_t)(b * p.N + mrow) * p.Hq + h) * kD + c0;
+        const float inv_l = 1.f / ltot;
+  #pragma unroll
+        for (int ch = 0; ch < 2; ch++) {
           uint32_t o[32];
           tmem_ld32(tO + ch * 32, o);
           tmem_wait_ld();
-#pragma unroll
-          for (int c = 0; c < 32; c++) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-          tmem_st32(tO + ch * 32, o);
+          uint4 pk[4];
+          uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+  #pragma unroll
+          for (int c2 = 0; c2 < 16; c2++)
+            pw[c2] = pack_bf16x2(__uint_as_float(o[2 * c2]) * inv_l,
+                                 __uint_as_float(o[2 * c2 + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+  #pragma unroll
+          for (int c4 = 0; c4 < 4; c4++) dst[c4] = pk[c4];
         }
+        if (half == 0)
+          p.lse[((size_t)b * p.Hq + h) * p.N + mrow] = (m + __log2f(ltot)) * 0.69314718055994531f;
       }
-      // pass 2: P = exp2(S * sl2 - m) as bf16 over the scores already consumed
-      const float nm = -m;
-      float rs = 0.f;
-#pragma unroll
-      for (int ch = 0; ch < 4; ch++) {
-        uint32_t x[32];
-        tmem_ld32(tS + ch * 32, x);
-        tmem_wait_ld();
-        uint32_t pk[16];
-#pragma unroll
-        for (int c2 = 0; c2 < 16; c2++) {
-          const float a0 = fmaf(__uint_as_float(x[2 * c2]), sl2, nm);
-          const float a1 = fmaf(__uint_as_float(x[2 * c2 + 1]), sl2, nm);
-          float p0, p1;
-          if ((kPolyMask >> c2) & 1u) {
-            p0 = exp2_poly(a0);
-            p1 = exp2_poly(a1);
-          } else {
-            p0 = fast_exp2(a0);
-            p1 = fast_exp2(a1);
-          }
-          if (diag) {
-            if (ch * 32 + 2 * c2 > row) p0 = 0.f;
-            if (ch * 32 + 2 * c2 + 1 > row) p1 = 0.f;
-          }
-          rs += p0 + p1;
-          pk[c2] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(tS + ch * 16, pk);
-      }
-      l = l * alpha + rs;
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(smem_addr(&bars.p_full[t]));
-    }
-    if (ok) {
-      ok = mbar_wait(smem_addr(&bars.o_final[t]), 0, ab);
-      __syncwarp();
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
-      tc_fence_after();
-      const int mrow = src_row(r0 + t * kTile + row, sh, p.G, p.N);
-      __nv_bfloat16* orow =
-          static_cast<__nv_bfloat16*>(p.o) + ((size_t)(b * p.N + mrow) * p.Hq + h) * kD;
-      const float inv_l = 1.f / l;
-#pragma unroll
-      for (int ch = 0; ch < 4; ch++) {
-        uint32_t o[32];
-        tmem_ld32(tO + ch * 32, o);
-        tmem_wait_ld();
-        uint4 pk[4];
-        uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
-#pragma unroll
-        for (int c2 = 0; c2 < 16; c2++)
-          pw[c2] = pack_bf16x2(__uint_as_float(o[2 * c2]) * inv_l,
-                               __uint_as_float(o[2 * c2 + 1]) * inv_l);
-        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
-#pragma unroll
-        for (int c4 = 0; c4 < 4; c4++) dst[c4] = pk[c4];
-      }
-      p.lse[((size_t)b * p.Hq + h) * p.N + mrow] = (m + __log2f(l)) * 0.69314718055994531f;
     }
   }
 
@@ -376,6 +415,12 @@ cudaError_t launch_tc_fwd(const Params& p, cudaStream_t st) {
   if ((e = cudaFuncSetAttribute(tc_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kSmemBytes)))
     return e;
+  // setmaxnreg.inc waits until the registers it asks for are free: refuse to launch unless the
+  // split fits what the launch hands out
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, tc_fwd_kernel))) return e;
+  if (128 * kRegsOther + (kThreads - 128) * kRegsSoftmax > kThreads * fa.numRegs)
+    return cudaErrorInvalidConfiguration;
   const long pairs = (long)p.B * p.Hq * (p.N / p.G) * (p.G / kTile / 2);
   tc_fwd_kernel<<<dim3((unsigned)pairs), dim3(kThreads), kSmemBytes, st>>>(p, tq, tk, tv);
   return cudaGetLastError();
