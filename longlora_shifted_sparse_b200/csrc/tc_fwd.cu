@@ -91,14 +91,88 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// A or B operand tile (128 rows x 128 bf16, two 64-column SW128 boxes), K-major, k-step kk.
-__device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_saddr, int kk) {
-  return smem_desc_sw128(tile_saddr + (kk >> 2) * kHalfBytes + (kk & 3) * 32, 16, 1024);
+__device__ __forceinline__ uint64_t opaque64(uint64_t v) {
+  uint64_t r;
+  asm volatile("mov.b64 %0, %1;" : "=l"(r) : "l"(v));
+  return r;
 }
 
-// V tile as the MN-major B operand of O += P V: k-step kk covers kv rows 16kk..16kk+15.
-__device__ __forceinline__ uint64_t v_desc(uint32_t tile_saddr, int kk) {
-  return smem_desc_sw128(tile_saddr + kk * 2048, kHalfBytes, 1024);
+// Max of a thread's 64 scores, as a tree (short dependency chain).
+__device__ __forceinline__ float max64(const uint32_t (&x0)[32], const uint32_t (&x1)[32]) {
+  float mm[16];
+#pragma unroll
+  for (int c = 0; c < 16; c++)
+    mm[c] = fmaxf(fmaxf(__uint_as_float(x0[2 * c]), __uint_as_float(x0[2 * c + 1])),
+                  fmaxf(__uint_as_float(x1[2 * c]), __uint_as_float(x1[2 * c + 1])));
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int c = 0; c < w; c++) mm[c] = fmaxf(mm[c], mm[c + w]);
+  return mm[0];
+}
+
+// P = exp2(S * sl2 - m) for a thread's 64 scores, written as bf16 pairs over the first 32
+// of its 64 TMEM columns of S (the PV MMA reads them from there); returns the sum of P.
+__device__ __forceinline__ float write_p64(const uint32_t (&x0)[32], const uint32_t (&x1)[32],
+                                           float sl2, float nm, uint32_t tS) {
+  float rs = 0.f;
+#pragma unroll
+  for (int ch = 0; ch < 2; ch++) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int c2 = 0; c2 < 16; c2++) {
+      const float s0 = __uint_as_float(ch ? x1[2 * c2] : x0[2 * c2]);
+      const float s1 = __uint_as_float(ch ? x1[2 * c2 + 1] : x0[2 * c2 + 1]);
+      const float a0 = fmaf(s0, sl2, nm);
+      const float a1 = fmaf(s1, sl2, nm);
+      float p0, p1;
+      if ((kPolyMask >> c2) & 1u) {
+        p0 = exp2_poly(a0);
+        p1 = exp2_poly(a1);
+      } else {
+        p0 = fast_exp2(a0);
+        p1 = fast_exp2(a1);
+      }
+      rs += p0 + p1;
+      pk[c2] = pack_bf16x2(p0, p1);
+    }
+    tmem_st16(tS + ch * 16, pk);
+  }
+  return rs;
+}
+
+// Multiplies the 64 bf16 P values a thread wrote (32 packed columns) by a power of two,
+// which is exact in bf16.
+__device__ __forceinline__ void scale_p64(uint32_t tS, float f) {
+  uint32_t x[32];
+  tmem_ld32(tS, x);
+  tmem_wait_ld();
+#pragma unroll
+  for (int c = 0; c < 32; c++)
+    x[c] = pack_bf16x2(__uint_as_float(x[c] << 16) * f, __uint_as_float(x[c] & 0xffff0000u) * f);
+  tmem_st32(tS, x);
+}
+
+// 2^k for an integral k <= 0 (k = -inf gives 0), exact.
+__device__ __forceinline__ float exp2_int(float k) {
+  return k < -126.f ? 0.f : __int_as_float((static_cast<int>(k) + 127) << 23);
+}
+
+// Loads the thread's 64 scores; on the diagonal tile the keys after the query (group-local
+// positions) get -inf, so that their P is 0.
+__device__ __forceinline__ void load_s64(uint32_t tS, bool diag, int first_col, int row,
+                                         uint32_t (&x0)[32], uint32_t (&x1)[32]) {
+  tmem_ld32(tS, x0);
+  tmem_ld32(tS + 32, x1);
+  tmem_wait_ld();
+  if (diag) {
+    const uint32_t ninf = 0xff800000u;
+#pragma unroll
+    for (int c = 0; c < 32; c++) {
+      x0[c] = first_col + c <= row ? x0[c] : ninf;
+      x1[c] = first_col + 32 + c <= row ? x1[c] : ninf;
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -209,6 +283,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         const uint32_t idesc_qk = idesc_bf16_f32(kTile, kTile, false, false);
         const uint32_t idesc_pv = idesc_bf16_f32(kTile, kD, false, true);
+        // Descriptors are built once; a k-step or a stage only adds a constant to the start
+        // address field (bytes / 16; every address stays below 256 KB, so no carry leaves it).
+        // One thread issues every MMA while four softmax warps share its scheduler, so the
+        // issue path is kept to a few instructions per MMA.
+        const uint64_t dQ = smem_desc_sw128(sQ, 16, 1024);
+        const uint64_t dK = smem_desc_sw128(smem_addr(smem + kOffK), 16, 1024);
+        const uint64_t dV = smem_desc_sw128(smem_addr(smem + kOffV), kHalfBytes, 1024);
+        constexpr uint32_t kTileDesc = kTileBytes >> 4;
         bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
         tc_fence_after();
         for (int j = 0; ok && j <= nB; j++) {
@@ -220,26 +302,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!mbar_wait(smem_addr(&bars.k_full[j & 1]), (j >> 1) & 1, ab)) break;
           }
           tc_fence_after();
-          const uint32_t sK = smem_addr(smem + kOffK + (j & 1) * kTileBytes);
-          const uint32_t sV = smem_addr(smem + kOffV + (jj & 1) * kTileBytes);
-  #pragma unroll
+          // opaque per-iteration bases: the per-k-step descriptors are formed by one add at
+          // their MMA instead of being hoisted out of the loop into (spilled) registers
+          const uint64_t dKj = opaque64(dK) + (uint64_t)((j & 1) * kTileDesc);
+          const uint64_t dVj = opaque64(dV) + (uint64_t)((jj & 1) * kTileDesc);
+          const uint64_t dQj = opaque64(dQ);
+#pragma unroll
           for (int t = 0; t < 2; t++) {
             const int nt = t ? nB : nA;
             const uint32_t tS = tmem + t * 128, tO = tmem + 256 + t * 128;
             if (j >= 1 && jj < nt) {
               if (!mbar_wait(smem_addr(&bars.p_full[t]), jj & 1, ab)) { ok = false; break; }
               tc_fence_after();
-  #pragma unroll
-              for (int kk = 0; kk < kTile / 16; kk++)  // P of key rows 64h.. at column 64h
-                mma_ts(tO, tS + (kk >> 2) * 64 + (kk & 3) * 8, v_desc(sV, kk), idesc_pv,
-                       (jj > 0 || kk > 0));
+              const uint32_t acc0 = jj > 0;
+#pragma unroll
+              for (int kk = 0; kk < kTile / 16; kk++)  // P of key rows 64h.. at column 64h;
+                mma_ts(tO, tS + (kk >> 2) * 64 + (kk & 3) * 8,  // V k-step = 16 rows
+                       dVj + (uint64_t)(kk * (2048 >> 4)), idesc_pv, kk ? 1u : acc0);
               if (jj == nt - 1) mma_commit(smem_addr(&bars.o_final[t]));
             }
             if (j < nt) {
-              const uint32_t sQt = sQ + t * kTileBytes;
-  #pragma unroll
-              for (int kk = 0; kk < kD / 16; kk++)
-                mma_ss(tS, kmajor_desc(sQt, kk), kmajor_desc(sK, kk), idesc_qk, kk > 0);
+              const uint64_t dQt = dQj + (uint64_t)(t * kTileDesc);
+#pragma unroll
+              for (int kk = 0; kk < kD / 16; kk++) {
+                const uint64_t koff = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+                mma_ss(tS, dQt + koff, dKj + koff, idesc_qk, kk > 0);
+              }
               mma_commit(smem_addr(&bars.s_full[t]));
             }
           }
@@ -280,72 +368,54 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
         const bool diag = p.causal && j == qt;
-        uint32_t x0[32], x1[32];
-        float mraw = -INFINITY;
+        float mraw = -INFINITY, rs = 0.f, alpha = 1.f;
+        bool rescale = false, stored = false;
         if (ok) {
-          tmem_ld32(tS, x0);
-          tmem_ld32(tS + 32, x1);
-          tmem_wait_ld();
-          if (diag) {  // keys after the query (group-local positions) get -inf, so P = 0 there
-            const uint32_t ninf = 0xff800000u;
-  #pragma unroll
-            for (int c = 0; c < 32; c++) {
-              x0[c] = c0 + c <= row ? x0[c] : ninf;
-              x1[c] = c0 + 32 + c <= row ? x1[c] : ninf;
-            }
+          uint32_t x0[32], x1[32];
+          load_s64(tS, diag, c0, row, x0, x1);
+          mraw = max64(x0, x1);
+          // Fast path: this warp's half rows all have a running max m already (m is -inf
+          // only before the first key tile) and stay within 2^8 of it, so P = exp2(S sl2 -
+          // m) can be written at once, before the other half's max is known. A half row
+          // that is wholly masked (mraw = -inf) gets P = 0 here. The decision is per warp:
+          // the TMEM stores are warp-collective.
+          if (__all_sync(0xffffffffu, m > -INFINITY && mraw * sl2 <= m + kRescaleThreshold)) {
+            rs = write_p64(x0, x1, sl2, -m, tS);
+            stored = true;
           }
-  #pragma unroll
-          for (int c = 0; c < 32; c++)
-            mraw = fmaxf(mraw, fmaxf(__uint_as_float(x0[c]), __uint_as_float(x1[c])));
         }
-        xmax[j & 1][t][half][row] = mraw;
-        // both warps of the row leave the loop together if either gave up
-        ok = named_bar_and(bar_id, 64, ok);
-        if (!ok) break;
-        mraw = fmaxf(mraw, xmax[j & 1][t][half ^ 1][row]);
-        const float mt = mraw * sl2;
-        float alpha = 1.f;
-        bool rescale = false;
-        if (mt > m + kRescaleThreshold) {
-          alpha = fast_exp2(m - mt);  // 0 while m is -inf
-          rescale = j > 0;
-          m = mt;
-        }
-        // P = exp2(S * sl2 - m) as bf16 over the first 32 of this warp's 64 columns of S
-        const float nm = -m;
-        float rs = 0.f;
-  #pragma unroll
-        for (int ch = 0; ch < 2; ch++) {
-          uint32_t pk[16];
-  #pragma unroll
-          for (int c2 = 0; c2 < 16; c2++) {
-            const float s0 = __uint_as_float(ch ? x1[2 * c2] : x0[2 * c2]);
-            const float s1 = __uint_as_float(ch ? x1[2 * c2 + 1] : x0[2 * c2 + 1]);
-            const float a0 = fmaf(s0, sl2, nm);
-            const float a1 = fmaf(s1, sl2, nm);
-            float p0, p1;
-            if ((kPolyMask >> c2) & 1u) {
-              p0 = exp2_poly(a0);
-              p1 = exp2_poly(a1);
-            } else {
-              p0 = fast_exp2(a0);
-              p1 = fast_exp2(a1);
-            }
-            rs += p0 + p1;
-            pk[c2] = pack_bf16x2(p0, p1);
+        // Slow path, taken by both warps of the row together when either half has not
+        // written its P (first key tile, a max that grew past the threshold) or gave up
+        // waiting: exchange the exact max; m moves to ceil(max * sl2), an integer, so a P
+        // already written with the old m is brought to the new one by an exact power of two.
+        if (named_bar_or(bar_id, 64, !stored || !ok)) {
+          xmax[j & 1][t][half][row] = mraw;
+          ok = named_bar_and(bar_id, 64, ok);
+          if (!ok) break;
+          const float mt = fmaxf(mraw, xmax[j & 1][t][half ^ 1][row]) * sl2;
+          const float mnew = mt > m + kRescaleThreshold ? ceilf(mt) : m;
+          alpha = exp2_int(m - mnew);  // 0 while m is -inf, 1 if m stays
+          rescale = j > 0 && mnew != m;
+          if (!stored) {  // (warp-uniform) S is intact: nothing was written over it
+            uint32_t x0[32], x1[32];
+            load_s64(tS, diag, c0, row, x0, x1);
+            rs = write_p64(x0, x1, sl2, -mnew, tS);
+          } else if (__any_sync(0xffffffffu, mnew != m)) {
+            scale_p64(tS, alpha);
+            rs *= alpha;
           }
-          tmem_st16(tS + ch * 16, pk);
+          m = mnew;
         }
         l = l * alpha + rs;
         // O rescale of this warp's 64 columns; PV of the previous key tile has completed
         // (S_t(j) landed after it), and PV of this one waits for p_full below
         if (__any_sync(0xffffffffu, rescale)) {
-  #pragma unroll
+#pragma unroll
           for (int ch = 0; ch < 4; ch++) {
             uint32_t o[16];
             tmem_ld16(tO + ch * 16, o);
             tmem_wait_ld();
-  #pragma unroll
+#pragma unroll
             for (int c = 0; c < 16; c++) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
             tmem_st16(tO + ch * 16, o);
           }
@@ -371,19 +441,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         __nv_bfloat16* orow =
             static_cast<__nv_bfloat16*>(p.o) + ((size_t)(b * p.N + mrow) * p.Hq + h) * kD + c0;
         const float inv_l = 1.f / ltot;
-  #pragma unroll
+#pragma unroll
         for (int ch = 0; ch < 2; ch++) {
           uint32_t o[32];
           tmem_ld32(tO + ch * 32, o);
           tmem_wait_ld();
           uint4 pk[4];
           uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
-  #pragma unroll
+#pragma unroll
           for (int c2 = 0; c2 < 16; c2++)
             pw[c2] = pack_bf16x2(__uint_as_float(o[2 * c2]) * inv_l,
                                  __uint_as_float(o[2 * c2 + 1]) * inv_l);
           uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
-  #pragma unroll
+#pragma unroll
           for (int c4 = 0; c4 < 4; c4++) dst[c4] = pk[c4];
         }
         if (half == 0)

@@ -200,3 +200,41 @@ def test_device_status_and_profiler(s2):
     assert summary["rope_pi"][0] == 2 and summary["bwd_rowsum"][0] == 1
     assert sum(n for n, _ in summary.values()) == 6
     assert all(ms > 0 for _, ms in summary.values())
+
+
+def test_softmax_rescale_paths(s2):
+    """Scores whose running row max climbs by well over the forward's rescale threshold
+    (2^8) along each group, so that the exact-max exchange, the power-of-two rescale of P
+    already written and the O rescale all run, checked forward and backward against the
+    oracle.
+
+    Inputs: q, k, v ~ N(0,1)*0.5, then channel 0 of every q row set to 8 and channel 0 of
+    every k row raised by 16 * (group-local position / G): the score gains ~11 nats from the
+    first to the last key of a group (~1.4 nats per 128-key tile), while the keys of one tile
+    stay within a few nats of each other, so the softmax rows are not one-hot and the
+    backward tolerances keep their meaning. A position-interpolation factor of 1e30 makes
+    every RoPE angle ~1e-27 rad: the rotation is the identity far below bf16 resolution on
+    both sides, so channel 0 keeps its role in every head. The test first checks its own
+    premise on the fp64 scores."""
+    w = Workload("rescale", 1, 2048, 4, 2, 128, 1024, 1e30, "bf16", 0.5, True, seed=31)
+    q, k, v, do = H.inputs(w, with_dout=True)
+    qf = synth.bf16_bits_to_f32(q)
+    kf = synth.bf16_bits_to_f32(k)
+    qf[..., 0] = 8.0
+    kf[..., 0] += (16.0 * (np.arange(w.N) % w.G) / w.G).astype(np.float32)[None, :, None]
+    q, k = synth.f32_to_bf16_bits(qf), synth.f32_to_bf16_bits(kf)
+    # premise: rows of the unshifted head 0, group 0 whose running max (log2 units) grows by
+    # more than 8 after their first key tile
+    qg = synth.bf16_bits_to_f32(q).astype(np.float64)[0, :w.G, 0]
+    kg = synth.bf16_bits_to_f32(k).astype(np.float64)[0, :w.G, 0]
+    sc = qg @ kg.T / np.sqrt(w.d) * np.log2(np.e)
+    sc[np.triu_indices(w.G, 1)] = -np.inf
+    grows = sum(sc[i, :i + 1].max() > sc[i, :128].max() + 8 for i in range(128, w.G))
+    assert grows > 100, grows
+    o, lse, grads = _run(s2, w, q, k, v, do)
+    o_ref, lse_ref = oracle.fwd(q, k, v, w.G, w.pi_scale, w.rope_base, w.causal)
+    H.assert_close_o(H.to_host_f64(o), o_ref, w.dtype)
+    H.assert_close_lse(H.to_host_f64(lse), lse_ref, w.dtype)
+    refs = oracle.bwd(q, k, v, do, w.G, w.pi_scale, w.rope_base, w.causal)
+    for name, g, r in zip(("dq", "dk", "dv"), grads, refs):
+        H.assert_close_grad(H.to_host_f64(g), r, w.dtype, name)
