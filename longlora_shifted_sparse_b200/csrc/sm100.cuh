@@ -51,6 +51,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep up to `suspend_ns` for the phase to complete
+// (it wakes when the phase completes). Sleeping waiters leave the shared-memory pipe to the
+// tensor cores, whose shared-memory operand reads need all of its bandwidth.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Shared abort state of one CTA: a flag in shared memory plus the call's global status word.
 struct Abort {
   volatile int* flag;   // shared memory
@@ -62,6 +78,9 @@ struct Abort {
 // false. Every other wait of the CTA, and of every other CTA of the launch (they poll the
 // status word), then gives up at its next check.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Longest sleep of one try-wait in the slow path; the abort flag, the status word and the
+// clock are checked every 16 try-waits.
+constexpr uint32_t kWaitSleepNs = 20000u;
 
 // kRegion gives each register budget of a kernel that splits its registers (setmaxnreg) its
 // own copy of the out-of-line slow path: a function called from two budgets cannot be
@@ -71,8 +90,8 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity
                                                    uint64_t limit_ns) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 0;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 255u) {
+    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+    if ((i & 15u) == 15u) {
       if (*ab.flag) return false;
       if (*reinterpret_cast<volatile unsigned*>(ab.status) != 0u) {  // another CTA gave up
         *ab.flag = 1;

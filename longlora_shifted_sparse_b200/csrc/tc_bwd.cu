@@ -71,6 +71,44 @@ __device__ __forceinline__ uint64_t mn_desc(uint32_t tile_saddr, int kk) {
   return smem_desc_sw128(tile_saddr + kk * 2048, kBoxBytes, 1024);
 }
 
+// The same descriptors' offsets (in 16-byte units) from the tile's k-step 0 descriptor.
+__device__ __forceinline__ uint64_t kmajor_koff(int kk) {
+  return (uint64_t)(((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4);
+}
+__device__ __forceinline__ uint64_t mn_koff(int kk) { return (uint64_t)((kk * 2048) >> 4); }
+constexpr uint32_t kTileDesc = kTileBytes >> 4;  // one tile, in descriptor address units
+
+// Keeps a value in a register as an opaque quantity, so that the descriptors derived from it
+// per stage and k-step are formed by one add where they are used instead of being hoisted
+// out of the loops (and spilled).
+__device__ __forceinline__ uint64_t opaque64(uint64_t v) {
+  uint64_t r;
+  asm volatile("mov.b64 %0, %1;" : "=l"(r) : "l"(v));
+  return r;
+}
+
+// Causal mask of a diagonal tile, applied to a thread's 64 raw scores (columns c = 0..63 of
+// its half) before the exponential: the score becomes -inf, so its probability is exactly 0.
+// upper = 0 masks the columns c < lim, upper = 1 the columns c > lim. Called only on the
+// diagonal tile (a warp-uniform branch), so the other tiles pay nothing for the mask.
+__device__ __forceinline__ void mask_scores(uint32_t (&x0)[32], uint32_t (&x1)[32], int lim,
+                                            int upper) {
+  const uint32_t ninf = 0xff800000u;
+#pragma unroll
+  for (int c = 0; c < 32; c++) {
+    if (upper ? c > lim : c < lim) x0[c] = ninf;
+    if (upper ? c + 32 > lim : c + 32 < lim) x1[c] = ninf;
+  }
+}
+
+// Makes the 64 values count as used here: the exponentials of the probabilities are then
+// computed before the wait that follows (while the tensor cores work) instead of being
+// scheduled after it, where they would lengthen the critical path of the next MMA.
+__device__ __forceinline__ void pin_regs(float (&x)[64]) {
+#pragma unroll
+  for (int c = 0; c < 64; c++) asm volatile("" : "+f"(x[c]));
+}
+
 // TMEM column of the bf16 A operand for k-step kk (16 K rows = 8 packed columns). Each
 // math warp owns 64 K rows (columns c0 = 0 or 64 of the tile) and writes them chunk by
 // chunk (32 K rows each) into the 32 fp32 columns it has just read:
@@ -330,14 +368,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(smem_addr(&bars.st_consumed));  // S^T may now be overwritten
+        if (diag) mask_scores(x0, x1, row - c0, 0);  // query row c0+c before key row: P = 0
 #pragma unroll
         for (int c = 0; c < 64; c++) {
           const float l = __shfl_sync(0xffffffffu, nl2[c >> 5], c & 31);
-          const float st = __uint_as_float(c < 32 ? x0[c] : x1[c - 32]);
-          float v = fast_exp2(fmaf(st, sl2, l));
-          if (diag && c0 + c < row) v = 0.f;  // query row c0+c before key row: masked
-          pr[c] = v;
+          pr[c] = fast_exp2(fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, l));
         }
+        pin_regs(pr);
       }
       ok = mbar_wait(smem_addr(&bars.dpt_full), n & 1, ab);
       __syncwarp();
@@ -407,16 +444,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ================================================================================ dQ
 
-// smem: Q | dO | K stages 0..2 | V stages 0..1
-constexpr int kKStages = 3, kVStages = 2;
-constexpr uint32_t kQOffQ = 0;
-constexpr uint32_t kQOffDO = kTileBytes;
-constexpr uint32_t kQOffK = 2 * kTileBytes;
-constexpr uint32_t kQOffV = (2 + kKStages) * kTileBytes;
-constexpr uint32_t kQSmem = (2 + kKStages + kVStages) * kTileBytes + 1024;
+// smem: K stages 0..3 | V stages 0..2 (Q~ and dO of the CTA's query tile live in TMEM)
+constexpr int kKStages = 4, kVStages = 3;
+constexpr uint32_t kQOffK = 0;
+constexpr uint32_t kQOffV = kKStages * kTileBytes;
+constexpr uint32_t kQSmem = (kKStages + kVStages) * kTileBytes + 1024;
 
 struct DqBarriers {
-  uint64_t q_full;
+  uint64_t qdo_ready;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full, s_consumed, dp_full, ds_ready;
@@ -452,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   Abort ab{&abort_flag, p.status};
   if (threadIdx.x == 0) {
     abort_flag = *reinterpret_cast<volatile unsigned*>(p.status) != 0u;
-    mbar_init(smem_addr(&bars.q_full), 1);
+    mbar_init(smem_addr(&bars.qdo_ready), kMathThreads);
     for (int s = 0; s < kKStages; s++) {
       mbar_init(smem_addr(&bars.k_full[s]), 1);
       mbar_init(smem_addr(&bars.k_empty[s]), 1);
@@ -474,24 +509,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  const uint32_t colS = 0, colDP = 128, colDQ = 256;
-  const uint32_t sQ = smem_addr(smem + kQOffQ), sDO = smem_addr(smem + kQOffDO);
+  // TMEM: S | dP (dS written over it) | dQ accumulator | Q~ and dO as bf16 A operands
+  const uint32_t colS = 0, colDP = 128, colDQ = 256, colQ = 384, colDO = 448;
   const bool skip = abort_flag != 0;
 
   if (skip) {
   } else if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_do);
-      const uint32_t qb = smem_addr(&bars.q_full);
-      mbar_arrive_expect_tx(qb, 2 * kTileBytes);
-      const int qrow = (b * p.Hq + h) * p.N + mq0;
-      tma_load_2d(sQ, &tm_q, qb, 0, qrow);
-      tma_load_2d(sQ + kBoxBytes, &tm_q, qb, 64, qrow);
-      tma_load_3d(sDO, &tm_do, qb, 0, h, b * p.N + mq0);
-      tma_load_3d(sDO + kBoxBytes, &tm_do, qb, 64, h, b * p.N + mq0);
       int nk_issued = 0, nv_issued = 0;
       for (int j = 0; j < nkv; j++) {
         const int mk = src_row(g * p.G + j * kTile, sh, p.G, p.N);
@@ -518,38 +544,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(smem_addr(&bars.k_full[j % kKStages]), (j / kKStages) & 1, local);
       for (int j = nv_issued - 1; j >= 0 && j >= nv_issued - kVStages; j--)
         mbar_wait(smem_addr(&bars.v_full[j % kVStages]), (j / kVStages) & 1, local);
-      mbar_wait(qb, 0, local);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
       const uint32_t idesc_g = idesc_bf16_f32(kTile, kD, false, true);
-      auto issue_s = [&](int j) -> bool {  // S(j) = Q K_j^T
+      // Descriptors are built once; a stage or a k-step only adds a constant to the start
+      // address field (bytes / 16; shared memory stays below 256 KB, so nothing carries out).
+      const uint64_t dK0 = smem_desc_sw128(smem_addr(smem + kQOffK), 16, 1024);
+      const uint64_t dKm0 = smem_desc_sw128(smem_addr(smem + kQOffK), kBoxBytes, 1024);
+      const uint64_t dV0 = smem_desc_sw128(smem_addr(smem + kQOffV), 16, 1024);
+      auto issue_s = [&](int j) -> bool {  // S(j) = Q K_j^T, Q from TMEM
         const int sk = j % kKStages;
         if (!mbar_wait(smem_addr(&bars.k_full[sk]), (j / kKStages) & 1, ab)) return false;
         tc_fence_after();
-        const uint32_t sKs = smem_addr(smem + kQOffK + sk * kTileBytes);
+        const uint64_t dk = opaque64(dK0) + (uint64_t)(sk * kTileDesc);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; kk++)
-          mma_ss(tmem + colS, kmajor_desc(sQ, kk), kmajor_desc(sKs, kk), idesc_s, kk > 0);
+          mma_ts(tmem + colS, tmem + colQ + kk * 8, dk + kmajor_koff(kk), idesc_s, kk > 0);
         mma_commit(smem_addr(&bars.s_full));
         return true;
       };
-      auto issue_dp = [&](int j) -> bool {  // dP(j) = dO V_j^T
+      auto issue_dp = [&](int j) -> bool {  // dP(j) = dO V_j^T, dO from TMEM
         const int sv = j % kVStages;
         if (!mbar_wait(smem_addr(&bars.v_full[sv]), (j / kVStages) & 1, ab)) return false;
         tc_fence_after();
-        const uint32_t sVs = smem_addr(smem + kQOffV + sv * kTileBytes);
+        const uint64_t dv = opaque64(dV0) + (uint64_t)(sv * kTileDesc);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; kk++)
-          mma_ss(tmem + colDP, kmajor_desc(sDO, kk), kmajor_desc(sVs, kk), idesc_s, kk > 0);
+          mma_ts(tmem + colDP, tmem + colDO + kk * 8, dv + kmajor_koff(kk), idesc_s, kk > 0);
         mma_commit(smem_addr(&bars.dp_full));
         mma_commit(smem_addr(&bars.v_empty[sv]));
         return true;
       };
       // issue order: S(0) dP(0) S(1) | dQ(0) dP(1) S(2) | dQ(1) dP(2) S(3) | ...
       // (see the dK/dV pass: the MMAs the next math phase waits for go first)
-      bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
+      bool ok = mbar_wait(smem_addr(&bars.qdo_ready), 0, ab);
       tc_fence_after();
       if (ok) ok = issue_s(0) && issue_dp(0);
       if (ok && nkv > 1) ok = mbar_wait(smem_addr(&bars.s_consumed), 0, ab) && issue_s(1);
@@ -557,11 +587,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ph = j & 1;
         if (!mbar_wait(smem_addr(&bars.ds_ready), ph, ab)) break;
         tc_fence_after();
-        const uint32_t sKs = smem_addr(smem + kQOffK + (j % kKStages) * kTileBytes);
+        const uint64_t dkm = opaque64(dKm0) + (uint64_t)((j % kKStages) * kTileDesc);
+        const uint32_t acc0 = j > 0;
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; kk++)
-          mma_ts(tmem + colDQ, tmem + packed_col(colDP, kk, 16), mn_desc(sKs, kk), idesc_g,
-                 (j > 0 || kk > 0));
+          mma_ts(tmem + colDQ, tmem + packed_col(colDP, kk, 16), dkm + mn_koff(kk), idesc_g,
+                 kk ? 1u : acc0);
         mma_commit(smem_addr(&bars.k_empty[j % kKStages]));
         if (j + 1 < nkv && !issue_dp(j + 1)) break;
         if (j + 2 < nkv) {
@@ -584,6 +615,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tDP = tmem + lane_off + colDP + c0;
     const int m = src_row(g * p.G + qt * kTile + row, sh, p.G, p.N);
     const size_t lrow = ((size_t)b * p.Hq + h) * p.N + m;
+    // This thread's half row (d = c0 .. c0+63) of Q~ and of dO into TMEM, as the bf16 A
+    // operands of S = Q K^T and dP = dO V^T: column j of a row holds elements 2j, 2j+1,
+    // which is the order of the row in memory.
+    {
+      const uint4* qsrc = reinterpret_cast<const uint4*>(
+          static_cast<const __nv_bfloat16*>(p.qr) + lrow * kD + c0);
+      const uint4* dsrc = reinterpret_cast<const uint4*>(
+          static_cast<const __nv_bfloat16*>(p.dout) + ((size_t)(b * p.N + m) * p.Hq + h) * kD + c0);
+      uint32_t w[32];
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const uint4 t = __ldg(qsrc + i);
+        w[4 * i] = t.x; w[4 * i + 1] = t.y; w[4 * i + 2] = t.z; w[4 * i + 3] = t.w;
+      }
+      tmem_st32(tmem + lane_off + colQ + c0 / 2, w);
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const uint4 t = __ldg(dsrc + i);
+        w[4 * i] = t.x; w[4 * i + 1] = t.y; w[4 * i + 2] = t.z; w[4 * i + 3] = t.w;
+      }
+      tmem_st32(tmem + lane_off + colDO + c0 / 2, w);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_addr(&bars.qdo_ready));
+    }
     const float nlse2 = -p.lse[lrow] * kLog2e;
     const float Dm = p.Dsum[lrow];
     const float sl2 = p.scale_log2;
@@ -602,12 +658,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(smem_addr(&bars.s_consumed));  // S may now be overwritten
+        if (diag) mask_scores(x0, x1, row - c0, 1);  // key column after the query row: P = 0
 #pragma unroll
-        for (int c = 0; c < 64; c++) {
-          float v = fast_exp2(fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, nlse2));
-          if (diag && c0 + c > row) v = 0.f;  // key column after the query row: masked
-          pr[c] = v;
-        }
+        for (int c = 0; c < 64; c++)
+          pr[c] = fast_exp2(fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, nlse2));
+        pin_regs(pr);
       }
       ok = mbar_wait(smem_addr(&bars.dp_full), j & 1, ab);
       __syncwarp();
