@@ -260,8 +260,10 @@ def run_ours(args):
     def step():
         s2.forward(tq, tk, tv, w.G, w.pi_scale, w.rope_base, w.causal, ws=ws, out=o, lse=lse)
         if w.backward:
+            # the training-step order: the backward reuses the rotation the forward left in
+            # the workspace (s2attn_bwd_after_fwd), as the autograd wrapper does
             s2.backward(tq, tk, tv, o, lse, tdo, w.G, w.pi_scale, w.rope_base, w.causal, ws=ws,
-                        grads=(gq, gk, gv))
+                        grads=(gq, gk, gv), after_forward=True)
 
     def barrier():
         if world > 1:

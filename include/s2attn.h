@@ -93,6 +93,22 @@ S2_API s2_status s2attn_bwd(const void* q, const void* k, const void* v, const v
                      float pi_scale, float rope_base, int dtype,
                      void* workspace, size_t ws_bytes, void* cuda_stream);
 
+/* Backward that reuses the forward's rotation: identical arguments, semantics and outputs
+ * to s2attn_bwd, but it skips the RoPE + PI pass (one read of q, k and one write of the
+ * rotated q~, k~ and of the (cos, sin) table) and reads those from the workspace instead.
+ * Precondition, not checked: `workspace` is the one s2attn_fwd used for these same q, k
+ * and shape/pi_scale/rope_base/dtype arguments, and neither it (beyond the status word) nor
+ * q, k changed since. This is the training-loop order (forward, then backward of the same
+ * batch); the method is unchanged, the rotation is computed once per step instead of twice
+ * ("LongLoRA: Efficient 100k Context LLM Fine-Tuning Guide", Step 1 applies RoPE once). The
+ * status word is reset at the start, as in every other call. */
+S2_API s2_status s2attn_bwd_after_fwd(const void* q, const void* k, const void* v,
+                                      const void* o, const float* lse, const void* dout,
+                                      void* dq, void* dk, void* dv, int B, int N, int H_q,
+                                      int H_kv, int d, int G, int causal, float pi_scale,
+                                      float rope_base, int dtype, void* workspace,
+                                      size_t ws_bytes, void* cuda_stream);
+
 /* Bytes of the fixed scratch array that s2attn_fwd_noalloc uses on each device. */
 #define S2ATTN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 

@@ -244,10 +244,16 @@ s2_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, float
   return to_status(enqueue_forward(p, dtype, static_cast<cudaStream_t>(cuda_stream)));
 }
 
-s2_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
-                     const void* dout, void* dq, void* dk, void* dv, int B, int N, int H_q,
-                     int H_kv, int d, int G, int causal, float pi_scale, float rope_base,
-                     int dtype, void* workspace, size_t ws_bytes, void* cuda_stream) {
+namespace s2 {
+namespace {
+
+// Shared body of the two backward entry points. rotate = false reuses the rotated q~, k~
+// and the (cos, sin) table that the forward left in the workspace.
+s2_status backward_impl(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                        int N, int H_q, int H_kv, int d, int G, int causal, float pi_scale,
+                        float rope_base, int dtype, void* workspace, size_t ws_bytes,
+                        void* cuda_stream, bool rotate) {
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return S2_ERR_NULL;
   s2_status st = common_checks(B, N, H_q, H_kv, d, G, causal, pi_scale, rope_base, dtype,
                                workspace, ws_bytes);
@@ -260,7 +266,8 @@ s2_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o,
   p.dout = dout; p.dq = dq; p.dk = dk; p.dv = dv;
   const bool bf16 = dtype == S2_BF16;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-  cudaError_t e = timed_launch(kRopePi, s, [&] { return launch_rope_pi(p, bf16, s); });
+  cudaError_t e = cudaSuccess;
+  if (rotate) e = timed_launch(kRopePi, s, [&] { return launch_rope_pi(p, bf16, s); });
   if (e == cudaSuccess)
     e = timed_launch(kBwdRowsum, s, [&] { return launch_bwd_rowsum(p, bf16, s); });
   if (e != cudaSuccess) return to_status(e);
@@ -273,6 +280,26 @@ s2_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o,
       e = timed_launch(kBwdDqSimt, s, [&] { return launch_simt_dq(p, bf16, s); });
   }
   return to_status(e);
+}
+
+}  // namespace
+}  // namespace s2
+
+s2_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, int B, int N, int H_q,
+                     int H_kv, int d, int G, int causal, float pi_scale, float rope_base,
+                     int dtype, void* workspace, size_t ws_bytes, void* cuda_stream) {
+  return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, N, H_q, H_kv, d, G, causal,
+                       pi_scale, rope_base, dtype, workspace, ws_bytes, cuda_stream, true);
+}
+
+s2_status s2attn_bwd_after_fwd(const void* q, const void* k, const void* v, const void* o,
+                               const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                               int B, int N, int H_q, int H_kv, int d, int G, int causal,
+                               float pi_scale, float rope_base, int dtype, void* workspace,
+                               size_t ws_bytes, void* cuda_stream) {
+  return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, N, H_q, H_kv, d, G, causal,
+                       pi_scale, rope_base, dtype, workspace, ws_bytes, cuda_stream, false);
 }
 
 s2_status s2attn_device_status(void* workspace, size_t ws_bytes, void* cuda_stream) {

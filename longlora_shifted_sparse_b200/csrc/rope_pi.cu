@@ -17,10 +17,8 @@
 namespace s2 {
 
 template <typename T>
-__device__ inline void rotate_vec(const T* __restrict__ src, T* __restrict__ dst,
-                                  const float2* __restrict__ cs_row) {
+__device__ inline uint4 rotate_vec(uint4 raw, const float2* __restrict__ cs_row) {
   constexpr int V = 16 / sizeof(T);
-  uint4 raw = *reinterpret_cast<const uint4*>(src);
   const T* x = reinterpret_cast<const T*>(&raw);
   uint4 out_raw;
   T* y = reinterpret_cast<T*>(&out_raw);
@@ -31,17 +29,36 @@ __device__ inline void rotate_vec(const T* __restrict__ src, T* __restrict__ dst
     y[2 * t] = from_f32<T>(fmaf(x0, c.x, -x1 * c.y));
     y[2 * t + 1] = from_f32<T>(fmaf(x0, c.y, x1 * c.x));
   }
-  *reinterpret_cast<uint4*>(dst) = out_raw;
+  return out_raw;
 }
 
+// The loads of a token's q and k vectors are issued first (kBatch per thread in flight),
+// the fp64 angles are computed while they are in flight, then the vectors are rotated and
+// stored: the kernel is bound by HBM, so it needs many loads outstanding per SM.
 template <typename T>
 __global__ void __launch_bounds__(256) rope_pi_kernel(Params p) {
   extern __shared__ float2 s_cs[];
   constexpr int V = 16 / sizeof(T);
+  constexpr int kBatch = 4;
   const int half = p.d / 2;
   const int tok = blockIdx.x;
   const int b = tok / p.N, n = tok - b * p.N;
   if (tok == 0 && threadIdx.x == 0) *p.status = 0u;  // each call starts with a clean status
+
+  const uint4* q = reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) +
+                                                  (size_t)tok * p.Hq * p.d);
+  const uint4* k = reinterpret_cast<const uint4*>(static_cast<const T*>(p.k) +
+                                                  (size_t)tok * p.Hkv * p.d);
+  T* qr = static_cast<T*>(p.qr);
+  T* kr = static_cast<T*>(p.kr);
+  const int vq = p.Hq * p.d / V, vk = p.Hkv * p.d / V, nv = vq + vk;
+
+  uint4 raw[kBatch];
+#pragma unroll
+  for (int u = 0; u < kBatch; u++) {
+    const int e = threadIdx.x + u * blockDim.x;
+    if (e < nv) raw[u] = __ldcs(e < vq ? q + e : k + (e - vq));
+  }
   for (int i = threadIdx.x; i < half; i += blockDim.x) {
     double theta = pow((double)p.rope_base, -2.0 * (double)i / (double)p.d);
     double phi = ((double)n / (double)p.pi_scale) * theta;
@@ -53,19 +70,25 @@ __global__ void __launch_bounds__(256) rope_pi_kernel(Params p) {
   }
   __syncthreads();
 
-  const T* q = static_cast<const T*>(p.q) + (size_t)tok * p.Hq * p.d;
-  const T* k = static_cast<const T*>(p.k) + (size_t)tok * p.Hkv * p.d;
-  T* qr = static_cast<T*>(p.qr);
-  T* kr = static_cast<T*>(p.kr);
-  const int vq = p.Hq * p.d / V, vk = p.Hkv * p.d / V;
-  for (int e = threadIdx.x; e < vq + vk; e += blockDim.x) {
-    const bool is_q = e < vq;
-    const int ee = is_q ? e : e - vq;
-    const int h = ee * V / p.d, c0 = ee * V - h * p.d;
-    const int H = is_q ? p.Hq : p.Hkv;
-    const T* src = (is_q ? q : k) + (size_t)ee * V;
-    T* dst = (is_q ? qr : kr) + (((size_t)b * H + h) * p.N + n) * p.d + c0;
-    rotate_vec<T>(src, dst, s_cs + c0 / 2);
+  for (int e0 = threadIdx.x;; e0 += kBatch * blockDim.x) {
+#pragma unroll
+    for (int u = 0; u < kBatch; u++) {
+      const int e = e0 + u * blockDim.x;
+      if (e < nv) {
+        const bool is_q = e < vq;
+        const int ee = is_q ? e : e - vq;
+        const int h = ee * V / p.d, c0 = ee * V - h * p.d;
+        const int H = is_q ? p.Hq : p.Hkv;
+        T* dst = (is_q ? qr : kr) + (((size_t)b * H + h) * p.N + n) * p.d + c0;
+        *reinterpret_cast<uint4*>(dst) = rotate_vec<T>(raw[u], s_cs + c0 / 2);
+      }
+    }
+    if (e0 + kBatch * (int)blockDim.x >= nv) break;
+#pragma unroll
+    for (int u = 0; u < kBatch; u++) {  // next batch (tokens with more than 1024 vectors)
+      const int e = e0 + kBatch * blockDim.x + u * blockDim.x;
+      if (e < nv) raw[u] = __ldcs(e < vq ? q + e : k + (e - vq));
+    }
   }
 }
 

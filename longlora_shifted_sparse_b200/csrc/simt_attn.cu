@@ -91,6 +91,9 @@ template <typename T, int DPL>
 __global__ void __launch_bounds__(256) bwd_rowsum_kernel(Params p) {
   const int lane = threadIdx.x & 31;
   const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  // the backward's first kernel when it reuses the forward's rotation: the call starts
+  // with a clean status word (no kernel of this launch reads it)
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.status = 0u;
   if (warp >= (long)p.B * p.N * p.Hq) return;
   const int h = (int)(warp % p.Hq);
   const long bm = warp / p.Hq;
@@ -101,6 +104,50 @@ __global__ void __launch_bounds__(256) bwd_rowsum_kernel(Params p) {
   load_row<T, DPL>(static_cast<const T*>(p.o) + off, c, lane);
   const float D = row_dot<DPL>(a, c);
   if (lane == 0) p.Dsum[((size_t)b * p.Hq + h) * p.N + m] = D;
+}
+
+// D = rowsum(dO * O) for bf16 rows of 128 (the tensor-core path's shape), HBM-bound: rows
+// [B][N][Hq] are contiguous, so 8 consecutive rows (2 KB) go to one warp, a half-warp per
+// row and 16 bytes per lane, with all 8 loads of dO and O issued before the first use.
+__global__ void __launch_bounds__(256) bwd_rowsum_bf16_d128_kernel(Params p) {
+  constexpr int kRowsPerWarp = 8;
+  const int lane = threadIdx.x & 31, half = lane >> 4, chunk = lane & 15;
+  const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.status = 0u;  // see bwd_rowsum_kernel
+  const long rows = (long)p.B * p.N * p.Hq;
+  const long r0 = warp * kRowsPerWarp;
+  if (r0 >= rows) return;
+  const uint4* dO = reinterpret_cast<const uint4*>(p.dout);
+  const uint4* O = reinterpret_cast<const uint4*>(p.o);
+  uint4 a[kRowsPerWarp / 2], c[kRowsPerWarp / 2];
+#pragma unroll
+  for (int i = 0; i < kRowsPerWarp / 2; i++) {
+    const long r = r0 + 2 * i + half;
+    const long e = r < rows ? r * 16 + chunk : 0;  // 16 uint4 per row
+    a[i] = __ldcs(dO + e);
+    c[i] = __ldcs(O + e);
+  }
+#pragma unroll
+  for (int i = 0; i < kRowsPerWarp / 2; i++) {
+    const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a[i]);
+    const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&c[i]);
+    float acc = 0.f;
+#pragma unroll
+    for (int t = 0; t < 4; t++) {
+      const float2 xf = __bfloat1622float2(x[t]), yf = __bfloat1622float2(y[t]);
+      acc = fmaf(xf.x, yf.x, acc);
+      acc = fmaf(xf.y, yf.y, acc);
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    const long r = r0 + 2 * i + half;
+    if (chunk == 0 && r < rows) {
+      const int h = (int)(r % p.Hq);
+      const long bm = r / p.Hq;
+      const int m = (int)(bm % p.N), b = (int)(bm / p.N);
+      p.Dsum[((size_t)b * p.Hq + h) * p.N + m] = acc;
+    }
+  }
 }
 
 template <typename T, int DPL>
@@ -239,6 +286,11 @@ cudaError_t launch_simt_fwd(const Params& p, bool bf16, cudaStream_t st) {
 }
 
 cudaError_t launch_bwd_rowsum(const Params& p, bool bf16, cudaStream_t st) {
+  if (bf16 && p.d == 128) {
+    const long warps = ((long)p.B * p.Hq * p.N + 7) / 8;
+    bwd_rowsum_bf16_d128_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p);
+    return cudaGetLastError();
+  }
   dim3 grid = warp_grid((long)p.B * p.Hq * p.N);
   S2_DISPATCH_TYPE(bwd_rowsum_kernel, bf16, grid, st, p)
   return cudaGetLastError();

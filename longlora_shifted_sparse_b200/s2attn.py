@@ -39,6 +39,8 @@ _lib.s2attn_fwd.argtypes = [_vp] * 5 + _SHAPE + [_vp, _sz, _vp]
 _lib.s2attn_fwd.restype = _i
 _lib.s2attn_bwd.argtypes = [_vp] * 9 + _SHAPE + [_vp, _sz, _vp]
 _lib.s2attn_bwd.restype = _i
+_lib.s2attn_bwd_after_fwd.argtypes = [_vp] * 9 + _SHAPE + [_vp, _sz, _vp]
+_lib.s2attn_bwd_after_fwd.restype = _i
 _lib.s2attn_fwd_noalloc.argtypes = [_vp] * 5 + _SHAPE + [_vp]
 _lib.s2attn_fwd_noalloc.restype = _i
 _lib.s2attn_kernel_path.argtypes = [_i] * 8
@@ -65,6 +67,7 @@ _lib.s2attn_profile_dropped.restype = _i
 s2attn_workspace_bytes = _lib.s2attn_workspace_bytes
 s2attn_fwd = _lib.s2attn_fwd
 s2attn_bwd = _lib.s2attn_bwd
+s2attn_bwd_after_fwd = _lib.s2attn_bwd_after_fwd
 s2attn_fwd_noalloc = _lib.s2attn_fwd_noalloc
 s2attn_kernel_path = _lib.s2attn_kernel_path
 s2attn_device_status = _lib.s2attn_device_status
@@ -153,18 +156,24 @@ def forward(q, k, v, G: int, pi_scale: float, rope_base: float = 10000.0, causal
 
 
 def backward(q, k, v, o, lse, dout, G: int, pi_scale: float, rope_base: float = 10000.0,
-             causal: bool = True, ws=None, grads=None):
-    """Returns (dq, dk, dv) for the forward that produced (o, lse)."""
+             causal: bool = True, ws=None, grads=None, after_forward: bool = False):
+    """Returns (dq, dk, dv) for the forward that produced (o, lse).
+
+    after_forward=True calls s2attn_bwd_after_fwd: `ws` must then be the workspace the
+    forward of these q, k used, unchanged since (it holds their rotation)."""
     import torch
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
     dt = _dtype_code(q)
     if ws is None:
+        if after_forward:
+            raise ValueError("after_forward=True needs the forward's workspace")
         ws = workspace(B, N, Hq, Hkv, d, dt, q.device)
     if grads is None:
         grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
     dq, dk, dv = grads
-    check(s2attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+    fn = s2attn_bwd_after_fwd if after_forward else s2attn_bwd
+    check(fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                      dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                      B, N, Hq, Hkv, d, G, int(causal), pi_scale, rope_base, dt,
                      ws.data_ptr(), ws.numel(), _stream_ptr(q.device)))
@@ -185,16 +194,21 @@ def _make_function():
         @staticmethod
         def forward(ctx, q, k, v, G, pi_scale, rope_base=10000.0, causal=True):
             q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
-            o, lse = forward(q, k, v, G, pi_scale, rope_base, causal)
-            ctx.save_for_backward(q, k, v, o, lse)
+            B, N, Hq, d = q.shape
+            ws = workspace(B, N, Hq, k.shape[2], d, _dtype_code(q), q.device)
+            o, lse = forward(q, k, v, G, pi_scale, rope_base, causal, ws=ws)
+            # the workspace keeps the rotated q, k for the backward (q, k are saved too, so
+            # autograd's version check catches an in-place change in between)
+            ctx.save_for_backward(q, k, v, o, lse, ws)
             ctx.args = (G, pi_scale, rope_base, causal)
             return o
 
         @staticmethod
         def backward(ctx, do):
-            q, k, v, o, lse = ctx.saved_tensors
+            q, k, v, o, lse, ws = ctx.saved_tensors
             G, pi_scale, rope_base, causal = ctx.args
-            dq, dk, dv = backward(q, k, v, o, lse, do.contiguous(), G, pi_scale, rope_base, causal)
+            dq, dk, dv = backward(q, k, v, o, lse, do.contiguous(), G, pi_scale, rope_base, causal,
+                                  ws=ws, after_forward=True)
             return dq, dk, dv, None, None, None, None
 
     return S2AttnFunction

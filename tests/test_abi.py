@@ -128,3 +128,13 @@ def test_flops_model():
     f = flops.attention_fwd_flops(1, 32768, 32, 128, 8192, True)
     assert f == 4 * 32 * 32768 * 8192 * 128 / 2
     assert flops.attention_bwd_flops(1, 32768, 32, 128, 8192, True) == 2.5 * f
+
+
+def test_bwd_after_fwd_rejects_bad_arguments(lib):
+    a = (1, 256, 4, 4, 64, 64, 1, 2.0, 10000.0, lib.S2_FP32)
+    f = lib.s2attn_bwd_after_fwd
+    assert f(P, P, P, P, P, P, None, P, P, *a, P, 1 << 40, None) == lib.S2_ERR_NULL
+    assert f(P, P, P, P, P, P, P, P, P, 1, 100, 4, 4, 64, 64, 1, 2.0, 10000.0, lib.S2_FP32,
+             P, 1 << 40, None) == lib.S2_ERR_SHAPE
+    assert f(P, P, P, P, P, P, P + 4, P, P, *a, P, 1 << 40, None) == lib.S2_ERR_ALIGN
+    assert f(P, P, P, P, P, P, P, P, P, *a, P, 16, None) == lib.S2_ERR_WORKSPACE

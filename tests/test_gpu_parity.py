@@ -202,6 +202,36 @@ def test_device_status_and_profiler(s2):
     assert all(ms > 0 for _, ms in summary.values())
 
 
+@pytest.mark.parametrize("case", [
+    # name, B, N, Hq, Hkv, d, G, s, dtype
+    ("tcgen05_gqa", 1, 1024, 4, 2, 128, 256, 2.0, "bf16"),
+    ("cuda_core_f32", 1, 256, 4, 4, 64, 64, 2.0, "f32"),
+], ids=lambda c: c[0])
+def test_backward_after_forward_is_bit_identical(s2, case):
+    """s2attn_bwd_after_fwd reuses the rotated q, k that the forward left in its workspace;
+    s2attn_bwd rotates them again into a fresh workspace. The rotation is deterministic and
+    so are the backward kernels (no atomics), so the gradients must agree bit for bit; the
+    autograd wrapper, which takes the first route, must agree as well."""
+    name, B, N, Hq, Hkv, d, G, s, dt = case
+    q, k, v, do = synth.s2attn_inputs(77, B, N, Hq, Hkv, d, 0.5 if dt == "bf16" else 1.0, dt)
+    tq, tk, tv, tdo = (H.to_device(x, dt) for x in (q, k, v, do))
+    code = s2.S2_BF16 if dt == "bf16" else s2.S2_FP32
+    ws = s2.workspace(B, N, Hq, Hkv, d, code, tq.device)
+    o, lse = s2.forward(tq, tk, tv, G, s, ws=ws)
+    g_after = s2.backward(tq, tk, tv, o, lse, tdo, G, s, ws=ws, after_forward=True)
+    g_fresh = s2.backward(tq, tk, tv, o, lse, tdo, G, s)
+    torch.cuda.synchronize()
+    assert s2.device_status(ws) == s2.S2_OK
+    for a, b in zip(g_after, g_fresh):
+        assert torch.equal(a, b)
+    xs = [t.clone().requires_grad_(True) for t in (tq, tk, tv)]
+    out = s2.s2_attention(xs[0], xs[1], xs[2], G, s)
+    out.backward(tdo)
+    assert torch.equal(out.detach(), o)
+    for x, g in zip(xs, g_fresh):
+        assert torch.equal(x.grad, g)
+
+
 def test_softmax_rescale_paths(s2):
     """Scores whose running row max climbs by well over the forward's rescale threshold
     (2^8) along each group, so that the exact-max exchange, the power-of-two rescale of P
