@@ -30,12 +30,14 @@
 //   The GQA sum over query heads happens in the TMEM accumulators (no atomics).
 //   Epilogue: dk = R^T (dK / sqrt(d)), dv = dV, bf16, at the key tokens' original rows.
 // dQ pass: one CTA per 128-row query tile (b, head, group, qt). For every key tile j <= qt:
-//   S = Q K^T (TMEM [0,128)), dP = dO V^T ([128,256)), dS = P (dP - D) bf16 over dP
-//   (the first 32 of each math warp's 64 columns), dQ += dS K (TS MMA, [256,384)).
-//   Epilogue: dq = R^T (dQ / sqrt(d)), bf16, at the query tokens' original rows.
+//   S = Q K^T (TMEM [0,128)), dP = dO V^T into one of two buffers ([128,256), [256,384)),
+//   dS = P (dP - D) bf16 over that dP (the first 32 of each math warp's 64 columns),
+//   dQ += dS K (TS MMA, [384,512)). Two MMA issuers (warp 1: S and dP; warp 2: dQ), see
+//   the kernel. Epilogue: dq = R^T (dQ / sqrt(d)), bf16, at the query tokens' original rows.
 // CTAs are launched head-group-major so that the CTAs running together share the tiles
 // they stream (L2 reuse). Roles: warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
-// warps 4..11 the per-row math. Every wait is bounded (see sm100.cuh).
+// (dQ pass: warp 2 second MMA issuer), warps 4..11 the per-row math. Every wait is bounded
+// (see sm100.cuh).
 #include "common.cuh"
 #include "sm100.cuh"
 #include "tc_kernels.h"
@@ -444,20 +446,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ================================================================================ dQ
 
-// smem: K stages 0..3 | V stages 0..2 (Q~ and dO of the CTA's query tile live in TMEM)
-constexpr int kKStages = 4, kVStages = 3;
-constexpr uint32_t kQOffK = 0;
-constexpr uint32_t kQOffV = kKStages * kTileBytes;
-constexpr uint32_t kQSmem = (kKStages + kVStages) * kTileBytes + 1024;
+// smem: Q | dO | K stages 0..2 | V stages 0..1
+constexpr int kKStages = 3, kVStages = 2;
+constexpr uint32_t kQOffQ = 0;
+constexpr uint32_t kQOffDO = kTileBytes;
+constexpr uint32_t kQOffK = 2 * kTileBytes;
+constexpr uint32_t kQOffV = (2 + kKStages) * kTileBytes;
+constexpr uint32_t kQSmem = (2 + kKStages + kVStages) * kTileBytes + 1024;
 
 struct DqBarriers {
-  uint64_t qdo_ready;
+  uint64_t q_full;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full, s_consumed, dp_full, ds_ready;
-  uint64_t acc_done, drain;
+  uint64_t s_full, s_consumed;
+  uint64_t dp_full[2], ds_ready[2], dq_done[2];
+  uint64_t acc_done, drain[2];
 };
 
+// Two MMA issuers (one thread issues a tcgen05.mma only every ~45 cycles, against 64 cycles
+// of tensor work per 128 x 128 x 16 MMA, and the dQ pass has 24 MMAs per key tile):
+//   warp 1 (TMEM owner): S(j) = Q K_j^T into TMEM [0,128) once the math warps hold S(j-1)
+//            in registers, then dP(j) = dO V_j^T into buffer j % 2 ([128,256) / [256,384))
+//            once dQ(j-2) has read the dS that buffer held;
+//   warp 2:  dQ += dS(j) K_j ([384,512)) once the math warps published dS(j).
+// With dP double-buffered, S and dP of key tile j+1 are computed while the math warps work
+// on tile j, so the math never waits for the tensor cores in the steady state.
 __global__ void __launch_bounds__(kThreads, 1)
     tc_dq_kernel(const Params p, const __grid_constant__ CUtensorMap tm_q,
                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -487,10 +500,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   Abort ab{&abort_flag, p.status};
   if (threadIdx.x == 0) {
     abort_flag = *reinterpret_cast<volatile unsigned*>(p.status) != 0u;
-    mbar_init(smem_addr(&bars.qdo_ready), kMathThreads);
+    mbar_init(smem_addr(&bars.q_full), 1);
     for (int s = 0; s < kKStages; s++) {
       mbar_init(smem_addr(&bars.k_full[s]), 1);
-      mbar_init(smem_addr(&bars.k_empty[s]), 1);
+      mbar_init(smem_addr(&bars.k_empty[s]), 2);  // S(j) and dQ(j) both read K_j
     }
     for (int s = 0; s < kVStages; s++) {
       mbar_init(smem_addr(&bars.v_full[s]), 1);
@@ -498,10 +511,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(smem_addr(&bars.s_full), 1);
     mbar_init(smem_addr(&bars.s_consumed), kMathThreads);
-    mbar_init(smem_addr(&bars.dp_full), 1);
-    mbar_init(smem_addr(&bars.ds_ready), kMathThreads);
+    for (int s = 0; s < 2; s++) {
+      mbar_init(smem_addr(&bars.ds_ready[s]), kMathThreads);
+      mbar_init(smem_addr(&bars.dp_full[s]), 1);
+      mbar_init(smem_addr(&bars.dq_done[s]), 1);
+      mbar_init(smem_addr(&bars.drain[s]), 1);
+    }
     mbar_init(smem_addr(&bars.acc_done), 1);
-    mbar_init(smem_addr(&bars.drain), 1);
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(smem_addr(&tmem_base_sh), kTmemCols);
@@ -509,15 +525,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
-  // TMEM: S | dP (dS written over it) | dQ accumulator | Q~ and dO as bf16 A operands
-  const uint32_t colS = 0, colDP = 128, colDQ = 256, colQ = 384, colDO = 448;
+  const uint32_t colS = 0, colDP = 128, colDQ = 384;  // dP buffers at colDP, colDP + 128
+  const uint32_t sQ = smem_addr(smem + kQOffQ), sDO = smem_addr(smem + kQOffDO);
   const bool skip = abort_flag != 0;
 
   if (skip) {
   } else if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      const uint32_t qb = smem_addr(&bars.q_full);
+      mbar_arrive_expect_tx(qb, 2 * kTileBytes);
+      const int qrow = (b * p.Hq + h) * p.N + mq0;
+      tma_load_2d(sQ, &tm_q, qb, 0, qrow);
+      tma_load_2d(sQ + kBoxBytes, &tm_q, qb, 64, qrow);
+      tma_load_3d(sDO, &tm_do, qb, 0, h, b * p.N + mq0);
+      tma_load_3d(sDO + kBoxBytes, &tm_do, qb, 64, h, b * p.N + mq0);
       int nk_issued = 0, nv_issued = 0;
       for (int j = 0; j < nkv; j++) {
         const int mk = src_row(g * p.G + j * kTile, sh, p.G, p.N);
@@ -538,108 +564,98 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sVs + kBoxBytes, &tm_v, vb, 64, kvh, b * p.N + mk);
         nv_issued = j + 1;
       }
+      // the last loads in flight land before the CTA can exit (own time limit, no abort)
       int no_abort = 0;
       Abort local{&no_abort, p.status};
       for (int j = nk_issued - 1; j >= 0 && j >= nk_issued - kKStages; j--)
         mbar_wait(smem_addr(&bars.k_full[j % kKStages]), (j / kKStages) & 1, local);
       for (int j = nv_issued - 1; j >= 0 && j >= nv_issued - kVStages; j--)
         mbar_wait(smem_addr(&bars.v_full[j % kVStages]), (j / kVStages) & 1, local);
+      mbar_wait(qb, 0, local);
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer: S, dP
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
-      const uint32_t idesc_g = idesc_bf16_f32(kTile, kD, false, true);
       // Descriptors are built once; a stage or a k-step only adds a constant to the start
       // address field (bytes / 16; shared memory stays below 256 KB, so nothing carries out).
+      const uint64_t dQd = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t dDOd = smem_desc_sw128(sDO, 16, 1024);
       const uint64_t dK0 = smem_desc_sw128(smem_addr(smem + kQOffK), 16, 1024);
-      const uint64_t dKm0 = smem_desc_sw128(smem_addr(smem + kQOffK), kBoxBytes, 1024);
       const uint64_t dV0 = smem_desc_sw128(smem_addr(smem + kQOffV), 16, 1024);
-      auto issue_s = [&](int j) -> bool {  // S(j) = Q K_j^T, Q from TMEM
-        const int sk = j % kKStages;
-        if (!mbar_wait(smem_addr(&bars.k_full[sk]), (j / kKStages) & 1, ab)) return false;
-        tc_fence_after();
-        const uint64_t dk = opaque64(dK0) + (uint64_t)(sk * kTileDesc);
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; kk++)
-          mma_ts(tmem + colS, tmem + colQ + kk * 8, dk + kmajor_koff(kk), idesc_s, kk > 0);
-        mma_commit(smem_addr(&bars.s_full));
-        return true;
-      };
-      auto issue_dp = [&](int j) -> bool {  // dP(j) = dO V_j^T, dO from TMEM
-        const int sv = j % kVStages;
-        if (!mbar_wait(smem_addr(&bars.v_full[sv]), (j / kVStages) & 1, ab)) return false;
-        tc_fence_after();
-        const uint64_t dv = opaque64(dV0) + (uint64_t)(sv * kTileDesc);
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; kk++)
-          mma_ts(tmem + colDP, tmem + colDO + kk * 8, dv + kmajor_koff(kk), idesc_s, kk > 0);
-        mma_commit(smem_addr(&bars.dp_full));
-        mma_commit(smem_addr(&bars.v_empty[sv]));
-        return true;
-      };
-      // issue order: S(0) dP(0) S(1) | dQ(0) dP(1) S(2) | dQ(1) dP(2) S(3) | ...
-      // (see the dK/dV pass: the MMAs the next math phase waits for go first)
-      bool ok = mbar_wait(smem_addr(&bars.qdo_ready), 0, ab);
+      bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
       tc_fence_after();
-      if (ok) ok = issue_s(0) && issue_dp(0);
-      if (ok && nkv > 1) ok = mbar_wait(smem_addr(&bars.s_consumed), 0, ab) && issue_s(1);
       for (int j = 0; ok && j < nkv; j++) {
-        const uint32_t ph = j & 1;
-        if (!mbar_wait(smem_addr(&bars.ds_ready), ph, ab)) break;
+        // S(j) = Q K_j^T, once the math warps hold S(j-1) in registers
+        if (j >= 1 && !mbar_wait(smem_addr(&bars.s_consumed), (j - 1) & 1, ab)) break;
+        const int sk = j % kKStages;
+        if (!mbar_wait(smem_addr(&bars.k_full[sk]), (j / kKStages) & 1, ab)) break;
         tc_fence_after();
-        const uint64_t dkm = opaque64(dKm0) + (uint64_t)((j % kKStages) * kTileDesc);
+        {
+          const uint64_t dk = opaque64(dK0) + (uint64_t)(sk * kTileDesc);
+          const uint64_t dq = opaque64(dQd);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; kk++)
+            mma_ss(tmem + colS, dq + kmajor_koff(kk), dk + kmajor_koff(kk), idesc_s, kk > 0);
+        }
+        mma_commit(smem_addr(&bars.s_full));
+        mma_commit(smem_addr(&bars.k_empty[sk]));
+        // dP(j) = dO V_j^T into buffer j % 2, once dQ(j-2) has read the dS it held
+        if (j >= 2 && !mbar_wait(smem_addr(&bars.dq_done[j & 1]), ((j - 2) >> 1) & 1, ab)) break;
+        const int sv = j % kVStages;
+        if (!mbar_wait(smem_addr(&bars.v_full[sv]), (j / kVStages) & 1, ab)) break;
+        tc_fence_after();
+        {
+          const uint64_t dv = opaque64(dV0) + (uint64_t)(sv * kTileDesc);
+          const uint64_t ddo = opaque64(dDOd);
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; kk++)
+            mma_ss(tmem + colDP + (j & 1) * 128, ddo + kmajor_koff(kk), dv + kmajor_koff(kk),
+                   idesc_s, kk > 0);
+        }
+        mma_commit(smem_addr(&bars.dp_full[j & 1]));
+        mma_commit(smem_addr(&bars.v_empty[sv]));
+      }
+      mma_commit(smem_addr(&bars.drain[0]));
+      int no_abort = 0;
+      Abort local{&no_abort, p.status};
+      mbar_wait(smem_addr(&bars.drain[0]), 0, local);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------------ MMA issuer: dQ
+    if (lane == 0) {
+      const uint32_t idesc_g = idesc_bf16_f32(kTile, kD, false, true);
+      const uint64_t dKm0 = smem_desc_sw128(smem_addr(smem + kQOffK), kBoxBytes, 1024);
+      for (int j = 0; j < nkv; j++) {
+        // dQ += dS(j) K_j, dS read from dP buffer j % 2
+        if (!mbar_wait(smem_addr(&bars.ds_ready[j & 1]), (j >> 1) & 1, ab)) break;
+        const int sk = j % kKStages;
+        if (!mbar_wait(smem_addr(&bars.k_full[sk]), (j / kKStages) & 1, ab)) break;
+        tc_fence_after();
+        const uint64_t dkm = opaque64(dKm0) + (uint64_t)(sk * kTileDesc);
         const uint32_t acc0 = j > 0;
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; kk++)
-          mma_ts(tmem + colDQ, tmem + packed_col(colDP, kk, 16), dkm + mn_koff(kk), idesc_g,
-                 kk ? 1u : acc0);
-        mma_commit(smem_addr(&bars.k_empty[j % kKStages]));
-        if (j + 1 < nkv && !issue_dp(j + 1)) break;
-        if (j + 2 < nkv) {
-          if (!mbar_wait(smem_addr(&bars.s_consumed), (j + 1) & 1, ab)) break;
-          if (!issue_s(j + 2)) break;
-        }
+          mma_ts(tmem + colDQ, tmem + packed_col(colDP + (j & 1) * 128, kk, 16),
+                 dkm + mn_koff(kk), idesc_g, kk ? 1u : acc0);
+        mma_commit(smem_addr(&bars.dq_done[j & 1]));
+        mma_commit(smem_addr(&bars.k_empty[sk]));
       }
       mma_commit(smem_addr(&bars.acc_done));
-      mma_commit(smem_addr(&bars.drain));
+      mma_commit(smem_addr(&bars.drain[1]));
       int no_abort = 0;
       Abort local{&no_abort, p.status};
-      mbar_wait(smem_addr(&bars.drain), 0, local);
+      mbar_wait(smem_addr(&bars.drain[1]), 0, local);
     }
   } else if (warp >= 4) {
+    // ------------------------------------------------------------------ per query row math
     const int quarter = warp & 3;
     const int c0 = ((warp - 4) >> 2) * 64;  // this warp's 64 key columns of the tile
     const int row = quarter * 32 + lane;    // query row inside the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + colS + c0;
-    const uint32_t tDP = tmem + lane_off + colDP + c0;
     const int m = src_row(g * p.G + qt * kTile + row, sh, p.G, p.N);
     const size_t lrow = ((size_t)b * p.Hq + h) * p.N + m;
-    // This thread's half row (d = c0 .. c0+63) of Q~ and of dO into TMEM, as the bf16 A
-    // operands of S = Q K^T and dP = dO V^T: column j of a row holds elements 2j, 2j+1,
-    // which is the order of the row in memory.
-    {
-      const uint4* qsrc = reinterpret_cast<const uint4*>(
-          static_cast<const __nv_bfloat16*>(p.qr) + lrow * kD + c0);
-      const uint4* dsrc = reinterpret_cast<const uint4*>(
-          static_cast<const __nv_bfloat16*>(p.dout) + ((size_t)(b * p.N + m) * p.Hq + h) * kD + c0);
-      uint32_t w[32];
-#pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const uint4 t = __ldg(qsrc + i);
-        w[4 * i] = t.x; w[4 * i + 1] = t.y; w[4 * i + 2] = t.z; w[4 * i + 3] = t.w;
-      }
-      tmem_st32(tmem + lane_off + colQ + c0 / 2, w);
-#pragma unroll
-      for (int i = 0; i < 8; i++) {
-        const uint4 t = __ldg(dsrc + i);
-        w[4 * i] = t.x; w[4 * i + 1] = t.y; w[4 * i + 2] = t.z; w[4 * i + 3] = t.w;
-      }
-      tmem_st32(tmem + lane_off + colDO + c0 / 2, w);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(smem_addr(&bars.qdo_ready));
-    }
     const float nlse2 = -p.lse[lrow] * kLog2e;
     const float Dm = p.Dsum[lrow];
     const float sl2 = p.scale_log2;
@@ -664,11 +680,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           pr[c] = fast_exp2(fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, nlse2));
         pin_regs(pr);
       }
-      ok = mbar_wait(smem_addr(&bars.dp_full), j & 1, ab);
+      ok = mbar_wait(smem_addr(&bars.dp_full[j & 1]), (j >> 1) & 1, ab);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
       {
+        const uint32_t tDP = tmem + lane_off + colDP + (j & 1) * 128 + c0;
         uint32_t x0[32], x1[32];
         tmem_ld32(tDP, x0);
         tmem_ld32(tDP + 32, x1);
@@ -688,7 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_addr(&bars.ds_ready));
+      mbar_arrive(smem_addr(&bars.ds_ready[j & 1]));
     }
     if (ok) {
       ok = mbar_wait(smem_addr(&bars.acc_done), 0, ab);
@@ -719,7 +736,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, kTmemCols);
   }
 }
-
 cudaError_t make_bwd_maps(const Params& p, CUtensorMap* tq, CUtensorMap* tk, CUtensorMap* tv,
                           CUtensorMap* tdo) {
   cudaError_t e;
