@@ -32,11 +32,11 @@
 // dQ pass: one CTA per 128-row query tile (b, head, group, qt). For every key tile j <= qt:
 //   S = Q K^T (TMEM [0,128)), dP = dO V^T into one of two buffers ([128,256), [256,384)),
 //   dS = P (dP - D) bf16 over that dP (the first 32 of each math warp's 64 columns),
-//   dQ += dS K (TS MMA, [384,512)). Two MMA issuers (warp 1: S and dP; warp 2: dQ), see
-//   the kernel. Epilogue: dq = R^T (dQ / sqrt(d)), bf16, at the query tokens' original rows.
+//   dQ += dS K (TS MMA, [384,512)). Three MMA issuers (warp 1: S, warp 2: dP, warp 3: dQ),
+//   see the kernel. Epilogue: dq = R^T (dQ / sqrt(d)), bf16, at the query tokens' original rows.
 // CTAs are launched head-group-major so that the CTAs running together share the tiles
 // they stream (L2 reuse). Roles: warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
-// (dQ pass: warp 2 second MMA issuer), warps 4..11 the per-row math. Every wait is bounded
+// (dQ pass: warps 1..3 MMA issuers), warps 4..11 the per-row math. Every wait is bounded
 // (see sm100.cuh).
 #include "common.cuh"
 #include "sm100.cuh"
@@ -460,15 +460,17 @@ struct DqBarriers {
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full, s_consumed;
   uint64_t dp_full[2], ds_ready[2], dq_done[2];
-  uint64_t acc_done, drain[2];
+  uint64_t acc_done, drain[3];
 };
 
-// Two MMA issuers (one thread issues a tcgen05.mma only every ~45 cycles, against 64 cycles
-// of tensor work per 128 x 128 x 16 MMA, and the dQ pass has 24 MMAs per key tile):
+// Three MMA issuers, one thread each (a thread issues a tcgen05.mma only every ~45 cycles,
+// against 64 cycles of tensor work per 128 x 128 x 16 MMA, and slower still while math
+// warps share its scheduler; the dQ pass has 24 MMAs per key tile):
 //   warp 1 (TMEM owner): S(j) = Q K_j^T into TMEM [0,128) once the math warps hold S(j-1)
-//            in registers, then dP(j) = dO V_j^T into buffer j % 2 ([128,256) / [256,384))
-//            once dQ(j-2) has read the dS that buffer held;
-//   warp 2:  dQ += dS(j) K_j ([384,512)) once the math warps published dS(j).
+//            in registers;
+//   warp 2:  dP(j) = dO V_j^T into buffer j % 2 ([128,256) / [256,384)) once dQ(j-2) has
+//            read the dS that buffer held;
+//   warp 3:  dQ += dS(j) K_j ([384,512)) once the math warps published dS(j).
 // With dP double-buffered, S and dP of key tile j+1 are computed while the math warps work
 // on tile j, so the math never waits for the tensor cores in the steady state.
 __global__ void __launch_bounds__(kThreads, 1)
@@ -515,8 +517,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_addr(&bars.ds_ready[s]), kMathThreads);
       mbar_init(smem_addr(&bars.dp_full[s]), 1);
       mbar_init(smem_addr(&bars.dq_done[s]), 1);
-      mbar_init(smem_addr(&bars.drain[s]), 1);
     }
+    for (int s = 0; s < 3; s++) mbar_init(smem_addr(&bars.drain[s]), 1);
     mbar_init(smem_addr(&bars.acc_done), 1);
     fence_barrier_init();
   }
@@ -574,47 +576,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(qb, 0, local);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer: S, dP
+    // ------------------------------------------------------------------ MMA issuer: S
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
       // Descriptors are built once; a stage or a k-step only adds a constant to the start
       // address field (bytes / 16; shared memory stays below 256 KB, so nothing carries out).
       const uint64_t dQd = smem_desc_sw128(sQ, 16, 1024);
-      const uint64_t dDOd = smem_desc_sw128(sDO, 16, 1024);
       const uint64_t dK0 = smem_desc_sw128(smem_addr(smem + kQOffK), 16, 1024);
-      const uint64_t dV0 = smem_desc_sw128(smem_addr(smem + kQOffV), 16, 1024);
       bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
-      tc_fence_after();
       for (int j = 0; ok && j < nkv; j++) {
         // S(j) = Q K_j^T, once the math warps hold S(j-1) in registers
         if (j >= 1 && !mbar_wait(smem_addr(&bars.s_consumed), (j - 1) & 1, ab)) break;
         const int sk = j % kKStages;
         if (!mbar_wait(smem_addr(&bars.k_full[sk]), (j / kKStages) & 1, ab)) break;
         tc_fence_after();
-        {
-          const uint64_t dk = opaque64(dK0) + (uint64_t)(sk * kTileDesc);
-          const uint64_t dq = opaque64(dQd);
+        const uint64_t dk = opaque64(dK0) + (uint64_t)(sk * kTileDesc);
+        const uint64_t dq = opaque64(dQd);
 #pragma unroll
-          for (int kk = 0; kk < kD / 16; kk++)
-            mma_ss(tmem + colS, dq + kmajor_koff(kk), dk + kmajor_koff(kk), idesc_s, kk > 0);
-        }
+        for (int kk = 0; kk < kD / 16; kk++)
+          mma_ss(tmem + colS, dq + kmajor_koff(kk), dk + kmajor_koff(kk), idesc_s, kk > 0);
         mma_commit(smem_addr(&bars.s_full));
         mma_commit(smem_addr(&bars.k_empty[sk]));
-        // dP(j) = dO V_j^T into buffer j % 2, once dQ(j-2) has read the dS it held
-        if (j >= 2 && !mbar_wait(smem_addr(&bars.dq_done[j & 1]), ((j - 2) >> 1) & 1, ab)) break;
-        const int sv = j % kVStages;
-        if (!mbar_wait(smem_addr(&bars.v_full[sv]), (j / kVStages) & 1, ab)) break;
-        tc_fence_after();
-        {
-          const uint64_t dv = opaque64(dV0) + (uint64_t)(sv * kTileDesc);
-          const uint64_t ddo = opaque64(dDOd);
-#pragma unroll
-          for (int kk = 0; kk < kD / 16; kk++)
-            mma_ss(tmem + colDP + (j & 1) * 128, ddo + kmajor_koff(kk), dv + kmajor_koff(kk),
-                   idesc_s, kk > 0);
-        }
-        mma_commit(smem_addr(&bars.dp_full[j & 1]));
-        mma_commit(smem_addr(&bars.v_empty[sv]));
       }
       mma_commit(smem_addr(&bars.drain[0]));
       int no_abort = 0;
@@ -622,6 +604,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(smem_addr(&bars.drain[0]), 0, local);
     }
   } else if (warp == 2) {
+    // ------------------------------------------------------------------ MMA issuer: dP
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
+      const uint64_t dDOd = smem_desc_sw128(sDO, 16, 1024);
+      const uint64_t dV0 = smem_desc_sw128(smem_addr(smem + kQOffV), 16, 1024);
+      bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
+      for (int j = 0; ok && j < nkv; j++) {
+        // dP(j) = dO V_j^T into buffer j % 2, once dQ(j-2) has read the dS it held
+        if (j >= 2 && !mbar_wait(smem_addr(&bars.dq_done[j & 1]), ((j - 2) >> 1) & 1, ab)) break;
+        const int sv = j % kVStages;
+        if (!mbar_wait(smem_addr(&bars.v_full[sv]), (j / kVStages) & 1, ab)) break;
+        tc_fence_after();
+        const uint64_t dv = opaque64(dV0) + (uint64_t)(sv * kTileDesc);
+        const uint64_t ddo = opaque64(dDOd);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; kk++)
+          mma_ss(tmem + colDP + (j & 1) * 128, ddo + kmajor_koff(kk), dv + kmajor_koff(kk),
+                 idesc_s, kk > 0);
+        mma_commit(smem_addr(&bars.dp_full[j & 1]));
+        mma_commit(smem_addr(&bars.v_empty[sv]));
+      }
+      mma_commit(smem_addr(&bars.drain[1]));
+      int no_abort = 0;
+      Abort local{&no_abort, p.status};
+      mbar_wait(smem_addr(&bars.drain[1]), 0, local);
+    }
+  } else if (warp == 3) {
     // ------------------------------------------------------------------ MMA issuer: dQ
     if (lane == 0) {
       const uint32_t idesc_g = idesc_bf16_f32(kTile, kD, false, true);
@@ -642,10 +651,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(smem_addr(&bars.k_empty[sk]));
       }
       mma_commit(smem_addr(&bars.acc_done));
-      mma_commit(smem_addr(&bars.drain[1]));
+      mma_commit(smem_addr(&bars.drain[2]));
       int no_abort = 0;
       Abort local{&no_abort, p.status};
-      mbar_wait(smem_addr(&bars.drain[1]), 0, local);
+      mbar_wait(smem_addr(&bars.drain[2]), 0, local);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ per query row math
