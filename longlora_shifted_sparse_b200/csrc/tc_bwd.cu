@@ -39,6 +39,7 @@
 // (dQ pass: warps 1..3 MMA issuers), warps 4..11 the per-row math. Every wait is bounded
 // (see sm100.cuh).
 #include "common.cuh"
+#include "fastmath.cuh"
 #include "sm100.cuh"
 #include "tc_kernels.h"
 #include "tma_host.h"
@@ -87,6 +88,25 @@ __device__ __forceinline__ uint64_t opaque64(uint64_t v) {
   uint64_t r;
   asm volatile("mov.b64 %0, %1;" : "=l"(r) : "l"(v));
   return r;
+}
+
+// Column c of a thread's 64 probabilities takes its exponential from the FMA-pipe polynomial
+// (fastmath.cuh) when bit c of the mask is set, else from the MUFU unit; off the diagonal
+// tiles only (no -inf scores there; the polynomial clamps its argument at -125). On a B200,
+// 32k workload, moving 1/8, 1/4 or 3/8 of a pass's exponentials to the polynomial left it
+// as fast or slowed it (dQ 2.96 -> 2.94 / 3.01 / 3.17 ms, dK/dV 4.41 -> 4.49 / 4.68 ms), so
+// both masks default to 0 (all exponentials on the MUFU).
+#ifndef S2_DKDV_POLY_MASK
+#define S2_DKDV_POLY_MASK 0x0ull
+#endif
+#ifndef S2_DQ_POLY_MASK
+#define S2_DQ_POLY_MASK 0x0ull
+#endif
+constexpr unsigned long long kDkdvPolyMask = S2_DKDV_POLY_MASK;
+constexpr unsigned long long kDqPolyMask = S2_DQ_POLY_MASK;
+template <unsigned long long kMask>
+__device__ __forceinline__ float exp2_mixed(float x, int c) {
+  return ((kMask >> c) & 1ull) ? exp2_poly(x) : fast_exp2(x);
 }
 
 // Causal mask of a diagonal tile, applied to a thread's 64 raw scores (columns c = 0..63 of
@@ -370,11 +390,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(smem_addr(&bars.st_consumed));  // S^T may now be overwritten
-        if (diag) mask_scores(x0, x1, row - c0, 0);  // query row c0+c before key row: P = 0
+        if (diag) {
+          mask_scores(x0, x1, row - c0, 0);  // query row c0+c before key row: P = 0
 #pragma unroll
-        for (int c = 0; c < 64; c++) {
-          const float l = __shfl_sync(0xffffffffu, nl2[c >> 5], c & 31);
-          pr[c] = fast_exp2(fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, l));
+          for (int c = 0; c < 64; c++) {
+            const float l = __shfl_sync(0xffffffffu, nl2[c >> 5], c & 31);
+            pr[c] = fast_exp2(fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, l));
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; c++) {
+            const float l = __shfl_sync(0xffffffffu, nl2[c >> 5], c & 31);
+            pr[c] = exp2_mixed<kDkdvPolyMask>(
+                fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, l), c);
+          }
         }
         pin_regs(pr);
       }
@@ -683,10 +712,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(smem_addr(&bars.s_consumed));  // S may now be overwritten
-        if (diag) mask_scores(x0, x1, row - c0, 1);  // key column after the query row: P = 0
+        if (diag) {
+          mask_scores(x0, x1, row - c0, 1);  // key column after the query row: P = 0
 #pragma unroll
-        for (int c = 0; c < 64; c++)
-          pr[c] = fast_exp2(fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, nlse2));
+          for (int c = 0; c < 64; c++)
+            pr[c] = fast_exp2(fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, nlse2));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; c++)
+            pr[c] = exp2_mixed<kDqPolyMask>(
+                fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, nlse2), c);
+        }
         pin_regs(pr);
       }
       ok = mbar_wait(smem_addr(&bars.dp_full[j & 1]), (j >> 1) & 1, ab);
