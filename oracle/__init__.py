@@ -96,26 +96,49 @@ def rope(x: np.ndarray, pos, s: float, base: float = 10000.0, inverse: bool = Fa
     return y
 
 
+# Shift patterns (which heads see the sequence rolled by -G/2); see shifted_head in
+# s2attn_oracle.c: "half" = the second half of the heads, "alternate" = odd kv heads,
+# "none" = no head.
+SHIFT_PATTERNS = {"half": 0, "alternate": 1, "none": 2}
+
+
+def _mode(causal, shift) -> int:
+    return int(bool(causal)) | (SHIFT_PATTERNS[shift] << 4)
+
+
+def head_is_shifted(h: int, Hq: int, Hkv: int, shift: str = "half") -> bool:
+    """Whether query head h sees the rolled sequence under the given pattern."""
+    R = Hq // Hkv
+    if shift == "alternate":
+        return (h // R) % 2 == 1
+    if shift == "none":
+        return False
+    return h >= Hq // 2
+
+
 def _dims(q, k):
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
     return B, N, Hq, Hkv, d
 
 
-def fwd(q, k, v, G: int, s: float, base: float = 10000.0, causal: bool = True):
+def fwd(q, k, v, G: int, s: float, base: float = 10000.0, causal: bool = True,
+        shift: str = "half"):
     """Full forward. Returns (o [B,N,Hq,d] fp64, lse [B,Hq,N] fp64)."""
     (q, dt), (k, _), (v, _) = _in(q), _in(k), _in(v)
     B, N, Hq, Hkv, d = _dims(q, k)
     o = np.empty((B, N, Hq, d), dtype=np.float64)
     lse = np.empty((B, Hq, N), dtype=np.float64)
-    rc = _load().s2o_fwd(_ptr(q), _ptr(k), _ptr(v), dt, B, N, Hq, Hkv, d, G, int(causal),
+    rc = _load().s2o_fwd(_ptr(q), _ptr(k), _ptr(v), dt, B, N, Hq, Hkv, d, G,
+                         _mode(causal, shift),
                          float(s), float(base), _ptr(o), _ptr(lse))
     if rc:
         raise ValueError("oracle fwd rejected the shape (rc=%d)" % rc)
     return o, lse
 
 
-def bwd(q, k, v, dout, G: int, s: float, base: float = 10000.0, causal: bool = True):
+def bwd(q, k, v, dout, G: int, s: float, base: float = 10000.0, causal: bool = True,
+        shift: str = "half"):
     """Full backward. Returns (dq, dk, dv) fp64 in the input layouts."""
     (q, dt), (k, _), (v, _), (dout, _) = _in(q), _in(k), _in(v), _in(dout)
     B, N, Hq, Hkv, d = _dims(q, k)
@@ -123,21 +146,23 @@ def bwd(q, k, v, dout, G: int, s: float, base: float = 10000.0, causal: bool = T
     dk = np.empty((B, N, Hkv, d), dtype=np.float64)
     dv = np.empty((B, N, Hkv, d), dtype=np.float64)
     rc = _load().s2o_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), dt, B, N, Hq, Hkv, d, G,
-                         int(causal), float(s), float(base), _ptr(dq), _ptr(dk), _ptr(dv))
+                         _mode(causal, shift), float(s), float(base), _ptr(dq), _ptr(dk),
+                         _ptr(dv))
     if rc:
         raise ValueError("oracle bwd rejected the shape (rc=%d)" % rc)
     return dq, dk, dv
 
 
 def fwd_unit(q, k, v, G: int, s: float, b: int, kvh: int, g: int, base: float = 10000.0,
-             causal: bool = True):
+             causal: bool = True, shift: str = "half"):
     """One unit's forward: (o_u [R,G,d], lse_u [R,G]) in rolled local-row order."""
     (q, dt), (k, _), (v, _) = _in(q), _in(k), _in(v)
     B, N, Hq, Hkv, d = _dims(q, k)
     R = Hq // Hkv
     o_u = np.empty((R, G, d), dtype=np.float64)
     lse_u = np.empty((R, G), dtype=np.float64)
-    rc = _load().s2o_fwd_unit(_ptr(q), _ptr(k), _ptr(v), dt, B, N, Hq, Hkv, d, G, int(causal),
+    rc = _load().s2o_fwd_unit(_ptr(q), _ptr(k), _ptr(v), dt, B, N, Hq, Hkv, d, G,
+                              _mode(causal, shift),
                               float(s), float(base), b, kvh, g, _ptr(o_u), _ptr(lse_u))
     if rc:
         raise ValueError("oracle fwd_unit rejected the arguments (rc=%d)" % rc)
@@ -145,7 +170,7 @@ def fwd_unit(q, k, v, G: int, s: float, b: int, kvh: int, g: int, base: float = 
 
 
 def bwd_unit(q, k, v, dout, G: int, s: float, b: int, kvh: int, g: int, base: float = 10000.0,
-             causal: bool = True):
+             causal: bool = True, shift: str = "half"):
     """One unit's backward: (dq_u [R,G,d], dk_u [G,d], dv_u [G,d]) in rolled local-row order."""
     (q, dt), (k, _), (v, _), (dout, _) = _in(q), _in(k), _in(v), _in(dout)
     B, N, Hq, Hkv, d = _dims(q, k)
@@ -154,30 +179,32 @@ def bwd_unit(q, k, v, dout, G: int, s: float, b: int, kvh: int, g: int, base: fl
     dk_u = np.empty((G, d), dtype=np.float64)
     dv_u = np.empty((G, d), dtype=np.float64)
     rc = _load().s2o_bwd_unit(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), dt, B, N, Hq, Hkv, d, G,
-                              int(causal), float(s), float(base), b, kvh, g, _ptr(dq_u),
+                              _mode(causal, shift), float(s), float(base), b, kvh, g, _ptr(dq_u),
                               _ptr(dk_u), _ptr(dv_u))
     if rc:
         raise ValueError("oracle bwd_unit rejected the arguments (rc=%d)" % rc)
     return dq_u, dk_u, dv_u
 
 
-def unit_rows(N: int, G: int, Hq: int, kvh: int, Hkv: int, g: int) -> np.ndarray:
+def unit_rows(N: int, G: int, Hq: int, kvh: int, Hkv: int, g: int,
+              shift: str = "half") -> np.ndarray:
     """Original token index of each rolled local row of unit (kvh, g)."""
     R = Hq // Hkv
-    shifted = kvh * R >= Hq // 2
+    shifted = head_is_shifted(kvh * R, Hq, Hkv, shift)
     r = g * G + np.arange(G)
     return (r + G // 2) % N if shifted else r
 
 
 def fwd_rows(q, k, v, G: int, s: float, b: int, h: int, g: int, rows, base: float = 10000.0,
-             causal: bool = True):
+             causal: bool = True, shift: str = "half"):
     """Forward at chosen rolled local rows of query head h, group g: (o [n,d], lse [n])."""
     (q, dt), (k, _), (v, _) = _in(q), _in(k), _in(v)
     B, N, Hq, Hkv, d = _dims(q, k)
     rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
     o = np.empty((rows.size, d), dtype=np.float64)
     lse = np.empty(rows.size, dtype=np.float64)
-    rc = _load().s2o_fwd_rows(_ptr(q), _ptr(k), _ptr(v), dt, B, N, Hq, Hkv, d, G, int(causal),
+    rc = _load().s2o_fwd_rows(_ptr(q), _ptr(k), _ptr(v), dt, B, N, Hq, Hkv, d, G,
+                              _mode(causal, shift),
                               float(s), float(base), b, h, g, rows.size, _ptr(rows), _ptr(o),
                               _ptr(lse))
     if rc:
@@ -186,7 +213,7 @@ def fwd_rows(q, k, v, G: int, s: float, b: int, h: int, g: int, rows, base: floa
 
 
 def bwd_rows(q, k, v, dout, G: int, s: float, b: int, kvh: int, g: int, qrows, krows,
-             base: float = 10000.0, causal: bool = True):
+             base: float = 10000.0, causal: bool = True, shift: str = "half"):
     """Backward of unit (b, kvh, g) at chosen rolled local rows:
     (dq [nq,R,d] for the R query heads of kvh, dk [nk,d], dv [nk,d])."""
     (q, dt), (k, _), (v, _), (dout, _) = _in(q), _in(k), _in(v), _in(dout)
@@ -198,7 +225,7 @@ def bwd_rows(q, k, v, dout, G: int, s: float, b: int, kvh: int, g: int, qrows, k
     dk = np.empty((krows.size, d), dtype=np.float64)
     dv = np.empty((krows.size, d), dtype=np.float64)
     rc = _load().s2o_bwd_rows(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), dt, B, N, Hq, Hkv, d, G,
-                              int(causal), float(s), float(base), b, kvh, g, qrows.size,
+                              _mode(causal, shift), float(s), float(base), b, kvh, g, qrows.size,
                               _ptr(qrows), krows.size, _ptr(krows), _ptr(dq), _ptr(dk), _ptr(dv))
     if rc:
         raise ValueError("oracle bwd_rows rejected the arguments (rc=%d)" % rc)

@@ -48,7 +48,7 @@
 enum { S2O_IN_BF16 = 0, S2O_IN_F32 = 1, S2O_IN_F64 = 2 };
 
 typedef struct {
-  int B, N, Hq, Hkv, d, G, causal;
+  int B, N, Hq, Hkv, d, G, causal, shift;
   double s, base;
 } cfg_t;
 
@@ -73,7 +73,22 @@ int s2o_check(int B, int N, int Hq, int Hkv, int d, int G) {
   return 0;
 }
 
-static int shifted_head(const cfg_t* c, int h) { return h >= c->Hq / 2; }
+/* Which heads see the rolled sequence (the shift pattern):
+ *   0 (default) the second half of the heads ("LongLoRA and Shifted Sparse Attention
+ *     (S^2-Attn)", definition; "LongLoRA: Efficient 100k Context LLM Fine-Tuning Guide",
+ *     Implementation, Step 1);
+ *   1 alternate heads, the odd ones ("LoRA for Long-Context Adaptation", section
+ *     "Shifted sparse attention: making training feasible": heads 0, 2, 4, ... unshifted,
+ *     heads 1, 3, 5, ... shifted by half a group);
+ *   2 no head (plain grouped attention; with G = N the dense attention the guide's
+ *     inference path falls back to, "Dual-Mode" paragraph).
+ * Query head h follows its kv head h / R, so with GQA the pattern applies to kv heads. */
+static int shifted_head(const cfg_t* c, int h) {
+  const int R = c->Hq / c->Hkv;
+  if (c->shift == 1) return (h / R) % 2 == 1;
+  if (c->shift == 2) return 0;
+  return h >= c->Hq / 2;
+}
 
 /* Rolled row r -> original row. np.roll(x, -G/2)[r] == x[(r + G/2) mod N]. */
 static long src_row(const cfg_t* c, long r, int shifted) {
@@ -184,9 +199,12 @@ static int unit_args_ok(const cfg_t* c, int b, int kvh, int g) {
   return b >= 0 && b < c->B && kvh >= 0 && kvh < c->Hkv && g >= 0 && g < c->N / c->G;
 }
 
+/* `causal` carries two fields: bit 0 the causal mask inside a group, bits 4-5 the shift
+ * pattern of shifted_head (0 when the caller passes a plain 0 / 1). */
 static void fill_cfg(cfg_t* c, int B, int N, int Hq, int Hkv, int d, int G, int causal, double s,
                      double base) {
-  c->B = B; c->N = N; c->Hq = Hq; c->Hkv = Hkv; c->d = d; c->G = G; c->causal = causal;
+  c->B = B; c->N = N; c->Hq = Hq; c->Hkv = Hkv; c->d = d; c->G = G; c->causal = causal & 1;
+  c->shift = (causal >> 4) & 3;
   c->s = s; c->base = base;
 }
 

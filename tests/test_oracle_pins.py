@@ -170,6 +170,75 @@ def test_wrap_group_mixes_end_and_start():
     np.testing.assert_array_equal(o2[0, 0, 0], o[0, 0, 0])
 
 
+def _read_alternate_examples():
+    rows = []
+    with open(os.path.join(GOLDEN, "alternate_heads.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                rows.append(tuple(int(x) for x in line.split()))
+    return rows
+
+
+@pytest.mark.parametrize("G,head,first,last", _read_alternate_examples())
+def test_alternate_head_pattern_worked_example(G, head, first, last):
+    """Alternate-head shift pattern: even heads see tokens 0 .. G-1 in their first group,
+    odd heads tokens G/2 .. 3G/2-1 (the pages' group figure, tests/golden)."""
+    rows = oracle.unit_rows(2 * G, G, Hq=8, kvh=head, Hkv=8, g=0, shift="alternate")
+    assert rows[0] == first and rows[-1] == last
+    np.testing.assert_array_equal(rows, np.arange(first, last + 1))
+
+
+@pytest.mark.parametrize("Hq,Hkv,causal", [(4, 4, True), (8, 4, True), (4, 4, False)])
+def test_alternate_pattern_is_the_half_pattern_on_reordered_heads(Hq, Hkv, causal):
+    """Heads are computed independently, so shifting the odd kv heads equals shifting the
+    second half after reordering the kv heads as [even..., odd...] (query heads follow their
+    kv head): the alternate pattern is pinned to the half pattern's pins, forward and
+    backward."""
+    B, N, d, G = 1, 32, 8, 8
+    q, k, v, do = _inputs(21, B, N, Hq, Hkv, d)
+    R = Hq // Hkv
+    kv_perm = np.r_[0:Hkv:2, 1:Hkv:2]
+    q_perm = np.concatenate([np.arange(h * R, (h + 1) * R) for h in kv_perm])
+    o_a, l_a = oracle.fwd(q, k, v, G, 2.0, causal=causal, shift="alternate")
+    o_h, l_h = oracle.fwd(q[:, :, q_perm], k[:, :, kv_perm], v[:, :, kv_perm], G, 2.0,
+                          causal=causal)
+    np.testing.assert_array_equal(o_a[:, :, q_perm], o_h)
+    np.testing.assert_array_equal(l_a[:, q_perm], l_h)
+    g_a = oracle.bwd(q, k, v, do, G, 2.0, causal=causal, shift="alternate")
+    g_h = oracle.bwd(q[:, :, q_perm], k[:, :, kv_perm], v[:, :, kv_perm], do[:, :, q_perm], G,
+                     2.0, causal=causal)
+    np.testing.assert_array_equal(g_a[0][:, :, q_perm], g_h[0])
+    np.testing.assert_array_equal(g_a[1][:, :, kv_perm], g_h[1])
+    np.testing.assert_array_equal(g_a[2][:, :, kv_perm], g_h[2])
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (4, 2)])
+def test_no_shift_one_group_is_dense_causal_on_every_head(Hq, Hkv):
+    """Pattern "none" with G = N: every head is textbook dense causal attention (torch SDPA),
+    the inference mode the guide's code falls back to ("Dual-Mode")."""
+    N, d = 32, 8
+    q, k, v, _ = _inputs(22, 1, N, Hq, Hkv, d)
+    o, _ = oracle.fwd(q, k, v, G=N, s=2.0, shift="none")
+    dense = ref.dense_causal(_t(q), _t(k), _t(v), 2.0).numpy()
+    np.testing.assert_allclose(o, dense, atol=1e-12)
+
+
+def test_no_shift_heads_are_block_diagonal():
+    """Pattern "none", G < N: every head (also those the half pattern shifts) attends inside
+    consecutive groups of its own rows only."""
+    N, G, d = 64, 16, 8
+    q, k, v, _ = _inputs(23, 1, N, 2, 2, d)
+    o, _ = oracle.fwd(q, k, v, G=G, s=1.0, shift="none")
+    qr = ref.rope_complex(_t(q), 1.0)
+    kr = ref.rope_complex(_t(k), 1.0)
+    for h in range(2):
+        for g in range(N // G):
+            sl = slice(g * G, (g + 1) * G)
+            og = torch.nn.functional.scaled_dot_product_attention(
+                qr[0, sl, h][None], kr[0, sl, h][None], _t(v)[0, sl, h][None], is_causal=True)
+            np.testing.assert_allclose(o[0, sl, h], og[0].numpy(), atol=1e-12)
+
+
 def test_roll_forward_then_back_is_identity():
     x = np.arange(40).reshape(1, 40, 1, 1)
     for G in (2, 8, 40):
