@@ -177,10 +177,11 @@ def _oracle_sample(w, inputs):
     q, k, v, do = inputs
     rows = np.arange(w.G)
     t0 = time.perf_counter()
-    oracle.fwd_rows(q, k, v, w.G, w.pi_scale, 0, 0, 0, rows, w.rope_base, w.causal)
+    oracle.fwd_rows(q, k, v, w.G, w.pi_scale, 0, 0, 0, rows, w.rope_base, w.causal,
+                    shift=w.shift)
     if w.backward:
         oracle.bwd_rows(q, k, v, do, w.G, w.pi_scale, 0, 0, 0, rows, rows, w.rope_base,
-                        w.causal)
+                        w.causal, shift=w.shift)
     dt = time.perf_counter() - t0
     R = w.Hq // w.Hkv
     unit_fwd = flops.attention_fwd_flops(1, w.G, 1, w.d, w.G, w.causal)
@@ -213,7 +214,9 @@ def run_reference(args):
         "ms_per_step": mean * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.Hq, "H_kv": w.Hkv,
-                   "d": w.d, "G": w.G, "pi_scale": w.pi_scale, "parallelism": "host threads"},
+                   "d": w.d, "G": w.G, "pi_scale": w.pi_scale, "rope_base": w.rope_base,
+                   "causal": w.causal, "shift": w.shift, "fwd_bwd": w.backward,
+                   "parallelism": "host threads"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": SAMPLE_DESC.format(name=w.name, G=w.G)},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -258,12 +261,13 @@ def run_ours(args):
     ws = s2.workspace(w.B, w.N, w.Hq, w.Hkv, w.d, code, dev)
 
     def step():
-        s2.forward(tq, tk, tv, w.G, w.pi_scale, w.rope_base, w.causal, ws=ws, out=o, lse=lse)
+        s2.forward(tq, tk, tv, w.G, w.pi_scale, w.rope_base, w.causal, ws=ws, out=o, lse=lse,
+                   shift=w.shift)
         if w.backward:
             # the training-step order: the backward reuses the rotation the forward left in
             # the workspace (s2attn_bwd_after_fwd), as the autograd wrapper does
             s2.backward(tq, tk, tv, o, lse, tdo, w.G, w.pi_scale, w.rope_base, w.causal, ws=ws,
-                        grads=(gq, gk, gv), after_forward=True)
+                        grads=(gq, gk, gv), after_forward=True, shift=w.shift)
 
     def barrier():
         if world > 1:
@@ -336,11 +340,11 @@ def run_ours(args):
             if used[k_]:
                 stream.wait_event(ev["out"][k_])         # step i-2's outputs are copied out
             s2.forward(ins[0], ins[1], ins[2], w.G, w.pi_scale, w.rope_base, w.causal, ws=ws_,
-                       out=outs[0], lse=outs[1])
+                       out=outs[0], lse=outs[1], shift=w.shift)
             if w.backward:
                 s2.backward(ins[0], ins[1], ins[2], outs[0], outs[1], ins[3], w.G, w.pi_scale,
                             w.rope_base, w.causal, ws=ws_, grads=tuple(outs[2:]),
-                            after_forward=True)
+                            after_forward=True, shift=w.shift)
             ev["comp"][k_].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev["comp"][k_])
@@ -403,14 +407,15 @@ def run_ours(args):
         cpu_baseline = {"value": counted / dt / 1e12, "unit": UNIT, "cores": cores,
                         "kind": "oracle", "sample": SAMPLE_DESC.format(name=w.name, G=w.G)}
 
-    paths = {s2.s2attn_kernel_path(w.B, w.N, w.Hq, w.Hkv, w.d, w.G, int(w.causal), code)}
+    paths = {s2.s2attn_kernel_path(w.B, w.N, w.Hq, w.Hkv, w.d, w.G, s2.mode(w.causal, w.shift),
+                                   code)}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "N": w.N, "H_q": w.Hq, "H_kv": w.Hkv,
-                   "d": w.d, "G": w.G, "pi_scale": w.pi_scale, "causal": w.causal,
-                   "fwd_bwd": w.backward, "parallelism": "independent batch per GPU",
+                   "d": w.d, "G": w.G, "pi_scale": w.pi_scale, "rope_base": w.rope_base,
+                   "causal": w.causal, "shift": w.shift, "fwd_bwd": w.backward, "parallelism": "independent batch per GPU",
                    "l2": "inputs exceed L2 (q, k, v, dO are %.0f MB each)" %
                          (tq.numel() * es / 1e6),
                    "kernel_path": "tcgen05" if paths == {1} else "cuda-core"},

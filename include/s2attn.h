@@ -11,10 +11,11 @@
  *    "LongLoRA: Efficient 100k Context LLM Fine-Tuning Guide", "How Shifted Short Attention
  *    Works" and "Implementation ... Step 1"): query heads h >= H_q/2 (and kv heads
  *    >= H_kv/2) see the sequence rolled by -G/2 with wrap-around: rolled row r holds
- *    original token (r + G/2) mod N.
+ *    original token (r + G/2) mod N. Two other head patterns are selectable through the
+ *    mode argument (S2_SHIFT_* below).
  *  - Group fold: rolled rows are cut into N/G groups of G rows; inside each group,
  *    softmax(q k^T / sqrt(d)) v with a causal mask on group-local positions (no mask
- *    when causal == 0). GQA: query head h uses kv head h / (H_q / H_kv).
+ *    without S2_CAUSAL). GQA: query head h uses kv head h / (H_q / H_kv).
  *  - Roll back: each shifted head's output row r is stored at token (r + G/2) mod N.
  *  - Backward: gradients of the above with respect to the pre-RoPE q, k and to v; dk and
  *    dv of a kv head are summed over the query heads that share it.
@@ -60,8 +61,25 @@ typedef enum {
   S2_ERR_WORKSPACE = 6,      /* workspace NULL or ws_bytes < s2attn_workspace_bytes(...) */
   S2_ERR_CUDA = 7,           /* a CUDA runtime/driver call failed */
   S2_ERR_DEVICE_TIMEOUT = 8, /* a bounded device-side wait expired (see s2attn_device_status) */
-  S2_ERR_ARG = 9             /* pi_scale or rope_base not finite and > 0, or causal not 0/1 */
+  S2_ERR_ARG = 9             /* pi_scale or rope_base not finite and > 0, or a bad mode */
 } s2_status;
+
+/* The `mode` argument of the attention calls: S2_CAUSAL or 0, ORed with one S2_SHIFT_*
+ * pattern. The values 0 and 1 are the plain causal flag with the method's half-head shift.
+ * Any other bit set is rejected with S2_ERR_ARG. Query heads follow their kv head under
+ * every pattern; with H_kv even, "h >= H_q/2" and "h / (H_q/H_kv) >= H_kv/2" agree. */
+#define S2_CAUSAL 0x01          /* causal mask on group-local positions; absent: no mask,
+                                   every query sees its whole group (the full-group reading
+                                   of "LoRA for Long-Context Adaptation", "Shifted sparse
+                                   attention: making training feasible") */
+#define S2_SHIFT_HALF 0x00      /* the second half of the heads is shifted (the definition) */
+#define S2_SHIFT_ALTERNATE 0x10 /* every odd kv head is shifted: the alternate-heads
+                                   wording of the same section of "LoRA for Long-Context
+                                   Adaptation" */
+#define S2_SHIFT_NONE 0x20      /* no head is shifted. With G == N and S2_CAUSAL this is
+                                   plain dense causal attention: the inference mode of the
+                                   guide's "Dual-Mode" paragraph ("LongLoRA: Efficient 100k
+                                   Context LLM Fine-Tuning Guide") */
 
 typedef enum {
   S2_BF16 = 0, /* bfloat16 storage, fp32 accumulation, tensor cores where the shape allows */
@@ -69,18 +87,21 @@ typedef enum {
 } s2_dtype;
 
 /* Bytes of device workspace that s2attn_fwd / s2attn_bwd need for this shape (it does not
- * depend on G or causal). Returns 0 for arguments that s2attn_fwd would reject with
+ * depend on G or mode). Returns 0 for arguments that s2attn_fwd would reject with
  * S2_ERR_SHAPE, S2_ERR_HEADDIM or S2_ERR_DTYPE. The workspace holds the rotated q and k
  * (head-major, original token order), the RoPE cos/sin table, the backward's row sums
  * D = rowsum(dO * O) and the device status word. */
 S2_API size_t s2attn_workspace_bytes(int B, int N, int H_q, int H_kv, int d, int dtype);
 
 /* Forward: o and lse from q, k, v. See the header comment for the operation and layouts.
- * G: group size (even, divides N). causal: 1 = causal mask inside each group, 0 = none.
+ * G: group size (even, divides N). mode: S2_CAUSAL (causal mask inside each group) or 0,
+ * ORed with the shifted-head pattern (S2_SHIFT_HALF = 0 by default).
  * pi_scale: position interpolation factor s = L_new / L_orig (1 = plain RoPE).
- * rope_base: RoPE base (10000 for LLaMA2). */
+ * rope_base: RoPE base (10000 for LLaMA2). Base scaling, the other rescaling of the same
+ * pages ("LoRA for Long-Context Adaptation", "A training recipe", step 1), is
+ * pi_scale = 1 with rope_base multiplied by the extension ratio. */
 S2_API s2_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
-                     int B, int N, int H_q, int H_kv, int d, int G, int causal,
+                     int B, int N, int H_q, int H_kv, int d, int G, int mode,
                      float pi_scale, float rope_base, int dtype,
                      void* workspace, size_t ws_bytes, void* cuda_stream);
 
@@ -89,7 +110,7 @@ S2_API s2_status s2attn_fwd(const void* q, const void* k, const void* v, void* o
  * arguments. The workspace may be the forward's or another one of the same size. */
 S2_API s2_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o,
                      const float* lse, const void* dout, void* dq, void* dk, void* dv,
-                     int B, int N, int H_q, int H_kv, int d, int G, int causal,
+                     int B, int N, int H_q, int H_kv, int d, int G, int mode,
                      float pi_scale, float rope_base, int dtype,
                      void* workspace, size_t ws_bytes, void* cuda_stream);
 
@@ -105,7 +126,7 @@ S2_API s2_status s2attn_bwd(const void* q, const void* k, const void* v, const v
 S2_API s2_status s2attn_bwd_after_fwd(const void* q, const void* k, const void* v,
                                       const void* o, const float* lse, const void* dout,
                                       void* dq, void* dk, void* dv, int B, int N, int H_q,
-                                      int H_kv, int d, int G, int causal, float pi_scale,
+                                      int H_kv, int d, int G, int mode, float pi_scale,
                                       float rope_base, int dtype, void* workspace,
                                       size_t ws_bytes, void* cuda_stream);
 
@@ -129,13 +150,13 @@ S2_API s2_status s2attn_bwd_after_fwd(const void* q, const void* k, const void* 
  *    kernels overlap on the GPU (e.g. on two streams) race on the array: serialise them. */
 S2_API s2_status s2attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o,
                                     float* lse, int B, int N, int H_q, int H_kv, int d, int G,
-                                    int causal, float pi_scale, float rope_base, int dtype,
+                                    int mode, float pi_scale, float rope_base, int dtype,
                                     void* cuda_stream);
 
 /* Which kernel family s2attn_fwd and s2attn_bwd launch for these arguments:
  * 1 = tcgen05 tensor-core kernels (bf16, d == 128, G % 256 == 0),
  * 0 = CUDA-core kernels (any other valid shape, and every fp32 call), -1 = invalid. */
-S2_API int s2attn_kernel_path(int B, int N, int H_q, int H_kv, int d, int G, int causal, int dtype);
+S2_API int s2attn_kernel_path(int B, int N, int H_q, int H_kv, int d, int G, int mode, int dtype);
 
 /* Waits for cuda_stream, then reads and clears the device status word of the workspace
  * used by the last call on it: S2_OK, or S2_ERR_DEVICE_TIMEOUT if a bounded wait in a

@@ -175,13 +175,25 @@ cudaError_t enqueue_forward(const Params& p, int dt, cudaStream_t s) {
   return timed_launch(kFwdSimt, s, [&] { return launch_simt_fwd(p, bf16, s); });
 }
 
-s2_status common_checks(int B, int N, int Hq, int Hkv, int d, int G, int causal, float s,
+// mode = S2_CAUSAL or 0, ORed with one S2_SHIFT_* pattern; nothing else.
+bool mode_ok(int mode) {
+  const int shift = mode & ~S2_CAUSAL;
+  return shift == S2_SHIFT_HALF || shift == S2_SHIFT_ALTERNATE || shift == S2_SHIFT_NONE;
+}
+
+int shift_pattern(int mode) {
+  const int shift = mode & ~S2_CAUSAL;
+  return shift == S2_SHIFT_ALTERNATE ? kShiftAlternate
+         : shift == S2_SHIFT_NONE    ? kShiftNone
+                                     : kShiftHalf;
+}
+
+s2_status common_checks(int B, int N, int Hq, int Hkv, int d, int G, int mode, float s,
                         float base, int dt, void* ws, size_t ws_bytes) {
   if (!dtype_ok(dt)) return S2_ERR_DTYPE;
   if (!shape_ok(B, N, Hq, Hkv, G)) return S2_ERR_SHAPE;
   if (!headdim_ok(d)) return S2_ERR_HEADDIM;
-  if (!(isfinite(s) && s > 0.f) || !(isfinite(base) && base > 0.f) ||
-      (causal != 0 && causal != 1))
+  if (!(isfinite(s) && s > 0.f) || !(isfinite(base) && base > 0.f) || !mode_ok(mode))
     return S2_ERR_ARG;
   if (!ws) return S2_ERR_WORKSPACE;
   if (!aligned16(ws)) return S2_ERR_ALIGN;
@@ -189,10 +201,12 @@ s2_status common_checks(int B, int N, int Hq, int Hkv, int d, int G, int causal,
   return S2_OK;
 }
 
-Params make_params(int B, int N, int Hq, int Hkv, int d, int G, int causal, float s, float base,
+Params make_params(int B, int N, int Hq, int Hkv, int d, int G, int mode, float s, float base,
                    int dt, void* ws) {
   Params p{};
-  p.B = B; p.N = N; p.Hq = Hq; p.Hkv = Hkv; p.d = d; p.G = G; p.causal = causal;
+  p.B = B; p.N = N; p.Hq = Hq; p.Hkv = Hkv; p.d = d; p.G = G;
+  p.causal = mode & S2_CAUSAL;
+  p.shift = shift_pattern(mode);
   p.pi_scale = s;
   p.rope_base = base;
   p.scale = (float)(1.0 / sqrt((double)d));
@@ -222,24 +236,23 @@ size_t s2attn_workspace_bytes(int B, int N, int H_q, int H_kv, int d, int dtype)
   return ws_layout(B, N, H_q, H_kv, d, dtype).total;
 }
 
-int s2attn_kernel_path(int B, int N, int H_q, int H_kv, int d, int G, int causal, int dtype) {
-  if (!dtype_ok(dtype) || !shape_ok(B, N, H_q, H_kv, G) || !headdim_ok(d) ||
-      (causal != 0 && causal != 1))
+int s2attn_kernel_path(int B, int N, int H_q, int H_kv, int d, int G, int mode, int dtype) {
+  if (!dtype_ok(dtype) || !shape_ok(B, N, H_q, H_kv, G) || !headdim_ok(d) || !mode_ok(mode))
     return -1;
   return tc_path(d, G, dtype) ? 1 : 0;
 }
 
 s2_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                     int N, int H_q, int H_kv, int d, int G, int causal, float pi_scale,
+                     int N, int H_q, int H_kv, int d, int G, int mode, float pi_scale,
                      float rope_base, int dtype, void* workspace, size_t ws_bytes,
                      void* cuda_stream) {
   if (!q || !k || !v || !o || !lse) return S2_ERR_NULL;
-  s2_status st = common_checks(B, N, H_q, H_kv, d, G, causal, pi_scale, rope_base, dtype,
+  s2_status st = common_checks(B, N, H_q, H_kv, d, G, mode, pi_scale, rope_base, dtype,
                                workspace, ws_bytes);
   if (st != S2_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return S2_ERR_ALIGN;
-  Params p = make_params(B, N, H_q, H_kv, d, G, causal, pi_scale, rope_base, dtype, workspace);
+  Params p = make_params(B, N, H_q, H_kv, d, G, mode, pi_scale, rope_base, dtype, workspace);
   p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
   return to_status(enqueue_forward(p, dtype, static_cast<cudaStream_t>(cuda_stream)));
 }
@@ -251,17 +264,17 @@ namespace {
 // and the (cos, sin) table that the forward left in the workspace.
 s2_status backward_impl(const void* q, const void* k, const void* v, const void* o,
                         const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
-                        int N, int H_q, int H_kv, int d, int G, int causal, float pi_scale,
+                        int N, int H_q, int H_kv, int d, int G, int mode, float pi_scale,
                         float rope_base, int dtype, void* workspace, size_t ws_bytes,
                         void* cuda_stream, bool rotate) {
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return S2_ERR_NULL;
-  s2_status st = common_checks(B, N, H_q, H_kv, d, G, causal, pi_scale, rope_base, dtype,
+  s2_status st = common_checks(B, N, H_q, H_kv, d, G, mode, pi_scale, rope_base, dtype,
                                workspace, ws_bytes);
   if (st != S2_OK) return st;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
       !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
     return S2_ERR_ALIGN;
-  Params p = make_params(B, N, H_q, H_kv, d, G, causal, pi_scale, rope_base, dtype, workspace);
+  Params p = make_params(B, N, H_q, H_kv, d, G, mode, pi_scale, rope_base, dtype, workspace);
   p.q = q; p.k = k; p.v = v; p.o = const_cast<void*>(o); p.lse = const_cast<float*>(lse);
   p.dout = dout; p.dq = dq; p.dk = dk; p.dv = dv;
   const bool bf16 = dtype == S2_BF16;
@@ -287,18 +300,18 @@ s2_status backward_impl(const void* q, const void* k, const void* v, const void*
 
 s2_status s2attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                      const void* dout, void* dq, void* dk, void* dv, int B, int N, int H_q,
-                     int H_kv, int d, int G, int causal, float pi_scale, float rope_base,
+                     int H_kv, int d, int G, int mode, float pi_scale, float rope_base,
                      int dtype, void* workspace, size_t ws_bytes, void* cuda_stream) {
-  return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, N, H_q, H_kv, d, G, causal,
+  return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, N, H_q, H_kv, d, G, mode,
                        pi_scale, rope_base, dtype, workspace, ws_bytes, cuda_stream, true);
 }
 
 s2_status s2attn_bwd_after_fwd(const void* q, const void* k, const void* v, const void* o,
                                const float* lse, const void* dout, void* dq, void* dk, void* dv,
-                               int B, int N, int H_q, int H_kv, int d, int G, int causal,
+                               int B, int N, int H_q, int H_kv, int d, int G, int mode,
                                float pi_scale, float rope_base, int dtype, void* workspace,
                                size_t ws_bytes, void* cuda_stream) {
-  return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, N, H_q, H_kv, d, G, causal,
+  return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, N, H_q, H_kv, d, G, mode,
                        pi_scale, rope_base, dtype, workspace, ws_bytes, cuda_stream, false);
 }
 
@@ -345,7 +358,8 @@ const char* s2attn_status_string(int status) {
     case S2_ERR_WORKSPACE: return "workspace missing or smaller than s2attn_workspace_bytes()";
     case S2_ERR_CUDA: return "a CUDA call failed";
     case S2_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
-    case S2_ERR_ARG: return "invalid argument (pi_scale, rope_base finite and > 0; causal 0/1)";
+    case S2_ERR_ARG: return "invalid argument (pi_scale, rope_base finite and > 0; mode = "
+                             "S2_CAUSAL or 0 | one S2_SHIFT_* pattern)";
     default: return "unknown status";
   }
 }
@@ -426,14 +440,14 @@ cudaError_t noalloc_scratch_address(void** out) {
 
 extern "C" s2_status s2attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o,
                                         float* lse, int B, int N, int H_q, int H_kv, int d, int G,
-                                        int causal, float pi_scale, float rope_base, int dtype,
+                                        int mode, float pi_scale, float rope_base, int dtype,
                                         void* cuda_stream) {
   if (!q || !k || !v || !o || !lse) return S2_ERR_NULL;
   if (!dtype_ok(dtype)) return S2_ERR_DTYPE;
   if (!shape_ok(B, N, H_q, H_kv, G)) return S2_ERR_SHAPE;
   if (!headdim_ok(d)) return S2_ERR_HEADDIM;
   if (!(isfinite(pi_scale) && pi_scale > 0.f) || !(isfinite(rope_base) && rope_base > 0.f) ||
-      (causal != 0 && causal != 1))
+      !mode_ok(mode))
     return S2_ERR_ARG;
   if (ws_layout(B, N, H_q, H_kv, d, dtype).total > (size_t)S2ATTN_NOALLOC_SCRATCH_BYTES)
     return S2_ERR_WORKSPACE;
@@ -443,7 +457,7 @@ extern "C" s2_status s2attn_fwd_noalloc(const void* q, const void* k, const void
   if (noalloc_scratch_address(&scratch) != cudaSuccess) return S2_ERR_CUDA;
   // The status word at the start of the scratch is reset by the first kernel of the call;
   // everything else the kernels read from the scratch is written earlier in the same call.
-  Params p = make_params(B, N, H_q, H_kv, d, G, causal, pi_scale, rope_base, dtype, scratch);
+  Params p = make_params(B, N, H_q, H_kv, d, G, mode, pi_scale, rope_base, dtype, scratch);
   p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
   return to_status(enqueue_forward(p, dtype, static_cast<cudaStream_t>(cuda_stream)));
 }

@@ -10,6 +10,7 @@ namespace s2 {
 // Everything a kernel of one call needs. Built once per call on the host, passed by value.
 struct Params {
   int B, N, Hq, Hkv, d, G, causal;
+  int shift;         // ShiftPattern: which heads are rolled by -G/2
   float pi_scale, rope_base;
   float scale;       // 1 / sqrt(d)
   float scale_log2;  // log2(e) / sqrt(d): scores go straight to the exp2 domain
@@ -33,8 +34,21 @@ struct Params {
 
 enum StatusBits : unsigned { kStatusTimeout = 1u };
 
-// Half-group shift: query heads h >= Hq/2 (equivalently kv heads >= Hkv/2) are shifted.
-__host__ __device__ inline bool head_shifted(int h, int H) { return h >= H / 2; }
+// Which heads are rolled by -G/2. kShiftHalf: the second half of the heads (the method's
+// definition). kShiftAlternate: every odd kv head (the alternate-heads wording of the
+// pages' group figure). kShiftNone: no head (with G = N, dense causal attention).
+enum ShiftPattern : int { kShiftHalf = 0, kShiftAlternate = 1, kShiftNone = 2 };
+
+// A query head is shifted with its kv head (h -> h / (Hq/Hkv)). With Hkv even this is the
+// same as "h >= Hq/2" for the half pattern.
+__host__ __device__ inline bool kv_head_shifted(int kvh, const Params& p) {
+  if (p.shift == kShiftAlternate) return (kvh & 1) != 0;
+  if (p.shift == kShiftNone) return false;
+  return kvh >= p.Hkv / 2;
+}
+__host__ __device__ inline bool q_head_shifted(int h, const Params& p) {
+  return kv_head_shifted(h / (p.Hq / p.Hkv), p);
+}
 
 // Rolled row r -> original token. Rolling by -G/2 puts token (r + G/2) mod N at row r.
 __host__ __device__ inline int src_row(int r, bool shifted, int G, int N) {

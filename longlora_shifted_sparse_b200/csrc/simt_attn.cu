@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Params p) {
   const int h = (int)((warp / p.N) % p.Hq);
   const int b = (int)(warp / ((long)p.N * p.Hq));
   const int kvh = h / (p.Hq / p.Hkv);
-  const bool sh = head_shifted(h, p.Hq);
+  const bool sh = q_head_shifted(h, p);
   const int g = r / p.G, i = r - g * p.G;
   const int m = src_row(r, sh, p.G, p.N);
   const int d = p.d;
@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(256) simt_dq_kernel(Params p) {
   const int h = (int)((warp / p.N) % p.Hq);
   const int b = (int)(warp / ((long)p.N * p.Hq));
   const int kvh = h / (p.Hq / p.Hkv);
-  const bool sh = head_shifted(h, p.Hq);
+  const bool sh = q_head_shifted(h, p);
   const int g = r / p.G, i = r - g * p.G;
   const int m = src_row(r, sh, p.G, p.N);
   const int d = p.d;
@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(256) simt_dkdv_kernel(Params p) {
   const int kvh = (int)((warp / p.N) % p.Hkv);
   const int b = (int)(warp / ((long)p.N * p.Hkv));
   const int R = p.Hq / p.Hkv;
-  const bool sh = head_shifted(kvh, p.Hkv);
+  const bool sh = kv_head_shifted(kvh, p);
   const int g = r / p.G, j = r - g * p.G;
   const int m = src_row(r, sh, p.G, p.N);
   const int d = p.d;

@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bkg = (int)(blockIdx.x / T);
   const int g = bkg % ng, bk = bkg / ng;
   const int kvh = bk % p.Hkv, b = bk / p.Hkv;
-  const bool sh = head_shifted(kvh, p.Hkv);
+  const bool sh = kv_head_shifted(kvh, p);
   const int it0 = p.causal ? kt : 0;
   const int nq = T - it0;      // query tiles per query head
   const int np = R * nq;       // (query head, query tile) pairs
@@ -524,7 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int g = bkg % ng, bk = bkg / ng;
   const int kvh = bk % p.Hkv, b = bk / p.Hkv;
   const int h = kvh * R + inner % R;
-  const bool sh = head_shifted(h, p.Hq);
+  const bool sh = q_head_shifted(h, p);
   const int nkv = p.causal ? qt + 1 : T;
   const int mq0 = src_row(g * p.G + qt * kTile, sh, p.G, p.N);
 

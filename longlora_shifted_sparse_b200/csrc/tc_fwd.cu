@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int g = bkg % ng, bk = bkg / ng;
   const int kvh = bk % p.Hkv, b = bk / p.Hkv;
   const int h = kvh * R + inner % R;
-  const bool sh = head_shifted(h, p.Hq);
+  const bool sh = q_head_shifted(h, p);
   const int qt0 = 2 * pr;                                  // tile A; tile B = qt0 + 1
   const int nA = p.causal ? qt0 + 1 : T;                   // key tiles of tile A
   const int nB = p.causal ? qt0 + 2 : T;                   // key tiles of tile B (>= nA)

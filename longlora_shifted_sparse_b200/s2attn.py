@@ -21,6 +21,8 @@ LIB_PATH = os.path.join(_HERE, "libs2attn.so")
 S2_OK, S2_ERR_NULL, S2_ERR_SHAPE, S2_ERR_DTYPE, S2_ERR_HEADDIM, S2_ERR_ALIGN, \
     S2_ERR_WORKSPACE, S2_ERR_CUDA, S2_ERR_DEVICE_TIMEOUT, S2_ERR_ARG = range(10)
 S2_BF16, S2_FP32 = 0, 1
+S2_CAUSAL, S2_SHIFT_HALF, S2_SHIFT_ALTERNATE, S2_SHIFT_NONE = 0x01, 0x00, 0x10, 0x20
+SHIFT_PATTERNS = {"half": S2_SHIFT_HALF, "alternate": S2_SHIFT_ALTERNATE, "none": S2_SHIFT_NONE}
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # S2ATTN_NOALLOC_SCRATCH_BYTES
 
 if not os.path.exists(LIB_PATH):
@@ -130,6 +132,13 @@ def _stream_ptr(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+def mode(causal: bool = True, shift: str = "half") -> int:
+    """The ABI's mode argument: the causal flag ORed with a shifted-head pattern."""
+    if shift not in SHIFT_PATTERNS:
+        raise ValueError("shift must be one of %s, got %r" % (sorted(SHIFT_PATTERNS), shift))
+    return (S2_CAUSAL if causal else 0) | SHIFT_PATTERNS[shift]
+
+
 def workspace(B, N, Hq, Hkv, d, dtype_code, device):
     import torch
     nbytes = s2attn_workspace_bytes(B, N, Hq, Hkv, d, dtype_code)
@@ -139,8 +148,9 @@ def workspace(B, N, Hq, Hkv, d, dtype_code, device):
 
 
 def forward(q, k, v, G: int, pi_scale: float, rope_base: float = 10000.0, causal: bool = True,
-            ws=None, out=None, lse=None):
-    """q [B,N,Hq,d], k/v [B,N,Hkv,d] CUDA tensors -> (o, lse)."""
+            ws=None, out=None, lse=None, shift: str = "half"):
+    """q [B,N,Hq,d], k/v [B,N,Hkv,d] CUDA tensors -> (o, lse). shift picks the shifted
+    heads: "half" (the method), "alternate" (odd kv heads) or "none"."""
     import torch
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
@@ -150,13 +160,14 @@ def forward(q, k, v, G: int, pi_scale: float, rope_base: float = 10000.0, causal
     o = out if out is not None else torch.empty_like(q)
     lse = lse if lse is not None else torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
     check(s2attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                     B, N, Hq, Hkv, d, G, int(causal), pi_scale, rope_base, dt,
+                     B, N, Hq, Hkv, d, G, mode(causal, shift), pi_scale, rope_base, dt,
                      ws.data_ptr(), ws.numel(), _stream_ptr(q.device)))
     return o, lse
 
 
 def backward(q, k, v, o, lse, dout, G: int, pi_scale: float, rope_base: float = 10000.0,
-             causal: bool = True, ws=None, grads=None, after_forward: bool = False):
+             causal: bool = True, ws=None, grads=None, after_forward: bool = False,
+             shift: str = "half"):
     """Returns (dq, dk, dv) for the forward that produced (o, lse).
 
     after_forward=True calls s2attn_bwd_after_fwd: `ws` must then be the workspace the
@@ -175,7 +186,7 @@ def backward(q, k, v, o, lse, dout, G: int, pi_scale: float, rope_base: float = 
     fn = s2attn_bwd_after_fwd if after_forward else s2attn_bwd
     check(fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                      dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                     B, N, Hq, Hkv, d, G, int(causal), pi_scale, rope_base, dt,
+                     B, N, Hq, Hkv, d, G, mode(causal, shift), pi_scale, rope_base, dt,
                      ws.data_ptr(), ws.numel(), _stream_ptr(q.device)))
     return dq, dk, dv
 
@@ -192,24 +203,24 @@ def _make_function():
         """Autograd wrapper: o = S2Attn(q, k, v); backward through the library's kernels."""
 
         @staticmethod
-        def forward(ctx, q, k, v, G, pi_scale, rope_base=10000.0, causal=True):
+        def forward(ctx, q, k, v, G, pi_scale, rope_base=10000.0, causal=True, shift="half"):
             q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
             B, N, Hq, d = q.shape
             ws = workspace(B, N, Hq, k.shape[2], d, _dtype_code(q), q.device)
-            o, lse = forward(q, k, v, G, pi_scale, rope_base, causal, ws=ws)
+            o, lse = forward(q, k, v, G, pi_scale, rope_base, causal, ws=ws, shift=shift)
             # the workspace keeps the rotated q, k for the backward (q, k are saved too, so
             # autograd's version check catches an in-place change in between)
             ctx.save_for_backward(q, k, v, o, lse, ws)
-            ctx.args = (G, pi_scale, rope_base, causal)
+            ctx.args = (G, pi_scale, rope_base, causal, shift)
             return o
 
         @staticmethod
         def backward(ctx, do):
             q, k, v, o, lse, ws = ctx.saved_tensors
-            G, pi_scale, rope_base, causal = ctx.args
+            G, pi_scale, rope_base, causal, shift = ctx.args
             dq, dk, dv = backward(q, k, v, o, lse, do.contiguous(), G, pi_scale, rope_base, causal,
-                                  ws=ws, after_forward=True)
-            return dq, dk, dv, None, None, None, None
+                                  ws=ws, after_forward=True, shift=shift)
+            return dq, dk, dv, None, None, None, None, None
 
     return S2AttnFunction
 
@@ -218,9 +229,9 @@ _fn = None
 
 
 def s2_attention(q, k, v, G: int, pi_scale: float, rope_base: float = 10000.0,
-                 causal: bool = True):
+                 causal: bool = True, shift: str = "half"):
     """Differentiable S2-Attn on CUDA tensors."""
     global _fn
     if _fn is None:
         _fn = _make_function()
-    return _fn.apply(q, k, v, G, pi_scale, rope_base, causal)
+    return _fn.apply(q, k, v, G, pi_scale, rope_base, causal, shift)

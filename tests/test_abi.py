@@ -57,6 +57,26 @@ def test_kernel_path_rule(lib):
     assert lib.s2attn_kernel_path(1, 256, 4, 4, 64, 60, 1, lib.S2_FP32) == -1
     assert lib.s2attn_kernel_path(1, 256, 4, 4, 64, 64, 2, lib.S2_FP32) == -1
     assert lib.s2attn_kernel_path(1, 256, 4, 4, 64, 64, 1, 5) == -1
+    # mode: S2_CAUSAL or 0, ORed with one S2_SHIFT_* pattern
+    for m in (0x00, 0x01, 0x10, 0x11, 0x20, 0x21):
+        assert lib.s2attn_kernel_path(1, 1024, 4, 4, 128, 256, m, lib.S2_BF16) == 1
+    for m in (0x30, 0x31, 0x02, 0x40, 0x100, -1):
+        assert lib.s2attn_kernel_path(1, 1024, 4, 4, 128, 256, m, lib.S2_BF16) == -1
+
+
+def test_mode_flags_match_header(lib):
+    text = open(os.path.join(ROOT, "include", "s2attn.h")).read()
+    defs = dict(re.findall(r"#define\s+(S2_(?:CAUSAL|SHIFT_\w+))\s+(0x[0-9a-fA-F]+)", text))
+    assert set(defs) == {"S2_CAUSAL", "S2_SHIFT_HALF", "S2_SHIFT_ALTERNATE", "S2_SHIFT_NONE"}
+    for name, val in defs.items():
+        assert getattr(lib, name) == int(val, 16), name
+
+
+def test_mode_helper(lib):
+    assert lib.mode(True) == 1 and lib.mode(False) == 0
+    assert lib.mode(True, "alternate") == 0x11 and lib.mode(False, "none") == 0x20
+    with pytest.raises(ValueError):
+        lib.mode(True, "odd")
 
 
 # fake but aligned, non-null device addresses: the calls below must fail in validation,
@@ -90,6 +110,7 @@ def _bwd(lib, **kw):
     (dict(q=P + 8), 5), (dict(o=P + 2), 5), (dict(ws=P + 4), 5),
     (dict(ws=None), 6), (dict(wsb=1000), 6),
     (dict(s=0.0), 9), (dict(s=float("nan")), 9), (dict(base=-1.0), 9), (dict(causal=3), 9),
+    (dict(causal=0x31), 9), (dict(causal=0x41), 9), (dict(causal=0x30), 9),
 ])
 def test_fwd_rejects_bad_arguments(lib, kw, code):
     assert _fwd(lib, **kw) == code

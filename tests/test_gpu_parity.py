@@ -24,11 +24,12 @@ def s2():
 
 def _run(s2, w, q, k, v, do):
     tq, tk, tv = (H.to_device(x, w.dtype) for x in (q, k, v))
-    o, lse = s2.forward(tq, tk, tv, w.G, w.pi_scale, w.rope_base, w.causal)
+    o, lse = s2.forward(tq, tk, tv, w.G, w.pi_scale, w.rope_base, w.causal, shift=w.shift)
     grads = None
     if do is not None:
         tdo = H.to_device(do, w.dtype)
-        grads = s2.backward(tq, tk, tv, o, lse, tdo, w.G, w.pi_scale, w.rope_base, w.causal)
+        grads = s2.backward(tq, tk, tv, o, lse, tdo, w.G, w.pi_scale, w.rope_base, w.causal,
+                            shift=w.shift)
     torch.cuda.synchronize()
     return o, lse, grads
 
@@ -36,11 +37,11 @@ def _run(s2, w, q, k, v, do):
 def _full_compare(s2, w):
     q, k, v, do = H.inputs(w, with_dout=w.backward)
     o, lse, grads = _run(s2, w, q, k, v, do)
-    o_ref, lse_ref = oracle.fwd(q, k, v, w.G, w.pi_scale, w.rope_base, w.causal)
+    o_ref, lse_ref = oracle.fwd(q, k, v, w.G, w.pi_scale, w.rope_base, w.causal, shift=w.shift)
     H.assert_close_o(H.to_host_f64(o), o_ref, w.dtype)
     H.assert_close_lse(H.to_host_f64(lse), lse_ref, w.dtype)
     if grads is not None:
-        refs = oracle.bwd(q, k, v, do, w.G, w.pi_scale, w.rope_base, w.causal)
+        refs = oracle.bwd(q, k, v, do, w.G, w.pi_scale, w.rope_base, w.causal, shift=w.shift)
         for name, g, r in zip(("dq", "dk", "dv"), grads, refs):
             H.assert_close_grad(H.to_host_f64(g), r, w.dtype, name)
 
@@ -75,6 +76,61 @@ def test_small_shapes_full(s2, case):
     _full_compare(s2, w)
 
 
+# The other head patterns, the full-group (no mask) reading and RoPE base scaling, on both
+# kernel families: Workload(name, B, N, Hq, Hkv, d, G, s, dtype, in_scale, backward, seed, ...)
+VARIANTS = [
+    Workload("bf16_alternate", 1, 1024, 4, 4, 128, 256, 2.0, "bf16", 0.5, True, 120,
+             shift="alternate"),
+    Workload("bf16_alternate_gqa_b2", 2, 1024, 8, 4, 128, 512, 4.0, "bf16", 0.5, True, 121,
+             shift="alternate"),
+    Workload("bf16_alternate_noncausal", 1, 1024, 4, 2, 128, 256, 2.0, "bf16", 0.5, True, 122,
+             causal=False, shift="alternate"),
+    Workload("bf16_none_dense_causal", 1, 1024, 4, 4, 128, 1024, 1.0, "bf16", 0.5, True, 123,
+             shift="none"),
+    Workload("bf16_none_groups_gqa", 1, 1024, 4, 2, 128, 256, 2.0, "bf16", 0.5, True, 124,
+             shift="none"),
+    Workload("bf16_base_scaled", 1, 1024, 4, 4, 128, 256, 1.0, "bf16", 0.5, True, 125,
+             rope_base=80000.0),
+    Workload("bf16_d64_alternate", 1, 512, 4, 4, 64, 64, 2.0, "bf16", 0.5, True, 126,
+             shift="alternate"),
+    Workload("f32_alternate_gqa", 1, 384, 4, 2, 64, 96, 3.0, "f32", 1.0, True, 127,
+             shift="alternate"),
+    Workload("f32_none_dense_causal", 1, 256, 2, 2, 64, 256, 1.0, "f32", 1.0, True, 128,
+             shift="none"),
+    Workload("f32_base_scaled_noncausal", 1, 256, 4, 4, 64, 64, 1.0, "f32", 1.0, True, 129,
+             causal=False, rope_base=40000.0),
+]
+
+
+@pytest.mark.parametrize("w", VARIANTS, ids=[w.name for w in VARIANTS])
+def test_variants_full(s2, w):
+    expect_tc = w.dtype == "bf16" and w.d == 128 and w.G % 256 == 0
+    code = s2.S2_BF16 if w.dtype == "bf16" else s2.S2_FP32
+    assert s2.s2attn_kernel_path(w.B, w.N, w.Hq, w.Hkv, w.d, w.G, s2.mode(w.causal, w.shift),
+                                 code) == int(expect_tc)
+    _full_compare(s2, w)
+
+
+def test_no_shift_one_group_matches_sdpa(s2):
+    """Pattern "none" with G = N on the tensor-core path against torch's causal SDPA (fp64,
+    CPU) on the rotated inputs: a library routine, independent of the oracle's attention."""
+    w = Workload("sdpa", 1, 1024, 4, 4, 128, 1024, 1.0, "bf16", 0.5, False, 130, shift="none")
+    q, k, v, _ = H.inputs(w, with_dout=False)
+    o, _, _ = _run(s2, w, q, k, v, None)
+    pos = np.arange(w.N)
+
+    def rotated(x):
+        xf = synth.bf16_bits_to_f32(x).astype(np.float64)[0]
+        return np.stack([oracle.rope(xf[:, h], pos, w.pi_scale, w.rope_base)
+                         for h in range(xf.shape[1])])          # [H, N, d]
+
+    vf = synth.bf16_bits_to_f32(v).astype(np.float64)[0].transpose(1, 0, 2)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(rotated(q)), torch.from_numpy(rotated(k)), torch.from_numpy(vf),
+        is_causal=True).numpy().transpose(1, 0, 2)[None]
+    H.assert_close_o(H.to_host_f64(o), ref, "bf16")
+
+
 def _sampled_fwd_check(w, q, k, v, o, lse):
     ng = w.N // w.G
     heads = sorted({0, w.Hq // 2 - 1, w.Hq // 2, w.Hq - 1})
@@ -84,9 +140,9 @@ def _sampled_fwd_check(w, q, k, v, o, lse):
     for h in heads:
         kvh = h // (w.Hq // w.Hkv)
         for g in groups:
-            tok = oracle.unit_rows(w.N, w.G, w.Hq, kvh, w.Hkv, g)[rows]
+            tok = oracle.unit_rows(w.N, w.G, w.Hq, kvh, w.Hkv, g, shift=w.shift)[rows]
             o_r, l_r = oracle.fwd_rows(q, k, v, w.G, w.pi_scale, 0, h, g, rows, w.rope_base,
-                                       w.causal)
+                                       w.causal, shift=w.shift)
             idx = torch.as_tensor(tok, device=o.device)
             got_o.append(H.to_host_f64(o[0, idx, h]))
             got_l.append(H.to_host_f64(lse[0, h, idx]))
@@ -102,9 +158,9 @@ def _sampled_bwd_check(w, q, k, v, do, grads, units):
     rows = H.sample_rows(w.G, extra=4, seed=1)
     gq, rq, gk, rk, gv, rv = [], [], [], [], [], []
     for (b, kvh, g) in units:
-        tok = oracle.unit_rows(w.N, w.G, w.Hq, kvh, w.Hkv, g)[rows]
+        tok = oracle.unit_rows(w.N, w.G, w.Hq, kvh, w.Hkv, g, shift=w.shift)[rows]
         dq_r, dk_r, dv_r = oracle.bwd_rows(q, k, v, do, w.G, w.pi_scale, b, kvh, g, rows, rows,
-                                           w.rope_base, w.causal)
+                                           w.rope_base, w.causal, shift=w.shift)
         idx = torch.as_tensor(tok, device=dq.device)
         gq.append(H.to_host_f64(dq[b, idx, kvh * R:(kvh + 1) * R]))
         rq.append(dq_r)
@@ -117,7 +173,9 @@ def _sampled_bwd_check(w, q, k, v, do, grads, units):
     H.assert_close_grad(np.concatenate(gv), np.concatenate(rv), w.dtype, "dv")
 
 
-BIG = ["llama2_7b_8k_fwd", "llama2_7b_32k", "llama2_70b_gqa_32k", "llama2_7b_100k"]
+BIG = ["llama2_7b_8k_fwd", "llama2_7b_32k", "llama2_70b_gqa_32k", "llama2_7b_100k",
+       "llama2_7b_32k_noncausal", "llama2_7b_32k_alternate", "llama2_7b_32k_base_scaled",
+       "llama2_7b_32k_dense_infer"]
 
 
 @pytest.mark.parametrize("name", BIG)
@@ -126,7 +184,8 @@ def test_llama2_workload_sampled(s2, name):
     (wrap) groups; dq/dk/dv on sampled rows of units in both halves incl. the wrap group."""
     w = WORKLOADS[name]
     # these shapes must take the tensor-core kernels
-    assert s2.s2attn_kernel_path(w.B, w.N, w.Hq, w.Hkv, w.d, w.G, int(w.causal), s2.S2_BF16) == 1
+    assert s2.s2attn_kernel_path(w.B, w.N, w.Hq, w.Hkv, w.d, w.G, s2.mode(w.causal, w.shift),
+                                 s2.S2_BF16) == 1
     q, k, v, do = H.inputs(w, with_dout=w.backward)
     o, lse, grads = _run(s2, w, q, k, v, do)
     _sampled_fwd_check(w, q, k, v, o, lse)
@@ -262,9 +321,9 @@ def test_softmax_rescale_paths(s2):
     grows = sum(sc[i, :i + 1].max() > sc[i, :128].max() + 8 for i in range(128, w.G))
     assert grows > 100, grows
     o, lse, grads = _run(s2, w, q, k, v, do)
-    o_ref, lse_ref = oracle.fwd(q, k, v, w.G, w.pi_scale, w.rope_base, w.causal)
+    o_ref, lse_ref = oracle.fwd(q, k, v, w.G, w.pi_scale, w.rope_base, w.causal, shift=w.shift)
     H.assert_close_o(H.to_host_f64(o), o_ref, w.dtype)
     H.assert_close_lse(H.to_host_f64(lse), lse_ref, w.dtype)
-    refs = oracle.bwd(q, k, v, do, w.G, w.pi_scale, w.rope_base, w.causal)
+    refs = oracle.bwd(q, k, v, do, w.G, w.pi_scale, w.rope_base, w.causal, shift=w.shift)
     for name, g, r in zip(("dq", "dk", "dv"), grads, refs):
         H.assert_close_grad(H.to_host_f64(g), r, w.dtype, name)

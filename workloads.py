@@ -26,6 +26,7 @@ class Workload:
     seed: int
     causal: bool = True
     rope_base: float = 10000.0
+    shift: str = "half"  # shifted heads: "half", "alternate" (odd kv heads) or "none"
 
 
 WORKLOADS = {
@@ -37,6 +38,19 @@ WORKLOADS = {
         Workload("llama2_70b_gqa_32k", 1, 32768, 64, 8, 128, 8192, 8.0, "bf16", 0.5, True, 4),
         # a smaller case of the same shape family for ncu captures (q is 134 MB > L2)
         Workload("llama2_7b_16k", 1, 16384, 32, 32, 128, 4096, 4.0, "bf16", 0.5, True, 5),
+        # variants of the 7B-32k step: no mask inside the groups (the full-group reading);
+        # odd kv heads shifted instead of the second half; RoPE base scaled by the extension
+        # ratio instead of interpolated positions (base 10000 * 8, s = 1)
+        Workload("llama2_7b_32k_noncausal", 1, 32768, 32, 32, 128, 8192, 8.0, "bf16", 0.5,
+                 True, 6, causal=False),
+        Workload("llama2_7b_32k_alternate", 1, 32768, 32, 32, 128, 8192, 8.0, "bf16", 0.5,
+                 True, 7, shift="alternate"),
+        Workload("llama2_7b_32k_base_scaled", 1, 32768, 32, 32, 128, 8192, 1.0, "bf16", 0.5,
+                 True, 8, rope_base=80000.0),
+        # inference at the extended length: one group of all 32k tokens, no shift, i.e.
+        # dense causal attention, forward only
+        Workload("llama2_7b_32k_dense_infer", 1, 32768, 32, 32, 128, 32768, 8.0, "bf16", 0.5,
+                 False, 9, shift="none"),
     ]
 }
 
