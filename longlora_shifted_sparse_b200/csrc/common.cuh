@@ -50,6 +50,20 @@ __host__ __device__ inline bool q_head_shifted(int h, const Params& p) {
   return kv_head_shifted(h / (p.Hq / p.Hkv), p);
 }
 
+// Work order of the tensor-core kernels: CTA x of a grid of U units (b, kv head, group)
+// times W items per unit -> (unit, item), item 0 being a unit's heaviest item. Units are
+// taken kLptChunk at a time; inside a chunk the items run heaviest first across all of the
+// chunk's units. The last wave then holds only light items (longest-processing-time order,
+// a short tail), while the few units in flight keep the tiles they share resident in L2.
+constexpr int kLptChunk = 8;
+__device__ inline void chunked_lpt(int x, int U, int W, int& unit, int& item) {
+  const int c0 = x / (kLptChunk * W) * kLptChunk;
+  const int cc = min(kLptChunk, U - c0);
+  const int r = x - c0 * W;
+  item = r / cc;
+  unit = c0 + (r - item * cc);
+}
+
 // Rolled row r -> original token. Rolling by -G/2 puts token (r + G/2) mod N at row r.
 __host__ __device__ inline int src_row(int r, bool shifted, int G, int N) {
   if (!shifted) return r;

@@ -197,9 +197,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.G / kTile, ng = p.N / p.G, R = p.Hq / p.Hkv;
-  // head-group-major: the key tiles of one (b, kv head, group) run together, heaviest first
-  const int kt = (int)(blockIdx.x % T);
-  const int bkg = (int)(blockIdx.x / T);
+  // the key tiles of a few (b, kv head, group) units run together (they stream the same Q
+  // and dO through L2), heaviest first: key tile kt sees T - kt query tiles when causal
+  int kt, bkg;
+  chunked_lpt((int)blockIdx.x, p.B * p.Hkv * ng, T, bkg, kt);
   const int g = bkg % ng, bk = bkg / ng;
   const int kvh = bk % p.Hkv, b = bk / p.Hkv;
   const bool sh = kv_head_shifted(kvh, p);
@@ -515,11 +516,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.G / kTile, ng = p.N / p.G, R = p.Hq / p.Hkv;
-  // head-group-major: the query tiles of all query heads of one (b, kv head, group) run
-  // together (they share K and V), heaviest query tiles first
-  const int per_kg = T * R;
-  const int inner = (int)(blockIdx.x % per_kg);
-  const int bkg = (int)(blockIdx.x / per_kg);
+  // the query tiles of all query heads of a few (b, kv head, group) units run together
+  // (they share K and V through L2), heaviest query tiles first
+  int inner, bkg;
+  chunked_lpt((int)blockIdx.x, p.B * p.Hkv * ng, T * R, bkg, inner);
   const int qt = T - 1 - inner / R;
   const int g = bkg % ng, bk = bkg / ng;
   const int kvh = bk % p.Hkv, b = bk / p.Hkv;

@@ -190,11 +190,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.G / kTile, ng = p.N / p.G, R = p.Hq / p.Hkv;
-  // head-group-major: the tile pairs of all query heads of one (b, kv head, group) run
-  // together (they stream the same K and V through L2), heaviest pairs first
-  const int per_kg = (T / 2) * R;
-  const int inner = (int)(blockIdx.x % per_kg);
-  const int bkg = (int)(blockIdx.x / per_kg);
+  // the tile pairs of all query heads of a few (b, kv head, group) units run together (they
+  // stream the same K and V through L2), heaviest pairs first
+  int inner, bkg;
+  chunked_lpt((int)blockIdx.x, p.B * p.Hkv * ng, (T / 2) * R, bkg, inner);
   const int pr = T / 2 - 1 - inner / R;
   const int g = bkg % ng, bk = bkg / ng;
   const int kvh = bk % p.Hkv, b = bk / p.Hkv;
