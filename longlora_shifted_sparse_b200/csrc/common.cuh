@@ -33,6 +33,9 @@ struct Params {
 };
 
 enum StatusBits : unsigned { kStatusTimeout = 1u };
+// Words after the status word (same 256-byte block of the workspace): the persistent
+// forward's work-item counter, zeroed by the RoPE pass at the start of every forward.
+constexpr int kFwdWorkCounter = 1;
 
 // Which heads are rolled by -G/2. kShiftHalf: the second half of the heads (the method's
 // definition). kShiftAlternate: every odd kv head (the alternate-heads wording of the

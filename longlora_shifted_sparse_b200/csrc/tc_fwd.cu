@@ -29,8 +29,12 @@
 //                columns of O / l (l = sum of both partial sums) as bf16 at the token's
 //                original row; LSE = ln 2 * (m + log2 l).
 // TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
-// CTAs are launched head-group-major (all tile pairs of the query heads that share one kv
-// head and group, heaviest first), so concurrently running CTAs reuse K and V from L2.
+// Persistent CTAs (one per SM) take work items from a counter in the workspace. Items are
+// numbered a few (b, kv head, group) units at a time, the heaviest tile pairs of those units
+// first, so the items in flight reuse K and V from L2 and the last items are light. Between
+// two items of a CTA the producer and the issuer run ahead: the next item's Q tiles load
+// once the last QK^T of the current one has completed, and its first QK^T MMAs run while
+// the softmax warps write the current item's output.
 // Every wait is bounded; on expiry the CTA records it in the status word and drains.
 #include "common.cuh"
 #include "fastmath.cuh"
@@ -78,7 +82,7 @@ constexpr uint32_t kOffV = 4 * kTileBytes;
 constexpr uint32_t kSmemBytes = 6 * kTileBytes + 1024;
 
 struct FwdBarriers {
-  uint64_t q_full;
+  uint64_t q_full, q_empty;
   uint64_t k_full[2], k_empty[2];
   uint64_t v_full[2], v_empty[2];
   uint64_t s_full[2], p_full[2], o_final[2];  // index: query tile A = 0, B = 1
@@ -175,40 +179,60 @@ __device__ __forceinline__ void load_s64(uint32_t tS, bool diag, int first_col, 
   }
 }
 
+// A work item: two consecutive 128-row query tiles (A = qt0, B = qt0 + 1) of one
+// (batch, query head, group). Items are numbered in the chunked longest-first order.
+struct FwdItem {
+  int b, h, kvh, g, qt0, nA, nB, r0;
+  bool sh;
+};
+
+__device__ __forceinline__ FwdItem decode_item(const Params& p, int item) {
+  const int T = p.G / kTile, ng = p.N / p.G, R = p.Hq / p.Hkv;
+  int inner, bkg;
+  chunked_lpt(item, p.B * p.Hkv * ng, (T / 2) * R, bkg, inner);
+  FwdItem it;
+  const int pr = T / 2 - 1 - inner / R;
+  it.g = bkg % ng;
+  const int bk = bkg / ng;
+  it.kvh = bk % p.Hkv;
+  it.b = bk / p.Hkv;
+  it.h = it.kvh * R + inner % R;
+  it.sh = q_head_shifted(it.h, p);
+  it.qt0 = 2 * pr;
+  it.nA = p.causal ? it.qt0 + 1 : T;   // key tiles of tile A
+  it.nB = p.causal ? it.qt0 + 2 : T;   // key tiles of tile B (>= nA)
+  it.r0 = it.g * p.G + it.qt0 * kTile; // rolled row of tile A's row 0
+  return it;
+}
+
+// Persistent: one CTA per SM takes work items from a counter in the workspace (zeroed by
+// the RoPE pass that precedes every forward) until none is left. While the softmax warps
+// finish one item (last key tiles, epilogue), the producer already loads the next item's
+// query tiles and key tiles and the issuer runs its first QK^T MMAs.
 __global__ void __launch_bounds__(kThreads, 1)
     tc_fwd_kernel(const Params p, const __grid_constant__ CUtensorMap tm_q,
-                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v) {
+                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  int nitems) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   __shared__ FwdBarriers bars;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
+  // the CTA's k-th work item sits in slot k & 1 (-1: no more work), published with q_full
+  __shared__ int item_slot[2];
   // row-max exchange between the two warps that share a row: [parity][tile][half][row]
   __shared__ float xmax[2][2][2][kTile];
   __shared__ float xsum[2][kTile];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int T = p.G / kTile, ng = p.N / p.G, R = p.Hq / p.Hkv;
-  // the tile pairs of all query heads of a few (b, kv head, group) units run together (they
-  // stream the same K and V through L2), heaviest pairs first
-  int inner, bkg;
-  chunked_lpt((int)blockIdx.x, p.B * p.Hkv * ng, (T / 2) * R, bkg, inner);
-  const int pr = T / 2 - 1 - inner / R;
-  const int g = bkg % ng, bk = bkg / ng;
-  const int kvh = bk % p.Hkv, b = bk / p.Hkv;
-  const int h = kvh * R + inner % R;
-  const bool sh = q_head_shifted(h, p);
-  const int qt0 = 2 * pr;                                  // tile A; tile B = qt0 + 1
-  const int nA = p.causal ? qt0 + 1 : T;                   // key tiles of tile A
-  const int nB = p.causal ? qt0 + 2 : T;                   // key tiles of tile B (>= nA)
-  const int r0 = g * p.G + qt0 * kTile;                    // rolled row of tile A's row 0
+  unsigned* const next_item = p.status + kFwdWorkCounter;
 
   Abort ab{&abort_flag, p.status};
   if (threadIdx.x == 0) {
-    // a CTA of this launch already gave up: do nothing (outputs are undefined then)
-    abort_flag = *reinterpret_cast<volatile unsigned*>(p.status) != 0u;
+    abort_flag = 0;
     mbar_init(smem_addr(&bars.q_full), 1);
+    mbar_init(smem_addr(&bars.q_empty), 1);
     for (int s = 0; s < 2; s++) {
       mbar_init(smem_addr(&bars.k_full[s]), 1);
       mbar_init(smem_addr(&bars.k_empty[s]), 1);
@@ -227,98 +251,119 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
   const uint32_t sQ = smem_addr(smem + kOffQ);
-  const bool skip = abort_flag != 0;
 
   if (warp < 4) {
     // warpgroup 0 (TMA producer, MMA issuer, two idle warps) gives registers away
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
-    if (!skip && warp == 0) {
+    if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------------ TMA producer
-      if (lane == 0) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      int nk = 0, nv = 0;            // K and V tiles loaded so far (ring positions)
+      int q_last = -1;               // item index (k) of the latest Q load, -1 after the stop
+      for (int k = 0, ok = 1; ok; k++) {
+        int item = (int)atomicAdd(next_item, 1u);
+        // stop when the work is done or a CTA of this launch gave up
+        if (item >= nitems || *reinterpret_cast<volatile unsigned*>(p.status) != 0u) item = -1;
+        // the query tiles of the previous item are no longer read
+        if (k > 0 && !mbar_wait(smem_addr(&bars.q_empty), (k - 1) & 1, ab)) break;
+        item_slot[k & 1] = item;
         const uint32_t qb = smem_addr(&bars.q_full);
+        if (item < 0) {
+          mbar_arrive(qb);  // completes the phase: the consumers read -1 and stop
+          q_last = -1;
+          break;
+        }
+        const FwdItem it = decode_item(p, item);
         mbar_arrive_expect_tx(qb, 2 * kTileBytes);
         for (int t = 0; t < 2; t++) {
-          const int qrow = (b * p.Hq + h) * p.N + src_row(r0 + t * kTile, sh, p.G, p.N);
+          const int qrow = (it.b * p.Hq + it.h) * p.N + src_row(it.r0 + t * kTile, it.sh, p.G, p.N);
           tma_load_2d(sQ + t * kTileBytes, &tm_q, qb, 0, qrow);
           tma_load_2d(sQ + t * kTileBytes + kHalfBytes, &tm_q, qb, 64, qrow);
         }
-        int issued = 0;
-        for (int j = 0; j < nB; j++) {
-          const int s = j & 1;
-          const uint32_t ph = (j >> 1) & 1;
-          const int mk = src_row(g * p.G + j * kTile, sh, p.G, p.N);
-          if (!mbar_wait(smem_addr(&bars.k_empty[s]), ph ^ 1, ab)) break;
+        q_last = k;
+        const int krow0 = (it.b * p.Hkv + it.kvh) * p.N;
+        for (int j = 0; j < it.nB; j++) {
+          const int s = nk & 1;
+          const uint32_t ph = (nk >> 1) & 1;
+          const int mk = src_row(it.g * p.G + j * kTile, it.sh, p.G, p.N);
+          if (!mbar_wait(smem_addr(&bars.k_empty[s]), ph ^ 1, ab)) { ok = 0; break; }
           const uint32_t sK = smem_addr(smem + kOffK + s * kTileBytes);
           mbar_arrive_expect_tx(smem_addr(&bars.k_full[s]), kTileBytes);
-          tma_load_2d(sK, &tm_k, smem_addr(&bars.k_full[s]), 0, (b * p.Hkv + kvh) * p.N + mk);
-          tma_load_2d(sK + kHalfBytes, &tm_k, smem_addr(&bars.k_full[s]), 64,
-                      (b * p.Hkv + kvh) * p.N + mk);
-          if (!mbar_wait(smem_addr(&bars.v_empty[s]), ph ^ 1, ab)) {
-            issued = 2 * j + 1;
-            break;
-          }
+          tma_load_2d(sK, &tm_k, smem_addr(&bars.k_full[s]), 0, krow0 + mk);
+          tma_load_2d(sK + kHalfBytes, &tm_k, smem_addr(&bars.k_full[s]), 64, krow0 + mk);
+          nk++;
+          if (!mbar_wait(smem_addr(&bars.v_empty[s]), ph ^ 1, ab)) { ok = 0; break; }
           const uint32_t sV = smem_addr(smem + kOffV + s * kTileBytes);
           mbar_arrive_expect_tx(smem_addr(&bars.v_full[s]), kTileBytes);
-          tma_load_3d(sV, &tm_v, smem_addr(&bars.v_full[s]), 0, kvh, b * p.N + mk);
-          tma_load_3d(sV + kHalfBytes, &tm_v, smem_addr(&bars.v_full[s]), 64, kvh, b * p.N + mk);
-          issued = 2 * j + 2;
+          tma_load_3d(sV, &tm_v, smem_addr(&bars.v_full[s]), 0, it.kvh, it.b * p.N + mk);
+          tma_load_3d(sV + kHalfBytes, &tm_v, smem_addr(&bars.v_full[s]), 64, it.kvh,
+                      it.b * p.N + mk);
+          nv++;
         }
-        // Let the last loads in flight land before the CTA can exit. This wait ignores the
-        // abort flag (it is set on this path) but keeps its own time limit.
-        int no_abort = 0;
-        Abort local{&no_abort, p.status};
-        for (int t = issued - 1; t >= 0 && t >= issued - 4; t--) {
-          const int j = t >> 1, s = j & 1;
-          const uint32_t ph = (j >> 1) & 1;
-          mbar_wait(smem_addr((t & 1) ? &bars.v_full[s] : &bars.k_full[s]), ph, local);
-        }
-        mbar_wait(qb, 0, local);
       }
-    } else if (!skip && warp == 1) {
+      // Let the loads in flight land before the CTA can exit: the last load into each ring
+      // stage (the latest phase of its barrier) and a query load not yet consumed. These
+      // waits ignore the abort flag (it may be set on this path) but keep their time limit.
+      int no_abort = 0;
+      Abort local{&no_abort, p.status};
+      for (int t = nk - 1; t >= 0 && t >= nk - 2; t--)
+        mbar_wait(smem_addr(&bars.k_full[t & 1]), (t >> 1) & 1, local);
+      for (int t = nv - 1; t >= 0 && t >= nv - 2; t--)
+        mbar_wait(smem_addr(&bars.v_full[t & 1]), (t >> 1) & 1, local);
+      if (q_last >= 0) mbar_wait(smem_addr(&bars.q_full), q_last & 1, local);
+    } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------------ MMA issuer
-      if (lane == 0) {
-        const uint32_t idesc_qk = idesc_bf16_f32(kTile, kTile, false, false);
-        const uint32_t idesc_pv = idesc_bf16_f32(kTile, kD, false, true);
-        // Descriptors are built once; a k-step or a stage only adds a constant to the start
-        // address field (bytes / 16; every address stays below 256 KB, so no carry leaves it).
-        // One thread issues every MMA while four softmax warps share its scheduler, so the
-        // issue path is kept to a few instructions per MMA.
-        const uint64_t dQ = smem_desc_sw128(sQ, 16, 1024);
-        const uint64_t dK = smem_desc_sw128(smem_addr(smem + kOffK), 16, 1024);
-        const uint64_t dV = smem_desc_sw128(smem_addr(smem + kOffV), kHalfBytes, 1024);
-        constexpr uint32_t kTileDesc = kTileBytes >> 4;
-        bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
+      const uint32_t idesc_qk = idesc_bf16_f32(kTile, kTile, false, false);
+      const uint32_t idesc_pv = idesc_bf16_f32(kTile, kD, false, true);
+      // Descriptors are built once; a k-step or a stage only adds a constant to the start
+      // address field (bytes / 16; every address stays below 256 KB, so no carry leaves it).
+      // One thread issues every MMA while four softmax warps share its scheduler, so the
+      // issue path is kept to a few instructions per MMA.
+      const uint64_t dQ = smem_desc_sw128(sQ, 16, 1024);
+      const uint64_t dK = smem_desc_sw128(smem_addr(smem + kOffK), 16, 1024);
+      const uint64_t dV = smem_desc_sw128(smem_addr(smem + kOffV), kHalfBytes, 1024);
+      constexpr uint32_t kTileDesc = kTileBytes >> 4;
+      int kv = 0;                        // ring position of the item's key tile 0
+      uint32_t pcnt[2] = {0u, 0u};       // p_full phases consumed per query tile
+      bool ok = true;
+      for (int k = 0; ok; k++) {
+        if (!mbar_wait(smem_addr(&bars.q_full), k & 1, ab)) break;
+        const int item = item_slot[k & 1];
+        if (item < 0) break;
+        const FwdItem it = decode_item(p, item);
         tc_fence_after();
-        for (int j = 0; ok && j <= nB; j++) {
-          const int jj = j - 1;
-          if (j >= 1) {
-            if (!mbar_wait(smem_addr(&bars.v_full[jj & 1]), (jj >> 1) & 1, ab)) break;
+        for (int j = 0; j <= it.nB; j++) {
+          const int gj = kv + j, gjj = gj - 1;   // ring positions of key tiles j and j - 1
+          if (j >= 1 && !mbar_wait(smem_addr(&bars.v_full[gjj & 1]), (gjj >> 1) & 1, ab)) {
+            ok = false;
+            break;
           }
-          if (j < nB) {
-            if (!mbar_wait(smem_addr(&bars.k_full[j & 1]), (j >> 1) & 1, ab)) break;
+          if (j < it.nB && !mbar_wait(smem_addr(&bars.k_full[gj & 1]), (gj >> 1) & 1, ab)) {
+            ok = false;
+            break;
           }
           tc_fence_after();
           // opaque per-iteration bases: the per-k-step descriptors are formed by one add at
           // their MMA instead of being hoisted out of the loop into (spilled) registers
-          const uint64_t dKj = opaque64(dK) + (uint64_t)((j & 1) * kTileDesc);
-          const uint64_t dVj = opaque64(dV) + (uint64_t)((jj & 1) * kTileDesc);
+          const uint64_t dKj = opaque64(dK) + (uint64_t)((gj & 1) * kTileDesc);
+          const uint64_t dVj = opaque64(dV) + (uint64_t)((gjj & 1) * kTileDesc);
           const uint64_t dQj = opaque64(dQ);
 #pragma unroll
           for (int t = 0; t < 2; t++) {
-            const int nt = t ? nB : nA;
+            const int nt = t ? it.nB : it.nA;
             const uint32_t tS = tmem + t * 128, tO = tmem + 256 + t * 128;
-            if (j >= 1 && jj < nt) {
-              if (!mbar_wait(smem_addr(&bars.p_full[t]), jj & 1, ab)) { ok = false; break; }
+            if (j >= 1 && j - 1 < nt) {
+              if (!mbar_wait(smem_addr(&bars.p_full[t]), pcnt[t] & 1, ab)) { ok = false; break; }
+              pcnt[t]++;
               tc_fence_after();
-              const uint32_t acc0 = jj > 0;
+              const uint32_t acc0 = j > 1;
 #pragma unroll
               for (int kk = 0; kk < kTile / 16; kk++)  // P of key rows 64h.. at column 64h;
                 mma_ts(tO, tS + (kk >> 2) * 64 + (kk & 3) * 8,  // V k-step = 16 rows
                        dVj + (uint64_t)(kk * (2048 >> 4)), idesc_pv, kk ? 1u : acc0);
-              if (jj == nt - 1) mma_commit(smem_addr(&bars.o_final[t]));
+              if (j == nt) mma_commit(smem_addr(&bars.o_final[t]));
             }
             if (j < nt) {
               const uint64_t dQt = dQj + (uint64_t)(t * kTileDesc);
@@ -331,38 +376,49 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (!ok) break;
-          if (j >= 1) mma_commit(smem_addr(&bars.v_empty[jj & 1]));
-          if (j < nB) mma_commit(smem_addr(&bars.k_empty[j & 1]));
+          if (j == it.nB - 1) mma_commit(smem_addr(&bars.q_empty));  // last QK^T of the item
+          if (j >= 1) mma_commit(smem_addr(&bars.v_empty[gjj & 1]));
+          if (j < it.nB) mma_commit(smem_addr(&bars.k_empty[gj & 1]));
         }
-        // every MMA issued above has completed before TMEM is released
-        mma_commit(smem_addr(&bars.drain));
-        int no_abort = 0;
-        Abort local{&no_abort, p.status};
-        mbar_wait(smem_addr(&bars.drain), 0, local);
+        kv += it.nB;
       }
+      // every MMA issued above has completed before TMEM is released
+      mma_commit(smem_addr(&bars.drain));
+      int no_abort = 0;
+      Abort local{&no_abort, p.status};
+      mbar_wait(smem_addr(&bars.drain), 0, local);
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
-    if (!skip) {
-      // ------------------------------------------------------------------ softmax / epilogue
-        // warps 4..11 tile A, 12..19 tile B; within a tile the first four warps take key columns
-      // 0..63 and the next four 64..127 of the same rows (lane quarter = warp % 4)
-      const int t = (warp - 4) >> 3;        // query tile
-      const int half = ((warp - 4) >> 2) & 1;
-      const int c0 = half * 64;             // this warp's 64 columns of S, P and O
-      const int qt = qt0 + t;
-      const int n = t ? nB : nA;
-      const int quarter = warp & 3;
-      const int row = quarter * 32 + lane;
-      const uint32_t bar_id = 1 + t * 4 + quarter;  // named barrier of the two warps of a row
-      const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-      const uint32_t tS = tmem + lane_off + t * 128 + c0;
-      const uint32_t tO = tmem + lane_off + 256 + t * 128 + c0;
-      const float sl2 = p.scale_log2;
+    // ------------------------------------------------------------------ softmax / epilogue
+    // warps 4..11 tile A, 12..19 tile B; within a tile the first four warps take key columns
+    // 0..63 and the next four 64..127 of the same rows (lane quarter = warp % 4)
+    const int t = (warp - 4) >> 3;        // query tile
+    const int half = ((warp - 4) >> 2) & 1;
+    const int c0 = half * 64;             // this warp's 64 columns of S, P and O
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t bar_id = 1 + t * 4 + quarter;  // named barrier of the two warps of a row
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128 + c0;
+    const uint32_t tO = tmem + lane_off + 256 + t * 128 + c0;
+    const float sl2 = p.scale_log2;
+    uint32_t scnt = 0;  // s_full phases consumed (key tiles processed) by this tile's warps
+    // Both warps of a row pass the same named barriers in the same order on every path, and
+    // decide together whether to go on (a wait that gave up in one of them stops both).
+    for (int k = 0;; k++) {
+      bool got = mbar_wait<1>(smem_addr(&bars.q_full), k & 1, ab);
+      __syncwarp();
+      got = __all_sync(0xffffffffu, got);
+      const int item = got ? item_slot[k & 1] : -1;
+      if (!named_bar_and(bar_id, 64, item >= 0)) break;
+      const FwdItem it = decode_item(p, item);
+      const int qt = it.qt0 + t;
+      const int n = t ? it.nB : it.nA;
       float m = -INFINITY, l = 0.f;   // running max (shared by both halves) and partial sum
       bool ok = true;
-      for (int j = 0; j < n; j++) {
-        ok = mbar_wait<1>(smem_addr(&bars.s_full[t]), j & 1, ab);
+      for (int j = 0; j < n; j++, scnt++) {
+        ok = mbar_wait<1>(smem_addr(&bars.s_full[t]), scnt & 1, ab);
         __syncwarp();
         ok = __all_sync(0xffffffffu, ok);
         tc_fence_after();
@@ -388,10 +444,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // waiting: exchange the exact max; m moves to ceil(max * sl2), an integer, so a P
         // already written with the old m is brought to the new one by an exact power of two.
         if (named_bar_or(bar_id, 64, !stored || !ok)) {
-          xmax[j & 1][t][half][row] = mraw;
+          xmax[scnt & 1][t][half][row] = mraw;
           ok = named_bar_and(bar_id, 64, ok);
           if (!ok) break;
-          const float mt = fmaxf(mraw, xmax[j & 1][t][half ^ 1][row]) * sl2;
+          const float mt = fmaxf(mraw, xmax[scnt & 1][t][half ^ 1][row]) * sl2;
           const float mnew = mt > m + kRescaleThreshold ? ceilf(mt) : m;
           alpha = exp2_int(m - mnew);  // 0 while m is -inf, 1 if m stays
           rescale = j > 0 && mnew != m;
@@ -424,40 +480,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(smem_addr(&bars.p_full[t]));
       }
       if (ok) {
-        ok = mbar_wait<1>(smem_addr(&bars.o_final[t]), 0, ab);
+        ok = mbar_wait<1>(smem_addr(&bars.o_final[t]), k & 1, ab);
         __syncwarp();
         ok = __all_sync(0xffffffffu, ok);
       }
-      // total row sum = both halves' partial sums (every path reaches this barrier)
+      // total row sum = both halves' partial sums; the second barrier also settles whether
+      // both warps go on
       if (half == 1) xsum[t][row] = l;
       named_bar_sync(bar_id, 64);
       if (half == 0) xsum[t][row] += l;
-      named_bar_sync(bar_id, 64);
+      ok = named_bar_and(bar_id, 64, ok);
       const float ltot = xsum[t][row];
-      if (ok) {
-        tc_fence_after();
-        const int mrow = src_row(r0 + t * kTile + row, sh, p.G, p.N);
-        __nv_bfloat16* orow =
-            static_cast<__nv_bfloat16*>(p.o) + ((size_t)(b * p.N + mrow) * p.Hq + h) * kD + c0;
-        const float inv_l = 1.f / ltot;
+      if (!ok) break;
+      tc_fence_after();
+      const int mrow = src_row(it.r0 + t * kTile + row, it.sh, p.G, p.N);
+      __nv_bfloat16* orow =
+          static_cast<__nv_bfloat16*>(p.o) + ((size_t)(it.b * p.N + mrow) * p.Hq + it.h) * kD + c0;
+      const float inv_l = 1.f / ltot;
 #pragma unroll
-        for (int ch = 0; ch < 2; ch++) {
-          uint32_t o[32];
-          tmem_ld32(tO + ch * 32, o);
-          tmem_wait_ld();
-          uint4 pk[4];
-          uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+      for (int ch = 0; ch < 2; ch++) {
+        uint32_t o[32];
+        tmem_ld32(tO + ch * 32, o);
+        tmem_wait_ld();
+        uint4 pk[4];
+        uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
-          for (int c2 = 0; c2 < 16; c2++)
-            pw[c2] = pack_bf16x2(__uint_as_float(o[2 * c2]) * inv_l,
-                                 __uint_as_float(o[2 * c2 + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+        for (int c2 = 0; c2 < 16; c2++)
+          pw[c2] = pack_bf16x2(__uint_as_float(o[2 * c2]) * inv_l,
+                               __uint_as_float(o[2 * c2 + 1]) * inv_l);
+        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
 #pragma unroll
-          for (int c4 = 0; c4 < 4; c4++) dst[c4] = pk[c4];
-        }
-        if (half == 0)
-          p.lse[((size_t)b * p.Hq + h) * p.N + mrow] = (m + __log2f(ltot)) * 0.69314718055994531f;
+        for (int c4 = 0; c4 < 4; c4++) dst[c4] = pk[c4];
       }
+      if (half == 0)
+        p.lse[((size_t)it.b * p.Hq + it.h) * p.N + mrow] =
+            (m + __log2f(ltot)) * 0.69314718055994531f;
     }
   }
 
@@ -490,8 +547,13 @@ cudaError_t launch_tc_fwd(const Params& p, cudaStream_t st) {
   if ((e = cudaFuncGetAttributes(&fa, tc_fwd_kernel))) return e;
   if (128 * kRegsOther + (kThreads - 128) * kRegsSoftmax > kThreads * fa.numRegs)
     return cudaErrorInvalidConfiguration;
-  const long pairs = (long)p.B * p.Hq * (p.N / p.G) * (p.G / kTile / 2);
-  tc_fwd_kernel<<<dim3((unsigned)pairs), dim3(kThreads), kSmemBytes, st>>>(p, tq, tk, tv);
+  // persistent: at most one CTA per SM (one fits), each taking items until none is left
+  const long items = (long)p.B * p.Hq * (p.N / p.G) * (p.G / kTile / 2);
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev))) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev))) return e;
+  const unsigned grid = (unsigned)(items < sms ? items : sms);
+  tc_fwd_kernel<<<dim3(grid), dim3(kThreads), kSmemBytes, st>>>(p, tq, tk, tv, (int)items);
   return cudaGetLastError();
 }
 
