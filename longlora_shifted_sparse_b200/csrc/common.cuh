@@ -33,9 +33,13 @@ struct Params {
 };
 
 enum StatusBits : unsigned { kStatusTimeout = 1u };
-// Words after the status word (same 256-byte block of the workspace): the persistent
-// forward's work-item counter, zeroed by the RoPE pass at the start of every forward.
+// Words after the status word (same 256-byte block of the workspace): the work-item
+// counters of the persistent kernels. The RoPE pass zeroes them all at the start of every
+// forward, the row-sum pass at the start of every backward.
 constexpr int kFwdWorkCounter = 1;
+constexpr int kDqWorkCounter = 2;
+constexpr int kDkdvWorkCounter = 3;
+constexpr int kNumWorkCounters = 3;
 
 // Which heads are rolled by -G/2. kShiftHalf: the second half of the heads (the method's
 // definition). kShiftAlternate: every odd kv head (the alternate-heads wording of the

@@ -44,8 +44,8 @@ __global__ void __launch_bounds__(256) rope_pi_kernel(Params p) {
   const int tok = blockIdx.x;
   const int b = tok / p.N, n = tok - b * p.N;
   if (tok == 0 && threadIdx.x == 0) {
-    p.status[0] = 0u;                // each call starts with a clean status
-    p.status[kFwdWorkCounter] = 0u;  // and the forward's work counter at item 0
+    p.status[0] = 0u;  // each call starts with a clean status and work counters at 0
+    for (int c = 1; c <= kNumWorkCounters; c++) p.status[c] = 0u;
   }
 
   const uint4* q = reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) +

@@ -92,8 +92,10 @@ __global__ void __launch_bounds__(256) bwd_rowsum_kernel(Params p) {
   const int lane = threadIdx.x & 31;
   const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   // the backward's first kernel when it reuses the forward's rotation: the call starts
-  // with a clean status word (no kernel of this launch reads it)
-  if (blockIdx.x == 0 && threadIdx.x == 0) *p.status = 0u;
+  // with a clean status word (no kernel of this launch reads it) and the work counters of
+  // the persistent kernels that follow at 0
+  if (blockIdx.x == 0 && threadIdx.x == 0)
+    for (int c = 0; c <= kNumWorkCounters; c++) p.status[c] = 0u;
   if (warp >= (long)p.B * p.N * p.Hq) return;
   const int h = (int)(warp % p.Hq);
   const long bm = warp / p.Hq;
@@ -113,7 +115,8 @@ __global__ void __launch_bounds__(256) bwd_rowsum_bf16_d128_kernel(Params p) {
   constexpr int kRowsPerWarp = 8;
   const int lane = threadIdx.x & 31, half = lane >> 4, chunk = lane & 15;
   const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *p.status = 0u;  // see bwd_rowsum_kernel
+  if (blockIdx.x == 0 && threadIdx.x == 0)  // see bwd_rowsum_kernel
+    for (int c = 0; c <= kNumWorkCounters; c++) p.status[c] = 0u;
   const long rows = (long)p.B * p.N * p.Hq;
   const long r0 = warp * kRowsPerWarp;
   if (r0 >= rows) return;

@@ -29,7 +29,8 @@
 //     dK  += dS^T Q      (TS MMA)             TMEM [384,512)
 //   The GQA sum over query heads happens in the TMEM accumulators (no atomics).
 //   Epilogue: dk = R^T (dK / sqrt(d)), dv = dV, bf16, at the key tokens' original rows.
-// dQ pass: one CTA per 128-row query tile (b, head, group, qt). For every key tile j <= qt:
+// dQ pass: persistent CTAs take 128-row query tiles (b, head, group, qt) from a work counter.
+// For every key tile j <= qt:
 //   S = Q K^T (TMEM [0,128)), dP = dO V^T into one of two buffers ([128,256), [256,384)),
 //   dS = P (dP - D) bf16 over that dP (the first 32 of each math warp's 64 columns),
 //   dQ += dS K (TS MMA, [384,512)). Three MMA issuers (warp 1: S, warp 2: dP, warp 3: dQ),
@@ -485,7 +486,7 @@ constexpr uint32_t kQOffV = (2 + kKStages) * kTileBytes;
 constexpr uint32_t kQSmem = (2 + kKStages + kVStages) * kTileBytes + 1024;
 
 struct DqBarriers {
-  uint64_t q_full;
+  uint64_t q_full, q_empty;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full, s_consumed;
@@ -493,45 +494,70 @@ struct DqBarriers {
   uint64_t acc_done, drain[3];
 };
 
-// Three MMA issuers, one thread each (a thread issues a tcgen05.mma only every ~45 cycles,
-// against 64 cycles of tensor work per 128 x 128 x 16 MMA, and slower still while math
-// warps share its scheduler; the dQ pass has 24 MMAs per key tile):
+// A dQ work item: one 128-row query tile (b, query head h, group g, tile qt).
+struct DqItem {
+  int b, h, kvh, g, qt, nkv, mq0;
+  bool sh;
+};
+
+__device__ __forceinline__ DqItem decode_dq_item(const Params& p, int item) {
+  const int T = p.G / kTile, ng = p.N / p.G, R = p.Hq / p.Hkv;
+  // the query tiles of all query heads of a few (b, kv head, group) units run together
+  // (they share K and V through L2), heaviest query tiles first
+  int inner, bkg;
+  chunked_lpt(item, p.B * p.Hkv * ng, T * R, bkg, inner);
+  DqItem it;
+  it.qt = T - 1 - inner / R;
+  it.g = bkg % ng;
+  const int bk = bkg / ng;
+  it.kvh = bk % p.Hkv;
+  it.b = bk / p.Hkv;
+  it.h = it.kvh * R + inner % R;
+  it.sh = q_head_shifted(it.h, p);
+  it.nkv = p.causal ? it.qt + 1 : T;
+  it.mq0 = src_row(it.g * p.G + it.qt * kTile, it.sh, p.G, p.N);
+  return it;
+}
+
+// q_empty completes once both Q/dO readers (the S and dP issuers) are done with an item and
+// every other role has read the item's slot; no role can then fall two items behind the
+// producer, so every parity wait on q_full sees the phase it means.
+constexpr uint32_t kDqQEmptyArrivals = 1 + 1 + 1 + kMathThreads / 32;
+
+// Persistent: one CTA per SM takes query tiles from a counter in the workspace (zeroed by
+// the row-sum pass in front of it). Three MMA issuers, one thread each (a thread issues a
+// tcgen05.mma only every ~45 cycles, against 64 cycles of tensor work per 128 x 128 x 16
+// MMA, and slower still while math warps share its scheduler; the dQ pass has 24 MMAs per
+// key tile):
 //   warp 1 (TMEM owner): S(j) = Q K_j^T into TMEM [0,128) once the math warps hold S(j-1)
 //            in registers;
 //   warp 2:  dP(j) = dO V_j^T into buffer j % 2 ([128,256) / [256,384)) once dQ(j-2) has
 //            read the dS that buffer held;
 //   warp 3:  dQ += dS(j) K_j ([384,512)) once the math warps published dS(j).
 // With dP double-buffered, S and dP of key tile j+1 are computed while the math warps work
-// on tile j, so the math never waits for the tensor cores in the steady state.
+// on tile j, so the math never waits for the tensor cores in the steady state. The rings
+// (K, V, S, dP) run on across the items of a CTA, so the next tile's S and dP are computed
+// while the math warps write the current tile's dq.
 __global__ void __launch_bounds__(kThreads, 1)
     tc_dq_kernel(const Params p, const __grid_constant__ CUtensorMap tm_q,
                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                 const __grid_constant__ CUtensorMap tm_do) {
+                 const __grid_constant__ CUtensorMap tm_do, int nitems) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   __shared__ DqBarriers bars;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_flag;
+  __shared__ int item_slot[2];  // the CTA's k-th item in slot k & 1 (-1: no more work)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int T = p.G / kTile, ng = p.N / p.G, R = p.Hq / p.Hkv;
-  // the query tiles of all query heads of a few (b, kv head, group) units run together
-  // (they share K and V through L2), heaviest query tiles first
-  int inner, bkg;
-  chunked_lpt((int)blockIdx.x, p.B * p.Hkv * ng, T * R, bkg, inner);
-  const int qt = T - 1 - inner / R;
-  const int g = bkg % ng, bk = bkg / ng;
-  const int kvh = bk % p.Hkv, b = bk / p.Hkv;
-  const int h = kvh * R + inner % R;
-  const bool sh = q_head_shifted(h, p);
-  const int nkv = p.causal ? qt + 1 : T;
-  const int mq0 = src_row(g * p.G + qt * kTile, sh, p.G, p.N);
+  unsigned* const next_item = p.status + kDqWorkCounter;
 
   Abort ab{&abort_flag, p.status};
   if (threadIdx.x == 0) {
-    abort_flag = *reinterpret_cast<volatile unsigned*>(p.status) != 0u;
+    abort_flag = 0;
     mbar_init(smem_addr(&bars.q_full), 1);
+    mbar_init(smem_addr(&bars.q_empty), kDqQEmptyArrivals);
     for (int s = 0; s < kKStages; s++) {
       mbar_init(smem_addr(&bars.k_full[s]), 1);
       mbar_init(smem_addr(&bars.k_empty[s]), 2);  // S(j) and dQ(j) both read K_j
@@ -558,51 +584,71 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = tmem_base_sh;
   const uint32_t colS = 0, colDP = 128, colDQ = 384;  // dP buffers at colDP, colDP + 128
   const uint32_t sQ = smem_addr(smem + kQOffQ), sDO = smem_addr(smem + kQOffDO);
-  const bool skip = abort_flag != 0;
+  const uint32_t qfull = smem_addr(&bars.q_full), qempty = smem_addr(&bars.q_empty);
 
-  if (skip) {
-  } else if (warp == 0) {
+  if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
-      const uint32_t qb = smem_addr(&bars.q_full);
-      mbar_arrive_expect_tx(qb, 2 * kTileBytes);
-      const int qrow = (b * p.Hq + h) * p.N + mq0;
-      tma_load_2d(sQ, &tm_q, qb, 0, qrow);
-      tma_load_2d(sQ + kBoxBytes, &tm_q, qb, 64, qrow);
-      tma_load_3d(sDO, &tm_do, qb, 0, h, b * p.N + mq0);
-      tma_load_3d(sDO + kBoxBytes, &tm_do, qb, 64, h, b * p.N + mq0);
-      int nk_issued = 0, nv_issued = 0;
-      for (int j = 0; j < nkv; j++) {
-        const int mk = src_row(g * p.G + j * kTile, sh, p.G, p.N);
-        const int krow = (b * p.Hkv + kvh) * p.N + mk;
-        const int sk = j % kKStages, sv = j % kVStages;
-        if (!mbar_wait(smem_addr(&bars.k_empty[sk]), ((j / kKStages) & 1) ^ 1, ab)) break;
-        const uint32_t kb = smem_addr(&bars.k_full[sk]);
-        const uint32_t sKs = smem_addr(smem + kQOffK + sk * kTileBytes);
-        mbar_arrive_expect_tx(kb, kTileBytes);
-        tma_load_2d(sKs, &tm_k, kb, 0, krow);
-        tma_load_2d(sKs + kBoxBytes, &tm_k, kb, 64, krow);
-        nk_issued = j + 1;
-        if (!mbar_wait(smem_addr(&bars.v_empty[sv]), ((j / kVStages) & 1) ^ 1, ab)) break;
-        const uint32_t vb = smem_addr(&bars.v_full[sv]);
-        const uint32_t sVs = smem_addr(smem + kQOffV + sv * kTileBytes);
-        mbar_arrive_expect_tx(vb, kTileBytes);
-        tma_load_3d(sVs, &tm_v, vb, 0, kvh, b * p.N + mk);
-        tma_load_3d(sVs + kBoxBytes, &tm_v, vb, 64, kvh, b * p.N + mk);
-        nv_issued = j + 1;
+      int nk = 0, nv = 0;   // K and V tiles loaded so far (ring positions)
+      int q_last = -1;      // item index (k) of the latest Q/dO load, -1 after the stop
+      for (int k = 0, ok = 1; ok; k++) {
+        int item = (int)atomicAdd(next_item, 1u);
+        // stop when the work is done or a CTA of this launch gave up
+        if (item >= nitems || *reinterpret_cast<volatile unsigned*>(p.status) != 0u) item = -1;
+        if (k > 0 && !mbar_wait(qempty, (k - 1) & 1, ab)) break;
+        item_slot[k & 1] = item;
+        if (item < 0) {
+          mbar_arrive(qfull);  // completes the phase: every role reads -1 and stops
+          q_last = -1;
+          break;
+        }
+        const DqItem it = decode_dq_item(p, item);
+        mbar_arrive_expect_tx(qfull, 2 * kTileBytes);
+        const int qrow = (it.b * p.Hq + it.h) * p.N + it.mq0;
+        tma_load_2d(sQ, &tm_q, qfull, 0, qrow);
+        tma_load_2d(sQ + kBoxBytes, &tm_q, qfull, 64, qrow);
+        tma_load_3d(sDO, &tm_do, qfull, 0, it.h, it.b * p.N + it.mq0);
+        tma_load_3d(sDO + kBoxBytes, &tm_do, qfull, 64, it.h, it.b * p.N + it.mq0);
+        q_last = k;
+        for (int j = 0; j < it.nkv; j++) {
+          const int mk = src_row(it.g * p.G + j * kTile, it.sh, p.G, p.N);
+          const int krow = (it.b * p.Hkv + it.kvh) * p.N + mk;
+          const int sk = nk % kKStages, sv = nv % kVStages;
+          if (!mbar_wait(smem_addr(&bars.k_empty[sk]), ((nk / kKStages) & 1) ^ 1, ab)) {
+            ok = 0;
+            break;
+          }
+          const uint32_t kb = smem_addr(&bars.k_full[sk]);
+          const uint32_t sKs = smem_addr(smem + kQOffK + sk * kTileBytes);
+          mbar_arrive_expect_tx(kb, kTileBytes);
+          tma_load_2d(sKs, &tm_k, kb, 0, krow);
+          tma_load_2d(sKs + kBoxBytes, &tm_k, kb, 64, krow);
+          nk++;
+          if (!mbar_wait(smem_addr(&bars.v_empty[sv]), ((nv / kVStages) & 1) ^ 1, ab)) {
+            ok = 0;
+            break;
+          }
+          const uint32_t vb = smem_addr(&bars.v_full[sv]);
+          const uint32_t sVs = smem_addr(smem + kQOffV + sv * kTileBytes);
+          mbar_arrive_expect_tx(vb, kTileBytes);
+          tma_load_3d(sVs, &tm_v, vb, 0, it.kvh, it.b * p.N + mk);
+          tma_load_3d(sVs + kBoxBytes, &tm_v, vb, 64, it.kvh, it.b * p.N + mk);
+          nv++;
+        }
       }
-      // the last loads in flight land before the CTA can exit (own time limit, no abort)
+      // the last load into each ring stage (the latest phase of its barrier) and a Q/dO load
+      // not yet consumed land before the CTA can exit (own time limit, no abort)
       int no_abort = 0;
       Abort local{&no_abort, p.status};
-      for (int j = nk_issued - 1; j >= 0 && j >= nk_issued - kKStages; j--)
-        mbar_wait(smem_addr(&bars.k_full[j % kKStages]), (j / kKStages) & 1, local);
-      for (int j = nv_issued - 1; j >= 0 && j >= nv_issued - kVStages; j--)
-        mbar_wait(smem_addr(&bars.v_full[j % kVStages]), (j / kVStages) & 1, local);
-      mbar_wait(qb, 0, local);
+      for (int t = nk - 1; t >= 0 && t >= nk - kKStages; t--)
+        mbar_wait(smem_addr(&bars.k_full[t % kKStages]), (t / kKStages) & 1, local);
+      for (int t = nv - 1; t >= 0 && t >= nv - kVStages; t--)
+        mbar_wait(smem_addr(&bars.v_full[t % kVStages]), (t / kVStages) & 1, local);
+      if (q_last >= 0) mbar_wait(qfull, q_last & 1, local);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer: S
@@ -612,20 +658,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       // address field (bytes / 16; shared memory stays below 256 KB, so nothing carries out).
       const uint64_t dQd = smem_desc_sw128(sQ, 16, 1024);
       const uint64_t dK0 = smem_desc_sw128(smem_addr(smem + kQOffK), 16, 1024);
-      bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
-      for (int j = 0; ok && j < nkv; j++) {
-        // S(j) = Q K_j^T, once the math warps hold S(j-1) in registers
-        if (j >= 1 && !mbar_wait(smem_addr(&bars.s_consumed), (j - 1) & 1, ab)) break;
-        const int sk = j % kKStages;
-        if (!mbar_wait(smem_addr(&bars.k_full[sk]), (j / kKStages) & 1, ab)) break;
+      int gs = 0;  // S tiles issued (all items)
+      bool ok = true;
+      for (int k = 0; ok; k++) {
+        if (!mbar_wait(qfull, k & 1, ab)) break;
+        const int item = item_slot[k & 1];
+        if (item < 0) break;
+        const int nkv = decode_dq_item(p, item).nkv;
         tc_fence_after();
-        const uint64_t dk = opaque64(dK0) + (uint64_t)(sk * kTileDesc);
-        const uint64_t dq = opaque64(dQd);
+        for (int j = 0; j < nkv; j++, gs++) {
+          // S = Q K_j^T, once the math warps hold the previous S in registers
+          if (gs >= 1 && !mbar_wait(smem_addr(&bars.s_consumed), (gs - 1) & 1, ab)) {
+            ok = false;
+            break;
+          }
+          const int sk = gs % kKStages;
+          if (!mbar_wait(smem_addr(&bars.k_full[sk]), (gs / kKStages) & 1, ab)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t dk = opaque64(dK0) + (uint64_t)(sk * kTileDesc);
+          const uint64_t dq = opaque64(dQd);
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; kk++)
-          mma_ss(tmem + colS, dq + kmajor_koff(kk), dk + kmajor_koff(kk), idesc_s, kk > 0);
-        mma_commit(smem_addr(&bars.s_full));
-        mma_commit(smem_addr(&bars.k_empty[sk]));
+          for (int kk = 0; kk < kD / 16; kk++)
+            mma_ss(tmem + colS, dq + kmajor_koff(kk), dk + kmajor_koff(kk), idesc_s, kk > 0);
+          mma_commit(smem_addr(&bars.s_full));
+          mma_commit(smem_addr(&bars.k_empty[sk]));
+        }
+        if (ok) mma_commit(qempty);  // Q is no longer read once these S have completed
       }
       mma_commit(smem_addr(&bars.drain[0]));
       int no_abort = 0;
@@ -638,21 +699,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
       const uint64_t dDOd = smem_desc_sw128(sDO, 16, 1024);
       const uint64_t dV0 = smem_desc_sw128(smem_addr(smem + kQOffV), 16, 1024);
-      bool ok = mbar_wait(smem_addr(&bars.q_full), 0, ab);
-      for (int j = 0; ok && j < nkv; j++) {
-        // dP(j) = dO V_j^T into buffer j % 2, once dQ(j-2) has read the dS it held
-        if (j >= 2 && !mbar_wait(smem_addr(&bars.dq_done[j & 1]), ((j - 2) >> 1) & 1, ab)) break;
-        const int sv = j % kVStages;
-        if (!mbar_wait(smem_addr(&bars.v_full[sv]), (j / kVStages) & 1, ab)) break;
+      int gd = 0;  // dP tiles issued (all items); buffer gd % 2
+      bool ok = true;
+      for (int k = 0; ok; k++) {
+        if (!mbar_wait(qfull, k & 1, ab)) break;
+        const int item = item_slot[k & 1];
+        if (item < 0) break;
+        const int nkv = decode_dq_item(p, item).nkv;
         tc_fence_after();
-        const uint64_t dv = opaque64(dV0) + (uint64_t)(sv * kTileDesc);
-        const uint64_t ddo = opaque64(dDOd);
+        for (int j = 0; j < nkv; j++, gd++) {
+          // dP = dO V_j^T into buffer gd % 2, once the dQ MMA two tiles back has read it
+          if (gd >= 2 &&
+              !mbar_wait(smem_addr(&bars.dq_done[gd & 1]), ((gd - 2) >> 1) & 1, ab)) {
+            ok = false;
+            break;
+          }
+          const int sv = gd % kVStages;
+          if (!mbar_wait(smem_addr(&bars.v_full[sv]), (gd / kVStages) & 1, ab)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t dv = opaque64(dV0) + (uint64_t)(sv * kTileDesc);
+          const uint64_t ddo = opaque64(dDOd);
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; kk++)
-          mma_ss(tmem + colDP + (j & 1) * 128, ddo + kmajor_koff(kk), dv + kmajor_koff(kk),
-                 idesc_s, kk > 0);
-        mma_commit(smem_addr(&bars.dp_full[j & 1]));
-        mma_commit(smem_addr(&bars.v_empty[sv]));
+          for (int kk = 0; kk < kD / 16; kk++)
+            mma_ss(tmem + colDP + (gd & 1) * 128, ddo + kmajor_koff(kk), dv + kmajor_koff(kk),
+                   idesc_s, kk > 0);
+          mma_commit(smem_addr(&bars.dp_full[gd & 1]));
+          mma_commit(smem_addr(&bars.v_empty[sv]));
+        }
+        if (ok) mma_commit(qempty);  // dO is no longer read once these dP have completed
       }
       mma_commit(smem_addr(&bars.drain[1]));
       int no_abort = 0;
@@ -664,22 +741,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t idesc_g = idesc_bf16_f32(kTile, kD, false, true);
       const uint64_t dKm0 = smem_desc_sw128(smem_addr(smem + kQOffK), kBoxBytes, 1024);
-      for (int j = 0; j < nkv; j++) {
-        // dQ += dS(j) K_j, dS read from dP buffer j % 2
-        if (!mbar_wait(smem_addr(&bars.ds_ready[j & 1]), (j >> 1) & 1, ab)) break;
-        const int sk = j % kKStages;
-        if (!mbar_wait(smem_addr(&bars.k_full[sk]), (j / kKStages) & 1, ab)) break;
-        tc_fence_after();
-        const uint64_t dkm = opaque64(dKm0) + (uint64_t)(sk * kTileDesc);
-        const uint32_t acc0 = j > 0;
+      int gq = 0;  // dQ steps issued (all items)
+      bool ok = true;
+      for (int k = 0; ok; k++) {
+        if (!mbar_wait(qfull, k & 1, ab)) break;
+        const int item = item_slot[k & 1];
+        if (item < 0) break;
+        mbar_arrive(qempty);  // slot read
+        const int nkv = decode_dq_item(p, item).nkv;
+        for (int j = 0; j < nkv; j++, gq++) {
+          // dQ += dS K_j, dS read from dP buffer gq % 2
+          if (!mbar_wait(smem_addr(&bars.ds_ready[gq & 1]), (gq >> 1) & 1, ab)) {
+            ok = false;
+            break;
+          }
+          const int sk = gq % kKStages;
+          if (!mbar_wait(smem_addr(&bars.k_full[sk]), (gq / kKStages) & 1, ab)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t dkm = opaque64(dKm0) + (uint64_t)(sk * kTileDesc);
+          const uint32_t acc0 = j > 0;
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; kk++)
-          mma_ts(tmem + colDQ, tmem + packed_col(colDP + (j & 1) * 128, kk, 16),
-                 dkm + mn_koff(kk), idesc_g, kk ? 1u : acc0);
-        mma_commit(smem_addr(&bars.dq_done[j & 1]));
-        mma_commit(smem_addr(&bars.k_empty[sk]));
+          for (int kk = 0; kk < kTile / 16; kk++)
+            mma_ts(tmem + colDQ, tmem + packed_col(colDP + (gq & 1) * 128, kk, 16),
+                   dkm + mn_koff(kk), idesc_g, kk ? 1u : acc0);
+          mma_commit(smem_addr(&bars.dq_done[gq & 1]));
+          mma_commit(smem_addr(&bars.k_empty[sk]));
+        }
+        if (ok) mma_commit(smem_addr(&bars.acc_done));
       }
-      mma_commit(smem_addr(&bars.acc_done));
       mma_commit(smem_addr(&bars.drain[2]));
       int no_abort = 0;
       Abort local{&no_abort, p.status};
@@ -692,75 +784,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quarter * 32 + lane;    // query row inside the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + colS + c0;
-    const int m = src_row(g * p.G + qt * kTile + row, sh, p.G, p.N);
-    const size_t lrow = ((size_t)b * p.Hq + h) * p.N + m;
-    const float nlse2 = -p.lse[lrow] * kLog2e;
-    const float Dm = p.Dsum[lrow];
     const float sl2 = p.scale_log2;
-    bool ok = true;
-    for (int j = 0; j < nkv; j++) {
-      ok = mbar_wait(smem_addr(&bars.s_full), j & 1, ab);
+    uint32_t gm = 0;  // key tiles processed (all items)
+    for (int k = 0;; k++) {
+      bool ok = mbar_wait(qfull, k & 1, ab);
       __syncwarp();
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-      const bool diag = p.causal && j == qt;
-      float pr[64];
-      {
-        uint32_t x0[32], x1[32];
-        tmem_ld32(tS, x0);
-        tmem_ld32(tS + 32, x1);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(smem_addr(&bars.s_consumed));  // S may now be overwritten
-        if (diag) {
-          mask_scores(x0, x1, row - c0, 1);  // key column after the query row: P = 0
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int item = item_slot[k & 1];
+      if (item < 0) break;
+      if (lane == 0) mbar_arrive(qempty);  // slot read
+      const DqItem it = decode_dq_item(p, item);
+      const int m = src_row(it.g * p.G + it.qt * kTile + row, it.sh, p.G, p.N);
+      const size_t lrow = ((size_t)it.b * p.Hq + it.h) * p.N + m;
+      const float nlse2 = -p.lse[lrow] * kLog2e;
+      const float Dm = p.Dsum[lrow];
+      for (int j = 0; j < it.nkv; j++, gm++) {
+        ok = mbar_wait(smem_addr(&bars.s_full), gm & 1, ab);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        const bool diag = p.causal && j == it.qt;
+        float pr[64];
+        {
+          uint32_t x0[32], x1[32];
+          tmem_ld32(tS, x0);
+          tmem_ld32(tS + 32, x1);
+          tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(smem_addr(&bars.s_consumed));  // S may now be overwritten
+          if (diag) {
+            mask_scores(x0, x1, row - c0, 1);  // key column after the query row: P = 0
 #pragma unroll
-          for (int c = 0; c < 64; c++)
-            pr[c] = fast_exp2(fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, nlse2));
-        } else {
+            for (int c = 0; c < 64; c++)
+              pr[c] = fast_exp2(fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, nlse2));
+          } else {
 #pragma unroll
-          for (int c = 0; c < 64; c++)
-            pr[c] = exp2_mixed<kDqPolyMask>(
-                fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, nlse2), c);
-        }
-        pin_regs(pr);
-      }
-      ok = mbar_wait(smem_addr(&bars.dp_full[j & 1]), (j >> 1) & 1, ab);
-      __syncwarp();
-      if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      tc_fence_after();
-      {
-        const uint32_t tDP = tmem + lane_off + colDP + (j & 1) * 128 + c0;
-        uint32_t x0[32], x1[32];
-        tmem_ld32(tDP, x0);
-        tmem_ld32(tDP + 32, x1);
-        tmem_wait_ld();
-#pragma unroll
-        for (int ch = 0; ch < 2; ch++) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int t = 0; t < 16; t++) {
-            const int c = ch * 32 + 2 * t;
-            const float dp0 = __uint_as_float(ch ? x1[2 * t] : x0[2 * t]);
-            const float dp1 = __uint_as_float(ch ? x1[2 * t + 1] : x0[2 * t + 1]);
-            pk[t] = pack_bf16x2(pr[c] * (dp0 - Dm), pr[c + 1] * (dp1 - Dm));
+            for (int c = 0; c < 64; c++)
+              pr[c] = exp2_mixed<kDqPolyMask>(
+                  fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, nlse2), c);
           }
-          tmem_st16(tDP + ch * 16, pk);  // dS of these 64 key columns, over dP already read
+          pin_regs(pr);
         }
+        ok = mbar_wait(smem_addr(&bars.dp_full[gm & 1]), (gm >> 1) & 1, ab);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        {
+          const uint32_t tDP = tmem + lane_off + colDP + (gm & 1) * 128 + c0;
+          uint32_t x0[32], x1[32];
+          tmem_ld32(tDP, x0);
+          tmem_ld32(tDP + 32, x1);
+          tmem_wait_ld();
+#pragma unroll
+          for (int ch = 0; ch < 2; ch++) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int t = 0; t < 16; t++) {
+              const int c = ch * 32 + 2 * t;
+              const float dp0 = __uint_as_float(ch ? x1[2 * t] : x0[2 * t]);
+              const float dp1 = __uint_as_float(ch ? x1[2 * t + 1] : x0[2 * t + 1]);
+              pk[t] = pack_bf16x2(pr[c] * (dp0 - Dm), pr[c + 1] * (dp1 - Dm));
+            }
+            tmem_st16(tDP + ch * 16, pk);  // dS of these 64 key columns, over dP already read
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_addr(&bars.ds_ready[gm & 1]));
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(smem_addr(&bars.ds_ready[j & 1]));
-    }
-    if (ok) {
-      ok = mbar_wait(smem_addr(&bars.acc_done), 0, ab);
+      if (!ok) break;
+      ok = mbar_wait(smem_addr(&bars.acc_done), k & 1, ab);
       __syncwarp();
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
+      if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       __nv_bfloat16* dq =
-          static_cast<__nv_bfloat16*>(p.dq) + ((size_t)(b * p.N + m) * p.Hq + h) * kD + c0;
+          static_cast<__nv_bfloat16*>(p.dq) + ((size_t)(it.b * p.N + m) * p.Hq + it.h) * kD + c0;
       const float2* cs_row = p.cs + (size_t)m * (kD / 2);
 #pragma unroll
       for (int ch = 0; ch < 2; ch++) {
@@ -771,6 +869,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         unrotate_pack(x, cs_row, (c0 + ch * 32) / 2, p.scale, o);
         store_row64(dq + ch * 32, o);
       }
+      // the next item's first dQ MMA overwrites the accumulator only after this item's
+      // dS of its first key tile, which these warps publish after the loads above
     }
   }
 
@@ -816,8 +916,13 @@ cudaError_t launch_tc_bwd_dq(const Params& p, cudaStream_t st) {
   if ((e = cudaFuncSetAttribute(tc_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kQSmem)))
     return e;
+  // persistent: at most one CTA per SM (one fits), each taking query tiles until none is left
   const long tiles = (long)p.B * p.Hq * (p.N / p.G) * (p.G / kTile);
-  tc_dq_kernel<<<dim3((unsigned)tiles), dim3(kThreads), kQSmem, st>>>(p, tq, tk, tv, tdo);
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev))) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev))) return e;
+  const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+  tc_dq_kernel<<<dim3(grid), dim3(kThreads), kQSmem, st>>>(p, tq, tk, tv, tdo, (int)tiles);
   return cudaGetLastError();
 }
 
