@@ -38,8 +38,7 @@ enum StatusBits : unsigned { kStatusTimeout = 1u };
 // forward, the row-sum pass at the start of every backward.
 constexpr int kFwdWorkCounter = 1;
 constexpr int kDqWorkCounter = 2;
-constexpr int kDkdvWorkCounter = 3;
-constexpr int kNumWorkCounters = 3;
+constexpr int kNumWorkCounters = 2;
 
 // Which heads are rolled by -G/2. kShiftHalf: the second half of the heads (the method's
 // definition). kShiftAlternate: every odd kv head (the alternate-heads wording of the
