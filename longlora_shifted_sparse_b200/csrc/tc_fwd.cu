@@ -101,25 +101,58 @@ __device__ __forceinline__ uint64_t opaque64(uint64_t v) {
   return r;
 }
 
-// Max of a thread's 64 scores, as a tree (short dependency chain).
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction per two values).
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// Three-input max (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Max of a thread's 64 scores, as a tree of three-input maxima (short dependency chain).
 __device__ __forceinline__ float max64(const uint32_t (&x0)[32], const uint32_t (&x1)[32]) {
-  float mm[16];
+  float v[64];
 #pragma unroll
-  for (int c = 0; c < 16; c++)
-    mm[c] = fmaxf(fmaxf(__uint_as_float(x0[2 * c]), __uint_as_float(x0[2 * c + 1])),
-                  fmaxf(__uint_as_float(x1[2 * c]), __uint_as_float(x1[2 * c + 1])));
+  for (int c = 0; c < 32; c++) {
+    v[c] = __uint_as_float(x0[c]);
+    v[32 + c] = __uint_as_float(x1[c]);
+  }
+  float m1[22];
 #pragma unroll
-  for (int w = 8; w >= 1; w >>= 1)
+  for (int c = 0; c < 21; c++) m1[c] = fmax3(v[3 * c], v[3 * c + 1], v[3 * c + 2]);
+  m1[21] = v[63];
+  float m2[8];
 #pragma unroll
-    for (int c = 0; c < w; c++) mm[c] = fmaxf(mm[c], mm[c + w]);
-  return mm[0];
+  for (int c = 0; c < 7; c++) m2[c] = fmax3(m1[3 * c], m1[3 * c + 1], m1[3 * c + 2]);
+  m2[7] = m1[21];
+  return fmax3(fmax3(m2[0], m2[1], m2[2]), fmax3(m2[3], m2[4], m2[5]), fmaxf(m2[6], m2[7]));
 }
 
 // P = exp2(S * sl2 - m) for a thread's 64 scores, written as bf16 pairs over the first 32
 // of its 64 TMEM columns of S (the PV MMA reads them from there); returns the sum of P.
+// The scale-and-shift and the running sums (even and odd columns) use packed fp32 pairs.
 __device__ __forceinline__ float write_p64(const uint32_t (&x0)[32], const uint32_t (&x1)[32],
                                            float sl2, float nm, uint32_t tS) {
-  float rs = 0.f;
+  const uint64_t sl2x2 = f2pack(sl2, sl2), nmx2 = f2pack(nm, nm);
+  uint64_t acc = f2pack(0.f, 0.f);
 #pragma unroll
   for (int ch = 0; ch < 2; ch++) {
     uint32_t pk[16];
@@ -127,8 +160,14 @@ __device__ __forceinline__ float write_p64(const uint32_t (&x0)[32], const uint3
     for (int c2 = 0; c2 < 16; c2++) {
       const float s0 = __uint_as_float(ch ? x1[2 * c2] : x0[2 * c2]);
       const float s1 = __uint_as_float(ch ? x1[2 * c2 + 1] : x0[2 * c2 + 1]);
-      const float a0 = fmaf(s0, sl2, nm);
-      const float a1 = fmaf(s1, sl2, nm);
+      float a0, a1;
+      f2unpack(ffma2(f2pack(s0, s1), sl2x2, nmx2), a0, a1);
+#ifdef S2_FWD_EX2_BF16X2
+      uint32_t pb;
+      asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(pb) : "r"(pack_bf16x2(a0, a1)));
+      pk[c2] = pb;
+      acc = fadd2(acc, f2pack(__uint_as_float(pb << 16), __uint_as_float(pb & 0xffff0000u)));
+#else
       float p0, p1;
       if ((kPolyMask >> c2) & 1u) {
         p0 = exp2_poly(a0);
@@ -137,12 +176,15 @@ __device__ __forceinline__ float write_p64(const uint32_t (&x0)[32], const uint3
         p0 = fast_exp2(a0);
         p1 = fast_exp2(a1);
       }
-      rs += p0 + p1;
+      acc = fadd2(acc, f2pack(p0, p1));
       pk[c2] = pack_bf16x2(p0, p1);
+#endif
     }
     tmem_st16(tS + ch * 16, pk);
   }
-  return rs;
+  float r0, r1;
+  f2unpack(acc, r0, r1);
+  return r0 + r1;
 }
 
 // Multiplies the 64 bf16 P values a thread wrote (32 packed columns) by a power of two,
