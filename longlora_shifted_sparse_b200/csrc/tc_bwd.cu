@@ -65,6 +65,19 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Columns c, c+1 of a thread's 64 loaded TMEM values, as a packed fp32 pair.
+__device__ __forceinline__ uint64_t score_pair(const uint32_t (&x0)[32], const uint32_t (&x1)[32],
+                                               int c) {
+  return c < 32 ? f2pack(__uint_as_float(x0[c]), __uint_as_float(x0[c + 1]))
+                : f2pack(__uint_as_float(x1[c - 32]), __uint_as_float(x1[c - 31]));
+}
+
+// -LSE log2(e) of query rows c, c+1 of a warp's 64 (lane l holds rows l and 32 + l).
+__device__ __forceinline__ uint64_t lse_pair(const float (&nl2)[2], int c) {
+  return f2pack(__shfl_sync(0xffffffffu, nl2[c >> 5], c & 31),
+                __shfl_sync(0xffffffffu, nl2[c >> 5], (c + 1) & 31));
+}
+
 // K-major operand (128 rows x 128 bf16 in two 64-column SW128 boxes), k-step kk.
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_saddr, int kk) {
   return smem_desc_sw128(tile_saddr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
@@ -362,6 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tST = tmem + lane_off + colST + c0;
     const uint32_t tDPT = tmem + lane_off + colDPT + c0;
     const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f2pack(sl2, sl2);
     // LSE and D of this warp's 64 query rows: lane l holds rows c0 + l and c0 + 32 + l;
     // loaded one pair ahead and broadcast with shuffles
     auto load_ld = [&](int n, float (&l2)[2], float (&dd)[2]) {
@@ -395,16 +409,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (diag) {
           mask_scores(x0, x1, row - c0, 0);  // query row c0+c before key row: P = 0
 #pragma unroll
-          for (int c = 0; c < 64; c++) {
-            const float l = __shfl_sync(0xffffffffu, nl2[c >> 5], c & 31);
-            pr[c] = fast_exp2(fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, l));
+          for (int c = 0; c < 64; c += 2) {
+            float a0, a1;
+            f2unpack(ffma2(score_pair(x0, x1, c), sl2x2, lse_pair(nl2, c)), a0, a1);
+            pr[c] = fast_exp2(a0);
+            pr[c + 1] = fast_exp2(a1);
           }
         } else {
 #pragma unroll
-          for (int c = 0; c < 64; c++) {
-            const float l = __shfl_sync(0xffffffffu, nl2[c >> 5], c & 31);
-            pr[c] = exp2_mixed<kDkdvPolyMask>(
-                fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, l), c);
+          for (int c = 0; c < 64; c += 2) {
+            float a0, a1;
+            f2unpack(ffma2(score_pair(x0, x1, c), sl2x2, lse_pair(nl2, c)), a0, a1);
+            pr[c] = exp2_mixed<kDkdvPolyMask>(a0, c);
+            pr[c + 1] = exp2_mixed<kDkdvPolyMask>(a1, c + 1);
           }
         }
         pin_regs(pr);
@@ -426,10 +443,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int c = ch * 32 + 2 * t;
             const float d0 = __shfl_sync(0xffffffffu, dsum[ch], 2 * t);
             const float d1 = __shfl_sync(0xffffffffu, dsum[ch], 2 * t + 1);
-            const float dp0 = __uint_as_float(ch ? x1[2 * t] : x0[2 * t]);
-            const float dp1 = __uint_as_float(ch ? x1[2 * t + 1] : x0[2 * t + 1]);
+            float s0, s1;
+            f2unpack(fmul2(f2pack(pr[c], pr[c + 1]), fsub2(score_pair(x0, x1, c), f2pack(d0, d1))),
+                     s0, s1);
             pp[t] = pack_bf16x2(pr[c], pr[c + 1]);
-            pd[t] = pack_bf16x2(pr[c] * (dp0 - d0), pr[c + 1] * (dp1 - d1));
+            pd[t] = pack_bf16x2(s0, s1);
           }
           tmem_st16(tDPT + ch * 32, pp);       // P^T of these 32 query rows
           tmem_st16(tDPT + ch * 32 + 16, pd);  // dS^T
@@ -785,6 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + colS + c0;
     const float sl2 = p.scale_log2;
+    const uint64_t sl2x2 = f2pack(sl2, sl2);
     uint32_t gm = 0;  // key tiles processed (all items)
     for (int k = 0;; k++) {
       bool ok = mbar_wait(qfull, k & 1, ab);
@@ -798,6 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const size_t lrow = ((size_t)it.b * p.Hq + it.h) * p.N + m;
       const float nlse2 = -p.lse[lrow] * kLog2e;
       const float Dm = p.Dsum[lrow];
+      const uint64_t nlse2x2 = f2pack(nlse2, nlse2), Dmx2 = f2pack(Dm, Dm);
       for (int j = 0; j < it.nkv; j++, gm++) {
         ok = mbar_wait(smem_addr(&bars.s_full), gm & 1, ab);
         __syncwarp();
@@ -815,13 +835,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (diag) {
             mask_scores(x0, x1, row - c0, 1);  // key column after the query row: P = 0
 #pragma unroll
-            for (int c = 0; c < 64; c++)
-              pr[c] = fast_exp2(fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, nlse2));
+            for (int c = 0; c < 64; c += 2) {
+              float a0, a1;
+              f2unpack(ffma2(score_pair(x0, x1, c), sl2x2, nlse2x2), a0, a1);
+              pr[c] = fast_exp2(a0);
+              pr[c + 1] = fast_exp2(a1);
+            }
           } else {
 #pragma unroll
-            for (int c = 0; c < 64; c++)
-              pr[c] = exp2_mixed<kDqPolyMask>(
-                  fmaf(__uint_as_float(c < 32 ? x0[c] : x1[c - 32]), sl2, nlse2), c);
+            for (int c = 0; c < 64; c += 2) {
+              float a0, a1;
+              f2unpack(ffma2(score_pair(x0, x1, c), sl2x2, nlse2x2), a0, a1);
+              pr[c] = exp2_mixed<kDqPolyMask>(a0, c);
+              pr[c + 1] = exp2_mixed<kDqPolyMask>(a1, c + 1);
+            }
           }
           pin_regs(pr);
         }
@@ -841,9 +868,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int t = 0; t < 16; t++) {
               const int c = ch * 32 + 2 * t;
-              const float dp0 = __uint_as_float(ch ? x1[2 * t] : x0[2 * t]);
-              const float dp1 = __uint_as_float(ch ? x1[2 * t + 1] : x0[2 * t + 1]);
-              pk[t] = pack_bf16x2(pr[c] * (dp0 - Dm), pr[c + 1] * (dp1 - Dm));
+              float s0, s1;
+              f2unpack(fmul2(f2pack(pr[c], pr[c + 1]), fsub2(score_pair(x0, x1, c), Dmx2)), s0,
+                       s1);
+              pk[t] = pack_bf16x2(s0, s1);
             }
             tmem_st16(tDP + ch * 16, pk);  // dS of these 64 key columns, over dP already read
           }
