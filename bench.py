@@ -84,8 +84,10 @@ def _kernel_work(name, w, es):
         work = 2.0 * fwd                # S, dP = dO V^T, dV += P^T dO, dK += dS^T Q
     elif name.startswith("bwd_dq"):
         work = 1.5 * fwd                # S, dP, dQ += dS K
-    elif name == "rope_pi":
+    elif name == "rope_pi":       # read q, k and the cos/sin table; write q~, k~
         return "hbm", 2.0 * w.B * w.N * (w.Hq + w.Hkv) * w.d * es + w.N * w.d * 4, "GB/s"
+    elif name == "rope_table":    # write the cos/sin table
+        return "hbm", w.N * w.d * 4.0, "GB/s"
     elif name == "bwd_rowsum":
         return "hbm", 2.0 * w.B * w.N * w.Hq * w.d * es + 4.0 * w.B * w.Hq * w.N, "GB/s"
     else:

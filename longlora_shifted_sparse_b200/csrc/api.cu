@@ -17,7 +17,8 @@ namespace {
 // ----------------------------------------------------------------------------- profiling
 
 enum KernelId {
-  kRopePi = 0,
+  kRopeTable = 0,
+  kRopePi,
   kFwdTc,
   kFwdSimt,
   kBwdRowsum,
@@ -29,8 +30,8 @@ enum KernelId {
 };
 
 const char* const kKernelNames[kNumKernels] = {
-    "rope_pi", "fwd_tc", "fwd_simt", "bwd_rowsum", "bwd_dkdv_tc", "bwd_dq_tc", "bwd_dq_simt",
-    "bwd_dkdv_simt"};
+    "rope_table", "rope_pi", "fwd_tc", "fwd_simt", "bwd_rowsum", "bwd_dkdv_tc", "bwd_dq_tc",
+    "bwd_dq_simt", "bwd_dkdv_simt"};
 
 struct Record {
   int id;
@@ -169,7 +170,8 @@ bool tc_path(int d, int G, int dt) { return dt == S2_BF16 && d == 128 && G % 256
 // RoPE+PI stage, then the forward kernel of the selected family.
 cudaError_t enqueue_forward(const Params& p, int dt, cudaStream_t s) {
   const bool bf16 = dt == S2_BF16;
-  cudaError_t e = timed_launch(kRopePi, s, [&] { return launch_rope_pi(p, bf16, s); });
+  cudaError_t e = timed_launch(kRopeTable, s, [&] { return launch_rope_table(p, s); });
+  if (e == cudaSuccess) e = timed_launch(kRopePi, s, [&] { return launch_rope_pi(p, bf16, s); });
   if (e != cudaSuccess) return e;
   if (tc_path(p.d, p.G, dt)) return timed_launch(kFwdTc, s, [&] { return launch_tc_fwd(p, s); });
   return timed_launch(kFwdSimt, s, [&] { return launch_simt_fwd(p, bf16, s); });
@@ -280,7 +282,10 @@ s2_status backward_impl(const void* q, const void* k, const void* v, const void*
   const bool bf16 = dtype == S2_BF16;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   cudaError_t e = cudaSuccess;
-  if (rotate) e = timed_launch(kRopePi, s, [&] { return launch_rope_pi(p, bf16, s); });
+  if (rotate) {
+    e = timed_launch(kRopeTable, s, [&] { return launch_rope_table(p, s); });
+    if (e == cudaSuccess) e = timed_launch(kRopePi, s, [&] { return launch_rope_pi(p, bf16, s); });
+  }
   if (e == cudaSuccess)
     e = timed_launch(kBwdRowsum, s, [&] { return launch_bwd_rowsum(p, bf16, s); });
   if (e != cudaSuccess) return to_status(e);

@@ -8,6 +8,7 @@
 namespace s2 {
 
 // RoPE + PI stage: q, k -> rotated head-major copies and the (cos, sin) table.
+cudaError_t launch_rope_table(const Params& p, cudaStream_t st);
 cudaError_t launch_rope_pi(const Params& p, bool bf16, cudaStream_t st);
 
 // CUDA-core kernels (any valid shape).

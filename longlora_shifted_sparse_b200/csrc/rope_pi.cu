@@ -7,10 +7,11 @@
 // roll of the shifted heads is never materialised, the attention kernels fold it into
 // their row coordinates.
 //
-// One CTA per token. The d/2 angles of a token are shared by all heads of q and k, so the
-// CTA computes them once in fp64 (sincos of an exact fp64 angle, rounded to fp32) and
-// keeps them in shared memory; the (cos, sin) table is also written to the workspace for
-// the backward's inverse rotation. The data moves in 16-byte vectors.
+// Two kernels. The first computes the (cos, sin) table once per call, [N][d/2], each entry
+// from an exact fp64 angle (sincos in fp64, rounded to fp32); the backward's inverse
+// rotation reads the same table from the workspace. The second streams q and k in 16-byte
+// vectors, one CTA per token, and reads the token's table row (shared by all its heads,
+// an L1/L2 hit) next to each vector: no CTA waits on fp64 arithmetic.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -32,26 +33,42 @@ __device__ inline uint4 rotate_vec(uint4 raw, const float2* __restrict__ cs_row)
   return out_raw;
 }
 
+// (cos, sin) of (m / s) * base^(-2i/d) for every token m and pair i. The first kernel of
+// every forward and of every backward that rotates: it also resets the status word and the
+// persistent kernels' work counters.
+__global__ void __launch_bounds__(256) rope_table_kernel(Params p) {
+  const int half = p.d / 2;
+  const long total = (long)p.N * half;
+  if (blockIdx.x == 0 && threadIdx.x == 0)
+    for (int c = 0; c <= kNumWorkCounters; c++) p.status[c] = 0u;
+  // the block size, hence the grid stride, is a multiple of d/2 (the launcher sizes it so),
+  // so a thread keeps one pair index i and computes its frequency once
+  const long stride = (long)gridDim.x * blockDim.x;
+  const long e0 = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int i = (int)(e0 % half);
+  const double theta = pow((double)p.rope_base, -2.0 * (double)i / (double)p.d);
+  for (long e = e0; e < total; e += stride) {
+    const int n = (int)(e / half);
+    const double phi = ((double)n / (double)p.pi_scale) * theta;
+    double sn, c;
+    sincos(phi, &sn, &c);
+    p.cs[e] = make_float2((float)c, (float)sn);
+  }
+}
+
 // The loads of a token's q and k vectors are issued first (kBatch per thread in flight),
-// the fp64 angles are computed while they are in flight, then the vectors are rotated and
-// stored: the kernel is bound by HBM, so it needs many loads outstanding per SM.
+// then each vector is rotated with its four (or two) table entries and stored.
 template <typename T>
 __global__ void __launch_bounds__(256) rope_pi_kernel(Params p) {
-  extern __shared__ float2 s_cs[];
   constexpr int V = 16 / sizeof(T);
   constexpr int kBatch = 4;
-  const int half = p.d / 2;
   const int tok = blockIdx.x;
   const int b = tok / p.N, n = tok - b * p.N;
-  if (tok == 0 && threadIdx.x == 0) {
-    p.status[0] = 0u;  // each call starts with a clean status and work counters at 0
-    for (int c = 1; c <= kNumWorkCounters; c++) p.status[c] = 0u;
-  }
-
   const uint4* q = reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) +
                                                   (size_t)tok * p.Hq * p.d);
   const uint4* k = reinterpret_cast<const uint4*>(static_cast<const T*>(p.k) +
                                                   (size_t)tok * p.Hkv * p.d);
+  const float2* cs_row = p.cs + (size_t)n * (p.d / 2);
   T* qr = static_cast<T*>(p.qr);
   T* kr = static_cast<T*>(p.kr);
   const int vq = p.Hq * p.d / V, vk = p.Hkv * p.d / V, nv = vq + vk;
@@ -62,17 +79,6 @@ __global__ void __launch_bounds__(256) rope_pi_kernel(Params p) {
     const int e = threadIdx.x + u * blockDim.x;
     if (e < nv) raw[u] = __ldcs(e < vq ? q + e : k + (e - vq));
   }
-  for (int i = threadIdx.x; i < half; i += blockDim.x) {
-    double theta = pow((double)p.rope_base, -2.0 * (double)i / (double)p.d);
-    double phi = ((double)n / (double)p.pi_scale) * theta;
-    double sn, c;
-    sincos(phi, &sn, &c);
-    float2 v = make_float2((float)c, (float)sn);
-    s_cs[i] = v;
-    if (b == 0) p.cs[(size_t)n * half + i] = v;
-  }
-  __syncthreads();
-
   for (int e0 = threadIdx.x;; e0 += kBatch * blockDim.x) {
 #pragma unroll
     for (int u = 0; u < kBatch; u++) {
@@ -82,8 +88,16 @@ __global__ void __launch_bounds__(256) rope_pi_kernel(Params p) {
         const int ee = is_q ? e : e - vq;
         const int h = ee * V / p.d, c0 = ee * V - h * p.d;
         const int H = is_q ? p.Hq : p.Hkv;
+        float2 cs[V / 2];
+        const float4* c4 = reinterpret_cast<const float4*>(cs_row + c0 / 2);  // 16-B aligned
+#pragma unroll
+        for (int t = 0; t < V / 4; t++) {
+          const float4 v = __ldg(c4 + t);
+          cs[2 * t] = make_float2(v.x, v.y);
+          cs[2 * t + 1] = make_float2(v.z, v.w);
+        }
         T* dst = (is_q ? qr : kr) + (((size_t)b * H + h) * p.N + n) * p.d + c0;
-        *reinterpret_cast<uint4*>(dst) = rotate_vec<T>(raw[u], s_cs + c0 / 2);
+        *reinterpret_cast<uint4*>(dst) = rotate_vec<T>(raw[u], cs);
       }
     }
     if (e0 + kBatch * (int)blockDim.x >= nv) break;
@@ -95,13 +109,23 @@ __global__ void __launch_bounds__(256) rope_pi_kernel(Params p) {
   }
 }
 
+cudaError_t launch_rope_table(const Params& p, cudaStream_t st) {
+  // a multiple of d/2 threads per block, so the grid stride is one too
+  const int half = p.d / 2;
+  const int threads = (256 / half) * half;
+  const long total = (long)p.N * half;
+  long blocks = (total + threads - 1) / threads;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  rope_table_kernel<<<dim3((unsigned)blocks), dim3(threads), 0, st>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_rope_pi(const Params& p, bool bf16, cudaStream_t st) {
   dim3 grid(p.B * p.N), block(256);
-  size_t smem = (size_t)(p.d / 2) * sizeof(float2);
   if (bf16)
-    rope_pi_kernel<__nv_bfloat16><<<grid, block, smem, st>>>(p);
+    rope_pi_kernel<__nv_bfloat16><<<grid, block, 0, st>>>(p);
   else
-    rope_pi_kernel<float><<<grid, block, smem, st>>>(p);
+    rope_pi_kernel<float><<<grid, block, 0, st>>>(p);
   return cudaGetLastError();
 }
 

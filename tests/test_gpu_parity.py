@@ -256,8 +256,9 @@ def test_device_status_and_profiler(s2):
     assert s2.device_status(ws) == s2.S2_OK
     summary = s2.profile_summary()
     s2.check(s2.s2attn_profile_enable(0))
-    assert summary["rope_pi"][0] == 2 and summary["bwd_rowsum"][0] == 1
-    assert sum(n for n, _ in summary.values()) == 6
+    assert summary["rope_table"][0] == summary["rope_pi"][0] == 2
+    assert summary["bwd_rowsum"][0] == 1
+    assert sum(n for n, _ in summary.values()) == 8
     assert all(ms > 0 for _, ms in summary.values())
 
 
