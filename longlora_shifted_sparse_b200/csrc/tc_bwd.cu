@@ -35,10 +35,11 @@
 //   dS = P (dP - D) bf16 over that dP (the first 32 of each math warp's 64 columns),
 //   dQ += dS K (TS MMA, [384,512)). Three MMA issuers (warp 1: S, warp 2: dP, warp 3: dQ),
 //   see the kernel. Epilogue: dq = R^T (dQ / sqrt(d)), bf16, at the query tokens' original rows.
-// CTAs are launched head-group-major so that the CTAs running together share the tiles
-// they stream (L2 reuse). Roles: warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
-// (dQ pass: warps 1..3 MMA issuers), warps 4..11 the per-row math. Every wait is bounded
-// (see sm100.cuh).
+// Work is numbered a few (b, kv head, group) units at a time, heaviest items first within
+// them (chunked_lpt), so the CTAs running together share the tiles they stream (L2 reuse)
+// and the last wave is light. Roles: warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
+// (dQ pass: warps 1..3 MMA issuers), warps 4..11 the per-row math, whose elementwise work
+// runs on packed fp32 pairs (f32x2). Every wait is bounded (see sm100.cuh).
 #include "common.cuh"
 #include "fastmath.cuh"
 #include "sm100.cuh"

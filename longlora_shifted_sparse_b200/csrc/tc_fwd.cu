@@ -10,8 +10,9 @@
 // above the diagonal are skipped, the diagonal tile is masked on group-local positions).
 //
 // Roles (640 threads, five warpgroups):
-//   warp 0       TMA producer: Q_A and Q_B once, then K_j, V_j into two 2-stage rings
-//                (each K/V tile serves both query tiles).
+//   warp 0       TMA producer: per work item Q_A and Q_B, then K_j, V_j into two 2-stage
+//                rings (each K/V tile serves both query tiles; the rings run on across
+//                the items of a CTA).
 //   warp 1       MMA issuer (one thread) and TMEM owner. Order per key tile j:
 //                PV_A(j-1), QK_A(j), PV_B(j-1), QK_B(j): while the tensor cores work on
 //                one tile, the other tile's softmax runs (ping-pong).
@@ -20,7 +21,8 @@
 //                lane) is shared by two warps, one per 64-column half of S: each loads its
 //                half once, takes the partial max, swaps it with its partner through shared
 //                memory (a 64-thread named barrier), and writes P = exp2(S log2(e)/sqrt(d)
-//                - m) as bf16 over the first 32 columns of its half. Four softmax warps per
+//                - m) as bf16 over the first 32 columns of its half (scale-and-shift and
+//                row sums on packed fp32 pairs, the row max with three-input max). Four softmax warps per
 //                scheduler hide the TMEM-load and MUFU latencies that bound a one-warp-per-
 //                row softmax. The O accumulator (TMEM) is rescaled only when the running max
 //                grows by more than 2^8; the stale max keeps every P <= 256 and l uses the
