@@ -138,12 +138,6 @@ __device__ __forceinline__ float write_p64(const uint32_t (&x0)[32], const uint3
       const float s1 = __uint_as_float(ch ? x1[2 * c2 + 1] : x0[2 * c2 + 1]);
       float a0, a1;
       f2unpack(ffma2(f2pack(s0, s1), sl2x2, nmx2), a0, a1);
-#ifdef S2_FWD_EX2_BF16X2
-      uint32_t pb;
-      asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(pb) : "r"(pack_bf16x2(a0, a1)));
-      pk[c2] = pb;
-      acc = fadd2(acc, f2pack(__uint_as_float(pb << 16), __uint_as_float(pb & 0xffff0000u)));
-#else
       float p0, p1;
       if ((kPolyMask >> c2) & 1u) {
         p0 = exp2_poly(a0);
@@ -154,7 +148,6 @@ __device__ __forceinline__ float write_p64(const uint32_t (&x0)[32], const uint3
       }
       acc = fadd2(acc, f2pack(p0, p1));
       pk[c2] = pack_bf16x2(p0, p1);
-#endif
     }
     tmem_st16(tS + ch * 16, pk);
   }
