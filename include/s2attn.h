@@ -90,7 +90,9 @@ typedef enum {
  * depend on G or mode). Returns 0 for arguments that s2attn_fwd would reject with
  * S2_ERR_SHAPE, S2_ERR_HEADDIM or S2_ERR_DTYPE. The workspace holds the rotated q and k
  * (head-major, original token order), the RoPE cos/sin table, the backward's row sums
- * D = rowsum(dO * O) and the device status word. */
+ * D = rowsum(dO * O), the device status word and the work counters of the persistent
+ * kernels. A workspace serves one call at a time: calls whose kernels may overlap on the
+ * GPU (e.g. on two streams) need a workspace each. */
 S2_API size_t s2attn_workspace_bytes(int B, int N, int H_q, int H_kv, int d, int dtype);
 
 /* Forward: o and lse from q, k, v. See the header comment for the operation and layouts.
