@@ -7,7 +7,6 @@ The test calls it through the C ABI twice in a row and checks each result agains
 workspace-based s2attn_fwd on the same inputs, within the parity tolerances of the other GPU
 tests. It lives in a file of its own, collected last, and needs no state from other tests.
 """
-import numpy as np
 import pytest
 import torch
 
