@@ -52,3 +52,34 @@ def test_two_gloo_ranks_independent_batches_and_max_time(tmp_path):
 def test_single_process_needs_no_group():
     assert bench.max_over_ranks(3.5) == 3.5
     assert bench.rank_seed(7, 0) == 7 and bench.rank_seed(7, 3) == 3007
+
+
+def _run_bench(args, env_extra=None):
+    import json
+    import subprocess
+    import sys
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py")] + args, cwd=root,
+                         env=env, capture_output=True, text=True, timeout=600)
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    return out.returncode, [json.loads(l) for l in lines]
+
+
+def test_reference_arm_prints_one_line_on_rank_0_only():
+    """The reference arm (the oracle on the host cores) prints the bench contract's line on
+    rank 0 and nothing on the other ranks."""
+    args = ["--impl", "reference", "--workload", "tiny_fp32", "--steps", "1", "--warmup", "3"]
+    rc, lines = _run_bench(args)
+    assert rc == 0 and len(lines) == 1
+    line = lines[0]
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["config"]["workload"] == "tiny_fp32"
+    rc, lines = _run_bench(args, {"RANK": "1", "WORLD_SIZE": "2"})
+    assert rc == 0 and lines == []
