@@ -185,6 +185,10 @@ __device__ __forceinline__ void store_row64(__nv_bfloat16* dst, const uint4 (&a)
 
 // smem: K | V | Q stages 0..2 | dO stages 0..1
 constexpr int kQStages = 3, kDOStages = 2;
+#ifndef S2_DKDV_PREFETCH_AHEAD
+#define S2_DKDV_PREFETCH_AHEAD 2
+#endif
+constexpr int kPrefetchAhead = S2_DKDV_PREFETCH_AHEAD;  // pairs between L2 prefetch and use
 constexpr uint32_t kKVOffK = 0;
 constexpr uint32_t kKVOffV = kTileBytes;
 constexpr uint32_t kKVOffQ = 2 * kTileBytes;
@@ -254,9 +258,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool skip = abort_flag != 0;
 
   // pair n -> query head, query tile
-  auto pair_q = [&](int n, int& h, int& mq0) {
-    h = kvh * R + n / nq;
-    mq0 = src_row(g * p.G + (it0 + n % nq) * kTile, sh, p.G, p.N);
+  // Pairs run query tile it0 .. T-1 of query head kvh*R, then of the next head, and so on.
+  // Each role walks them with a cursor (no division by nq: an integer division uses the
+  // MUFU reciprocal, which the math warps' exponentials keep busy).
+  struct PairCursor {
+    int h, iq;
+  };
+  auto pair_first = [&]() { return PairCursor{kvh * R, it0}; };
+  auto pair_next = [&](PairCursor& c) {
+    if (++c.iq == T) {
+      c.iq = it0;
+      ++c.h;
+    }
+  };
+  auto pair_row0 = [&](const PairCursor& c) {
+    return src_row(g * p.G + c.iq * kTile, sh, p.G, p.N);
   };
 
   if (skip) {
@@ -275,10 +291,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(sV, &tm_v, kvb, 0, kvh, b * p.N + mk0);
       tma_load_3d(sV + kBoxBytes, &tm_v, kvb, 64, kvh, b * p.N + mk0);
       int nq_issued = 0, ndo_issued = 0;
-      for (int n = 0; n < np; n++) {
-        int h, mq0;
-        pair_q(n, h, mq0);
+      PairCursor pc = pair_first(), pf = pair_first();
+      for (int t = 0; t < kPrefetchAhead; t++) pair_next(pf);
+      for (int n = 0; n < np; n++, pair_next(pc), pair_next(pf)) {
+        const int h = pc.h, mq0 = pair_row0(pc);
         const int sq = n % kQStages, sd = n % kDOStages;
+        // the Q and dO tiles of pair n + kPrefetchAhead into L2 before this thread blocks on
+        // a free ring stage: their loads into shared memory then hit in L2
+        if (n + kPrefetchAhead < np) {
+          const int mqp = pair_row0(pf);
+          const int qrowp = (b * p.Hq + pf.h) * p.N + mqp;
+          tma_prefetch_l2_2d(&tm_q, 0, qrowp);
+          tma_prefetch_l2_2d(&tm_q, 64, qrowp);
+          tma_prefetch_l2_3d(&tm_do, 0, pf.h, b * p.N + mqp);
+          tma_prefetch_l2_3d(&tm_do, 64, pf.h, b * p.N + mqp);
+        }
         if (!mbar_wait(smem_addr(&bars.q_empty[sq]), ((n / kQStages) & 1) ^ 1, ab)) break;
         const uint32_t qb = smem_addr(&bars.q_full[sq]);
         const uint32_t sQ = smem_addr(smem + kKVOffQ + sq * kTileBytes);
@@ -379,22 +406,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t sl2x2 = f2pack(sl2, sl2);
     // LSE and D of this warp's 64 query rows: lane l holds rows c0 + l and c0 + 32 + l;
     // loaded one pair ahead and broadcast with shuffles
-    auto load_ld = [&](int n, float (&l2)[2], float (&dd)[2]) {
-      int h, mq0;
-      pair_q(n, h, mq0);
-      const size_t base = ((size_t)b * p.Hq + h) * p.N + mq0 + c0 + lane;
+    auto load_ld = [&](const PairCursor& pc, float (&l2)[2], float (&dd)[2]) {
+      const size_t base = ((size_t)b * p.Hq + pc.h) * p.N + pair_row0(pc) + c0 + lane;
       l2[0] = -__ldg(p.lse + base) * kLog2e;
       l2[1] = -__ldg(p.lse + base + 32) * kLog2e;
       dd[0] = __ldg(p.Dsum + base);
       dd[1] = __ldg(p.Dsum + base + 32);
     };
     float nl2[2], dsum[2], nl2_next[2] = {0.f, 0.f}, dsum_next[2] = {0.f, 0.f};
-    if (np > 0) load_ld(0, nl2, dsum);
+    PairCursor cur = pair_first(), nxt = pair_first();
+    if (np > 0) load_ld(cur, nl2, dsum);
+    pair_next(nxt);
     bool ok = true;
     for (int n = 0; n < np; n++) {
-      if (n + 1 < np) load_ld(n + 1, nl2_next, dsum_next);
-      const int it = it0 + n % nq;
-      const bool diag = p.causal && it == kt;
+      if (n + 1 < np) load_ld(nxt, nl2_next, dsum_next);
+      const bool diag = p.causal && cur.iq == kt;
+      cur = nxt;
+      pair_next(nxt);
       ok = mbar_wait(smem_addr(&bars.st_full), n & 1, ab);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
