@@ -2,6 +2,8 @@
 inputs. Small shapes are compared element by element in full; the LLaMA2-sized workloads
 run at full size in the configuration the bench times and are compared on sampled rows
 (tile edges, the half-group boundary, the wrap group of the shifted heads)."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -328,3 +330,11 @@ def test_softmax_rescale_paths(s2):
     refs = oracle.bwd(q, k, v, do, w.G, w.pi_scale, w.rope_base, w.causal, shift=w.shift)
     for name, g, r in zip(("dq", "dk", "dv"), grads, refs):
         H.assert_close_grad(H.to_host_f64(g), r, w.dtype, name)
+
+
+@pytest.mark.skipif(os.environ.get("S2_FULL_PARITY") != "1",
+                    reason="minutes of host time: run with S2_FULL_PARITY=1")
+def test_llama2_7b_32k_every_element(s2):
+    """The bench's 32k workload compared element by element: every output of o, lse, dq,
+    dk, dv against the full fp64 oracle (about 8e12 fp64 FLOPs on the host cores)."""
+    _full_compare(s2, WORKLOADS["llama2_7b_32k"])
