@@ -64,6 +64,17 @@ def test_kernel_path_rule(lib):
         assert lib.s2attn_kernel_path(1, 1024, 4, 4, 128, 256, m, lib.S2_BF16) == -1
 
 
+def test_largest_shape_limits(lib):
+    # B * N * H_q must stay below 2^31 (row indices are 32-bit): the largest accepted shape
+    # is sized and checked, one token more is rejected before anything is enqueued
+    N = (1 << 31) // 32 // 2 - 128      # B = 2, H_q = 32: 2^31 - 8192 rows, G | N
+    assert lib.s2attn_kernel_path(2, N, 32, 32, 128, 128, 1, lib.S2_BF16) == 0
+    assert lib.s2attn_workspace_bytes(2, N, 32, 32, 128, lib.S2_BF16) > 0
+    big = 1 << 26                       # 2 * 2^26 * 32 = 2^32 rows
+    assert lib.s2attn_kernel_path(2, big, 32, 32, 128, 1 << 13, 1, lib.S2_BF16) == -1
+    assert _fwd(lib, B=2, N=big, Hq=32, Hkv=32, d=128, G=1 << 13, dt=lib.S2_BF16) == 2
+
+
 def test_mode_flags_match_header(lib):
     text = open(os.path.join(ROOT, "include", "s2attn.h")).read()
     defs = dict(re.findall(r"#define\s+(S2_(?:CAUSAL|SHIFT_\w+))\s+(0x[0-9a-fA-F]+)", text))
