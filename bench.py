@@ -108,6 +108,7 @@ class ClockSampler:
         self.proc = None
         self.lines = []
         self.thread = None
+        self.first = 0   # index of the first sample taken after mark()
 
     def start(self):
         try:
@@ -120,6 +121,15 @@ class ClockSampler:
             return
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
+        # nvidia-smi takes a moment to start: wait for its first sample (bounded), so that a
+        # short timed region still gets samples of its own
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 5.0 and self.proc.poll() is None:
+            time.sleep(0.01)
+
+    def mark(self):
+        """The timed region starts: samples from here on describe it."""
+        self.first = len(self.lines)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -128,6 +138,11 @@ class ClockSampler:
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        # a region shorter than the sampling period may end before its first sample: take the
+        # next one (at most one period later, bounded wait)
+        t0 = time.time()
+        while len(self.lines) <= self.first and time.time() - t0 < 0.5 and self.proc.poll() is None:
+            time.sleep(0.005)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -135,7 +150,7 @@ class ClockSampler:
             self.proc.kill()
         self.thread.join(timeout=5)
         sm, smax, reasons = [], [], set()
-        for ln in self.lines:
+        for ln in self.lines[self.first:]:
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) != len(self.FIELDS):
                 continue
@@ -289,10 +304,10 @@ def run_ours(args):
         gpu_uuid = "GPU-" + gpu_uuid
     sampler = ClockSampler(gpu_uuid)
     sampler.start()
-    time.sleep(0.3)
     s2.check(s2.s2attn_profile_enable(1))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
+    sampler.mark()
     e0.record(stream)
     for _ in range(args.steps):
         step()
