@@ -258,6 +258,31 @@ def test_first_row_of_each_group_is_its_value_row():
             np.testing.assert_array_equal(o[0, t, h], v[0, t, h])
 
 
+def test_lse_closed_forms():
+    """LSE is the natural log of the sum of exp(q.k / sqrt(d)) over the visible keys.
+    (1) Token 0 of an unshifted head sees only itself and RoPE at position 0 is the
+    identity: LSE = q0.k0 / sqrt(d), computed here by hand. (2) With q = 0 every score is 0:
+    local row i of a causal group sees i + 1 keys, so LSE = ln(i + 1) and O is the mean of
+    the visible v rows; without the mask LSE = ln(G) on every row."""
+    N, G, d, H = 64, 16, 8, 4
+    q, k, v, _ = _inputs(31, 1, N, H, H, d)
+    _, lse = oracle.fwd(q, k, v, G=G, s=2.0)
+    for h in range(H // 2):   # unshifted heads
+        assert lse[0, h, 0] == pytest.approx(float(q[0, 0, h] @ k[0, 0, h]) / math.sqrt(d),
+                                             abs=1e-13)
+    z = np.zeros_like(q)
+    o, lse = oracle.fwd(z, k, v, G=G, s=2.0)
+    for h in range(H):
+        for g in range(N // G):
+            rows = oracle.unit_rows(N, G, H, h, H, g)
+            for i, t in enumerate(rows):
+                assert lse[0, h, t] == pytest.approx(math.log(i + 1), abs=1e-13)
+                np.testing.assert_allclose(o[0, t, h], v[0, rows[:i + 1], h].mean(axis=0),
+                                           atol=1e-13)
+    _, lse = oracle.fwd(z, k, v, G=G, s=2.0, causal=False)
+    np.testing.assert_allclose(lse, math.log(G), atol=1e-13)
+
+
 def test_output_in_convex_hull_of_visible_values():
     N, G, d = 64, 16, 8
     q, k, v, _ = _inputs(10, 1, N, 2, 2, d)
