@@ -257,7 +257,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sK = smem_addr(smem + kKVOffK), sV = smem_addr(smem + kKVOffV);
   const bool skip = abort_flag != 0;
 
-  // pair n -> query head, query tile
   // Pairs run query tile it0 .. T-1 of query head kvh*R, then of the next head, and so on.
   // Each role walks them with a cursor (no division by nq: an integer division uses the
   // MUFU reciprocal, which the math warps' exponentials keep busy).
