@@ -101,6 +101,13 @@ VARIANTS = [
              shift="none"),
     Workload("f32_base_scaled_noncausal", 1, 256, 4, 4, 64, 64, 1.0, "f32", 1.0, True, 129,
              causal=False, rope_base=40000.0),
+    # edge cases of the persistent kernels: fewer work items than SMs, one group of two
+    # tiles per batch entry, an 8:1 query-to-kv head ratio, one group holding everything
+    Workload("bf16_b3_one_group_two_tiles", 3, 256, 2, 2, 128, 256, 1.0, "bf16", 0.5, True,
+             131),
+    Workload("bf16_gqa_8to1", 1, 512, 16, 2, 128, 256, 2.0, "bf16", 0.5, True, 132),
+    Workload("bf16_one_group_alternate_noncausal", 1, 2048, 4, 2, 128, 2048, 1.0, "bf16",
+             0.5, True, 133, causal=False, shift="alternate"),
 ]
 
 
