@@ -96,12 +96,15 @@ def _kernel_work(name, w, es):
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    """SM clock and throttle reasons while the timed region runs: `nvidia-smi` samples (100 ms
+    period) plus NVML reads of the same counters every few milliseconds, so that a timed
+    region shorter than the `nvidia-smi` period still has samples of its own."""
 
     FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
               "clocks_event_reasons.hw_thermal_slowdown",
               "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
     REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    NVML_PERIOD_S = 0.005
 
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
@@ -109,8 +112,14 @@ class ClockSampler:
         self.lines = []
         self.thread = None
         self.first = 0   # index of the first sample taken after mark()
+        self.nvml = None         # (module, device handle) when NVML answers
+        self.nvml_samples = []   # (sm MHz, max MHz, reason bits) taken after mark()
+        self.nvml_on = threading.Event()
+        self.nvml_stop = threading.Event()
+        self.nvml_thread = None
 
     def start(self):
+        self._start_nvml()
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
@@ -127,44 +136,88 @@ class ClockSampler:
         while not self.lines and time.time() - t0 < 5.0 and self.proc.poll() is None:
             time.sleep(0.01)
 
+    def _start_nvml(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByUUID(self.gpu_id)
+            pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            return
+        self.nvml = (pynvml, h)
+        self.nvml_thread = threading.Thread(target=self._poll_nvml, daemon=True)
+        self.nvml_thread.start()
+
+    def _poll_nvml(self):
+        nv, h = self.nvml
+        smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        while not self.nvml_stop.is_set():
+            if self.nvml_on.is_set():
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                    bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                except Exception:
+                    return
+                self.nvml_samples.append((float(sm), float(smax), int(bits)))
+            time.sleep(self.NVML_PERIOD_S)
+
     def mark(self):
         """The timed region starts: samples from here on describe it."""
         self.first = len(self.lines)
+        self.nvml_on.set()
 
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        # a region shorter than the sampling period may end before its first sample: take the
-        # next one (at most one period later, bounded wait)
-        t0 = time.time()
-        while len(self.lines) <= self.first and time.time() - t0 < 0.5 and self.proc.poll() is None:
-            time.sleep(0.005)
-        self.proc.terminate()
+    def _stop_nvml(self):
+        if self.nvml is None:
+            return []
+        self.nvml_stop.set()
+        self.nvml_thread.join(timeout=5)
+        nv = self.nvml[0]
+        bit = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+               "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+               "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+               "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
         try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.thread.join(timeout=5)
-        sm, smax, reasons = [], [], set()
-        for ln in self.lines[self.first:]:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) != len(self.FIELDS):
-                continue
+            nv.nvmlShutdown()
+        except Exception:
+            pass
+        return [(sm, smax, {r for r in self.REASONS if bits & bit[r]})
+                for sm, smax, bits in self.nvml_samples]
+
+    def stop(self):
+        nvml = self._stop_nvml()
+        smi = []
+        if self.proc is not None:
+            # without NVML, a region shorter than the sampling period may end before its
+            # first sample: take the next one (at most one period later, bounded wait)
+            t0 = time.time()
+            while (not nvml and len(self.lines) <= self.first and time.time() - t0 < 0.5
+                   and self.proc.poll() is None):
+                time.sleep(0.005)
+            self.proc.terminate()
             try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-            except ValueError:
-                continue
-            for name, val in zip(self.REASONS, parts[3:]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+            for ln in self.lines[self.first:]:
+                parts = [x.strip() for x in ln.split(",")]
+                if len(parts) != len(self.FIELDS):
+                    continue
+                try:
+                    sm, smax = float(parts[0]), float(parts[1])
+                except ValueError:
+                    continue
+                smi.append((sm, smax, {r for r, v in zip(self.REASONS, parts[3:])
+                                       if v.lower() == "active"}))
+        allx = smi + nvml
+        reasons = set().union(*(r for _, _, r in allx)) if allx else set()
+        return {"sm_mhz": statistics.median(x[0] for x in allx) if allx else None,
+                "sm_max_mhz": max(x[1] for x in allx) if allx else None,
+                "reasons": sorted(reasons), "samples": len(smi), "nvml_samples": len(nvml)}
 
 
 def _traffic(kernel: str):
@@ -327,8 +380,9 @@ def run_ours(args):
     # End to end: every step copies its inputs from pinned host memory to the device, runs
     # forward + backward through the C ABI, and copies all of its outputs back to pinned host
     # memory. As a training input pipeline does, the three stages run on separate streams
-    # with two device buffer sets: the copy-in of step i+1 and the copy-out of step i-1
-    # overlap step i's kernels (the copy engines and the SMs work at the same time).
+    # (two copy streams per direction) with two device buffer sets: the copy-in of step i+1
+    # and the copy-out of step i-1 overlap step i's kernels (the copy engines and the SMs
+    # work at the same time).
     e2e = None
     if not args.no_e2e:
         outs0 = [o, lse] + ([gq, gk, gv] if w.backward else [])
@@ -340,22 +394,31 @@ def run_ours(args):
         sets = [(ins0, outs0, ws),
                 ([torch.empty_like(x) for x in ins0], [torch.empty_like(x) for x in outs0],
                  torch.empty_like(ws))]
-        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-        ev = {key: [torch.cuda.Event() for _ in range(2)] for key in ("in", "comp", "out")}
+        NS = 2   # copy streams per direction: concurrent copies keep more copy engines busy
+        s_ins = [torch.cuda.Stream(dev) for _ in range(NS)]
+        s_outs = [torch.cuda.Stream(dev) for _ in range(NS)]
+        s_in, s_out = s_ins[0], s_outs[-1]
+        ev = {key: [[torch.cuda.Event() for _ in range(NS)] for _ in range(2)]
+              for key in ("in", "out")}
+        ev["comp"] = [torch.cuda.Event() for _ in range(2)]
         used = [False, False]
 
         def e2e_step(i):
             k_ = i % 2
             ins, outs, ws_ = sets[k_]
-            with torch.cuda.stream(s_in):
-                if used[k_]:
-                    s_in.wait_event(ev["comp"][k_])      # step i-2 has read these inputs
-                for d, hsrc in zip(ins, hins):
-                    d.copy_(hsrc, non_blocking=True)
-                ev["in"][k_].record(s_in)
-            stream.wait_event(ev["in"][k_])
+            for si, st in enumerate(s_ins):
+                with torch.cuda.stream(st):
+                    if used[k_]:
+                        st.wait_event(ev["comp"][k_])
+                    for j, (d, hsrc) in enumerate(zip(ins, hins)):
+                        if j % NS == si:
+                            d.copy_(hsrc, non_blocking=True)
+                    ev["in"][k_][si].record(st)
+            for si in range(NS):
+                stream.wait_event(ev["in"][k_][si])
             if used[k_]:
-                stream.wait_event(ev["out"][k_])         # step i-2's outputs are copied out
+                for si in range(NS):
+                    stream.wait_event(ev["out"][k_][si])
             s2.forward(ins[0], ins[1], ins[2], w.G, w.pi_scale, w.rope_base, w.causal, ws=ws_,
                        out=outs[0], lse=outs[1], shift=w.shift)
             if w.backward:
@@ -363,11 +426,13 @@ def run_ours(args):
                             w.rope_base, w.causal, ws=ws_, grads=tuple(outs[2:]),
                             after_forward=True, shift=w.shift)
             ev["comp"][k_].record(stream)
-            with torch.cuda.stream(s_out):
-                s_out.wait_event(ev["comp"][k_])
-                for hx, x in zip(houts, outs):
-                    hx.copy_(x, non_blocking=True)
-                ev["out"][k_].record(s_out)
+            for si, st in enumerate(s_outs):
+                with torch.cuda.stream(st):
+                    st.wait_event(ev["comp"][k_])
+                    for j, (hx, x) in enumerate(zip(houts, outs)):
+                        if j % NS == si:
+                            hx.copy_(x, non_blocking=True)
+                    ev["out"][k_][si].record(st)
             used[k_] = True
 
         for i in range(2):
@@ -375,8 +440,12 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         barrier()
         e0.record(s_in)
+        for st in s_ins[1:]:
+            st.wait_stream(s_in)
         for i in range(args.steps):
             e2e_step(i)
+        for st in s_outs[:-1]:
+            s_out.wait_stream(st)
         e1.record(s_out)   # after the last copy-out, which follows every earlier stage
         torch.cuda.synchronize(dev)
         barrier()
@@ -387,8 +456,8 @@ def run_ours(args):
         e2e = {"value": aggregate_tflops(step_flops, world, e2e_ms / args.steps), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                "ms_per_step": e2e_ms / args.steps,
-               "pipeline": "copy-in, kernels and copy-out of consecutive steps on three "
-                           "streams with two device buffer sets"}
+               "pipeline": "copy-in (two streams), kernels and copy-out (two streams) of "
+                           "consecutive steps overlapped, two device buffer sets"}
 
     peaks = _peaks()
     roofline = None
