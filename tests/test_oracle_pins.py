@@ -44,6 +44,30 @@ def test_rope_matches_complex_closed_form():
         np.testing.assert_allclose(y[:, 1::2], w.imag, rtol=0, atol=1e-9)
 
 
+@pytest.mark.parametrize("base", [80000.0, 500000.0])
+def test_rope_base_scaling_closed_form(base):
+    """RoPE base scaling (a larger base, positions not interpolated): the closed form with
+    that base; pair 0 keeps angle m for every base, every other pair turns more slowly."""
+    rng = np.random.default_rng(4)
+    d, n = 16, 24
+    x = rng.standard_normal((n, d))
+    pos = rng.integers(0, 100000, size=n)
+    y = oracle.rope(x, pos, 1.0, base)
+    z = (x[:, 0::2] + 1j * x[:, 1::2]) * np.exp(
+        1j * pos[:, None] * base ** (-np.arange(0, d, 2) / d)[None, :])
+    np.testing.assert_allclose(y[:, 0::2], z.real, rtol=0, atol=1e-9)
+    np.testing.assert_allclose(y[:, 1::2], z.imag, rtol=0, atol=1e-9)
+    e = np.zeros((d // 2, d))
+    for i in range(d // 2):
+        e[i, 2 * i] = 1.0
+    one = np.ones(d // 2, dtype=np.int64)
+    ang = lambda b: np.array([math.atan2(r[2 * i + 1], r[2 * i])
+                              for i, r in enumerate(oracle.rope(e, one, 1.0, b))])
+    a_ref, a_big = ang(10000.0), ang(base)
+    assert a_big[0] == pytest.approx(1.0, abs=1e-15) and a_ref[0] == pytest.approx(1.0, abs=1e-15)
+    assert np.all(a_big[1:] < a_ref[1:])
+
+
 def test_rope_frequency_decreases_geometrically():
     """The angle of pair i at m = 1, s = 1 is theta_i = base^(-2i/d): a geometric sequence."""
     d = 8
