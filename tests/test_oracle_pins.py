@@ -473,3 +473,63 @@ def test_flop_model_matches_pages_worked_example():
         dense = flops.attention_fwd_flops(1, L, 8, D // 8, L, causal)
         s2 = flops.attention_fwd_flops(1, L, 8, D // 8, G, causal)
         assert dense / s2 == L / G
+
+
+# ---------------------------------------------------------------- bf16 inputs (the format's definition)
+
+def _bf16_by_definition(bits: int) -> float:
+    """Value of a bfloat16 bit pattern from its fields alone: bfloat16 is the top half of an
+    IEEE 754 binary32 (1 sign bit, 8 exponent bits with bias 127, 7 fraction bits), so a
+    normal number is (-1)^s 2^(e-127) (1 + f/128) and a subnormal (-1)^s 2^(-126) (f/128).
+    No bit reinterpretation is involved here."""
+    s, e, f = bits >> 15, (bits >> 7) & 0xFF, bits & 0x7F
+    assert e != 0xFF, "infinities and NaNs are not inputs of the method"
+    mag = math.ldexp(1.0 + f / 128.0, e - 127) if e else math.ldexp(f / 128.0, -126)
+    return -mag if s else mag
+
+
+# Hand-decoded patterns: 1.0, -3.0, -0.0, the smallest subnormal 2^-133, the largest finite.
+_BF16_PATTERNS = [(0x3F80, 1.0), (0xC040, -3.0), (0x8000, -0.0), (0x0001, 2.0 ** -133),
+                  (0x7F7F, 3.3895313892515355e38)]
+
+
+def test_bf16_decode_follows_the_binary32_definition():
+    for bits, want in _BF16_PATTERNS:
+        assert _bf16_by_definition(bits) == want
+        got = float(synth.bf16_bits_to_f32(np.array([bits], dtype=np.uint16))[0])
+        assert got == want and math.copysign(1.0, got) == math.copysign(1.0, want)
+    finite = np.array([b for b in range(1 << 16) if (b >> 7) & 0xFF != 0xFF], dtype=np.uint16)
+    want = np.array([_bf16_by_definition(int(b)) for b in finite])
+    np.testing.assert_array_equal(synth.bf16_bits_to_f32(finite).astype(np.float64), want)
+
+
+def test_oracle_reads_bf16_inputs_by_the_definition():
+    """Local row 0 of a causal group sees one key, so O there is that token's v row exactly:
+    the oracle's bf16 input path must hand v through unchanged. Row 0 of unshifted head 0 is
+    token 0; with G = N = 2 row 0 of shifted head 1 is token 1 (rolled by -G/2)."""
+    B, N, H, d, G = 1, 2, 2, 8, 2
+    q, k, v, _ = synth.s2attn_inputs(17, B, N, H, H, d, 0.5, "bf16")
+    pats = [b for b, _ in _BF16_PATTERNS] + [0x4049, 0xBE00, 0x0080]  # + 3.140625, -0.125, 2^-126
+    v = v.copy()
+    v[0, 0, 0, :] = pats
+    v[0, 1, 1, :] = pats[::-1]
+    o, _ = oracle.fwd(q, k, v, G=G, s=2.0)
+    want = np.array([_bf16_by_definition(b) for b in pats])
+    np.testing.assert_array_equal(o[0, 0, 0], want)
+    np.testing.assert_array_equal(o[0, 1, 1], want[::-1])
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_oracle_bf16_path_equals_decoded_fp64_inputs(causal):
+    """The oracle reads bf16 bit patterns (every bf16 parity test) exactly as it reads the
+    same values handed over in fp64: forward and backward agree bit for bit, GQA shape."""
+    B, N, Hq, Hkv, d, G = 2, 48, 4, 2, 16, 16
+    q, k, v, do = synth.s2attn_inputs(23, B, N, Hq, Hkv, d, 0.5, "bf16")
+    dec = [synth.bf16_bits_to_f32(x).astype(np.float64) for x in (q, k, v, do)]
+    o_b, lse_b = oracle.fwd(q, k, v, G=G, s=2.0, causal=causal)
+    o_f, lse_f = oracle.fwd(*dec[:3], G=G, s=2.0, causal=causal)
+    np.testing.assert_array_equal(o_b, o_f)
+    np.testing.assert_array_equal(lse_b, lse_f)
+    for gb, gf in zip(oracle.bwd(q, k, v, do, G=G, s=2.0, causal=causal),
+                      oracle.bwd(*dec, G=G, s=2.0, causal=causal)):
+        np.testing.assert_array_equal(gb, gf)
