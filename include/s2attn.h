@@ -146,7 +146,9 @@ S2_API s2_status s2attn_bwd_after_fwd(const void* q, const void* k, const void* 
  *  - Limit: shapes whose s2attn_workspace_bytes() exceeds S2ATTN_NOALLOC_SCRATCH_BYTES are
  *    rejected with S2_ERR_WORKSPACE before anything is enqueued.
  *  - Set-up: the first call on a device looks up the array's device address (with that
- *    device current) and caches it; make that first call before any stream capture.
+ *    device current) and caches it, keyed by the device's CUDA context, so that after a
+ *    device reset (a new context) the address is looked up again; make the first call,
+ *    and the first call after a reset, before any stream capture.
  *  - Sharing: every call on a device uses the same array and leaves its contents behind
  *    (each call rewrites what it reads, and resets the status word first). Calls whose
  *    kernels overlap on the GPU (e.g. on two streams) race on the array: serialise them. */
@@ -154,6 +156,16 @@ S2_API s2_status s2attn_fwd_noalloc(const void* q, const void* k, const void* v,
                                     float* lse, int B, int N, int H_q, int H_kv, int d, int G,
                                     int mode, float pi_scale, float rope_base, int dtype,
                                     void* cuda_stream);
+
+/* Device status of s2attn_fwd_noalloc, for the same callers (no passage of the pages
+ * corresponds to it). Their status word lives in the library's fixed scratch array, which
+ * they cannot address, so s2attn_device_status() cannot reach it. This call waits for
+ * cuda_stream, then reads and clears the status word of the current device's scratch:
+ * S2_OK, or S2_ERR_DEVICE_TIMEOUT if a bounded wait of the last no-allocation forward on
+ * this device expired (its o and lse are then undefined). S2_ERR_CUDA on a CUDA error.
+ * It allocates nothing. Every no-allocation call on a device shares this word, so read it
+ * after the call whose status is wanted and before the next one starts. */
+S2_API s2_status s2attn_noalloc_device_status(void* cuda_stream);
 
 /* Which kernel family s2attn_fwd and s2attn_bwd launch for these arguments:
  * 1 = tcgen05 tensor-core kernels (bf16, d == 128, G % 256 == 0),
@@ -172,6 +184,28 @@ S2_API s2_status s2attn_device_status(void* workspace, size_t ws_bytes, void* cu
  * the CUDA context stays usable. Needs only the first 256 bytes of a workspace. */
 S2_API s2_status s2attn_selftest_wait_timeout(void* workspace, size_t ws_bytes,
                                               void* cuda_stream);
+
+/* Self-test of the tensor-core kernels' own failure path. Runs the tcgen05 forward
+ * (site S2_INJECT_FWD; the arguments of s2attn_fwd, dout/dq/dk/dv unused and may be NULL)
+ * or the whole backward (site S2_INJECT_DKDV; the arguments of s2attn_bwd, with o and lse
+ * from a forward of the same inputs) with
+ * two changes: every bounded wait gives up after 50 ms instead of 2 s, and the MMA issuer of
+ * the launch's first CTA withholds one barrier arrival (the completion of one score tile:
+ * tile B at key tile 1 of its first item in the forward, S^T of pair 1 of key tile 0 in the
+ * dK/dV pass). The waits on it expire, the CTA records S2_ERR_DEVICE_TIMEOUT in the status
+ * word, every CTA of the launch gives up, drains its TMA loads and MMAs and frees its TMEM;
+ * the CUDA context stays usable. Afterwards s2attn_device_status() reports the timeout and
+ * the outputs are undefined. Needs the tcgen05 path (s2attn_kernel_path() == 1), else
+ * S2_ERR_ARG; argument checks as in s2attn_fwd / s2attn_bwd. No trap, fault or endless
+ * wait is involved: the failure is a missing arrival and every wait is bounded. */
+#define S2_INJECT_FWD 1
+#define S2_INJECT_DKDV 2
+S2_API s2_status s2attn_selftest_inject(int site, const void* q, const void* k, const void* v,
+                                        void* o, float* lse, const void* dout, void* dq,
+                                        void* dk, void* dv, int B, int N, int H_q, int H_kv,
+                                        int d, int G, int mode, float pi_scale,
+                                        float rope_base, int dtype, void* workspace,
+                                        size_t ws_bytes, void* cuda_stream);
 
 /* Self-test of the FMA-pipe exp2 the softmax kernels use for part of their exponentials
  * (range reduction + degree-3 polynomial): y[i] = 2^x[i] for n device floats, enqueued on

@@ -6,6 +6,8 @@
 #include <mutex>
 #include <vector>
 
+#include <cudaTypedefs.h>
+
 #include "../../include/s2attn.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -220,6 +222,8 @@ Params make_params(int B, int N, int Hq, int Hkv, int d, int G, int mode, float 
   p.cs = reinterpret_cast<float2*>(c + w.cs);
   p.Dsum = reinterpret_cast<float*>(c + w.dsum);
   p.status = reinterpret_cast<unsigned*>(c + w.status);
+  p.wait_limit_ns = kWaitLimitNs;
+  p.inject = kInjectNone;
   return p;
 }
 
@@ -268,7 +272,7 @@ s2_status backward_impl(const void* q, const void* k, const void* v, const void*
                         const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
                         int N, int H_q, int H_kv, int d, int G, int mode, float pi_scale,
                         float rope_base, int dtype, void* workspace, size_t ws_bytes,
-                        void* cuda_stream, bool rotate) {
+                        void* cuda_stream, bool rotate, int inject = kInjectNone) {
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return S2_ERR_NULL;
   s2_status st = common_checks(B, N, H_q, H_kv, d, G, mode, pi_scale, rope_base, dtype,
                                workspace, ws_bytes);
@@ -279,6 +283,10 @@ s2_status backward_impl(const void* q, const void* k, const void* v, const void*
   Params p = make_params(B, N, H_q, H_kv, d, G, mode, pi_scale, rope_base, dtype, workspace);
   p.q = q; p.k = k; p.v = v; p.o = const_cast<void*>(o); p.lse = const_cast<float*>(lse);
   p.dout = dout; p.dq = dq; p.dk = dk; p.dv = dv;
+  if (inject != kInjectNone) {
+    p.inject = inject;
+    p.wait_limit_ns = kSelftestWaitLimitNs;
+  }
   const bool bf16 = dtype == S2_BF16;
   cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
   cudaError_t e = cudaSuccess;
@@ -341,8 +349,32 @@ s2_status s2attn_selftest_wait_timeout(void* workspace, size_t ws_bytes, void* c
   if (ws_bytes < kAlign) return S2_ERR_WORKSPACE;
   if (!aligned16(workspace)) return S2_ERR_ALIGN;
   return to_status(launch_wait_timeout_selftest(static_cast<unsigned*>(workspace),
-                                                50ull * 1000 * 1000,
+                                                kSelftestWaitLimitNs,
                                                 static_cast<cudaStream_t>(cuda_stream)));
+}
+
+s2_status s2attn_selftest_inject(int site, const void* q, const void* k, const void* v, void* o,
+                                 float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                                 int N, int H_q, int H_kv, int d, int G, int mode,
+                                 float pi_scale, float rope_base, int dtype, void* workspace,
+                                 size_t ws_bytes, void* cuda_stream) {
+  if (site != S2_INJECT_FWD && site != S2_INJECT_DKDV) return S2_ERR_ARG;
+  if (s2attn_kernel_path(B, N, H_q, H_kv, d, G, mode, dtype) != 1) return S2_ERR_ARG;
+  if (site == S2_INJECT_DKDV)
+    return backward_impl(q, k, v, o, lse, dout, dq, dk, dv, B, N, H_q, H_kv, d, G, mode,
+                         pi_scale, rope_base, dtype, workspace, ws_bytes, cuda_stream, true,
+                         kInjectDkdv);
+  if (!q || !k || !v || !o || !lse) return S2_ERR_NULL;
+  s2_status st = common_checks(B, N, H_q, H_kv, d, G, mode, pi_scale, rope_base, dtype,
+                               workspace, ws_bytes);
+  if (st != S2_OK) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return S2_ERR_ALIGN;
+  Params p = make_params(B, N, H_q, H_kv, d, G, mode, pi_scale, rope_base, dtype, workspace);
+  p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
+  p.inject = kInjectFwd;
+  p.wait_limit_ns = kSelftestWaitLimitNs;
+  return to_status(enqueue_forward(p, dtype, static_cast<cudaStream_t>(cuda_stream)));
 }
 
 s2_status s2attn_selftest_exp2(const float* x, float* y, int n, void* cuda_stream) {
@@ -419,24 +451,53 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[S2ATTN_NOALLOC_SCRATCH_BYTES];
 
+// The current CUDA context (cuCtxGetCurrent, reached through the runtime's driver
+// entry-point query so that the library does not link libcuda directly), or null.
+CUcontext current_context() {
+  static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 4000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+  });
+  CUcontext ctx = nullptr;
+  if (!fn || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+  return ctx;
+}
+
 // Device address of g_noalloc_scratch on the current device. In host code the array's
 // name is only a host-side stand-in, so the address is looked up with the device current,
-// once per device, and cached.
+// once per device, and cached together with the context it belongs to: after a device
+// reset the device has a new context, the library's device code is loaded again and the
+// array may sit elsewhere, so a changed context makes the lookup run again.
 cudaError_t noalloc_scratch_address(void** out) {
   static std::mutex mu;
-  static std::vector<void*> addr;
+  struct Entry {
+    CUcontext ctx;
+    void* addr;
+  };
+  static std::vector<Entry> cache;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   std::lock_guard<std::mutex> lk(mu);
-  if ((int)addr.size() <= dev) addr.resize(dev + 1, nullptr);
-  if (!addr[dev]) {
+  if ((int)cache.size() <= dev) cache.resize(dev + 1, Entry{nullptr, nullptr});
+  Entry& c = cache[dev];
+  // A thread that has not yet used the runtime has no current context (null): the lookup
+  // below then binds the device's context to it.
+  CUcontext ctx = current_context();
+  if (!c.addr || !ctx || c.ctx != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return e;
-    addr[dev] = p;
+    c.addr = p;
+    c.ctx = current_context();
   }
-  *out = addr[dev];
+  *out = c.addr;
   return cudaSuccess;
 }
 
@@ -465,4 +526,11 @@ extern "C" s2_status s2attn_fwd_noalloc(const void* q, const void* k, const void
   Params p = make_params(B, N, H_q, H_kv, d, G, mode, pi_scale, rope_base, dtype, scratch);
   p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
   return to_status(enqueue_forward(p, dtype, static_cast<cudaStream_t>(cuda_stream)));
+}
+
+extern "C" s2_status s2attn_noalloc_device_status(void* cuda_stream) {
+  void* scratch = nullptr;
+  if (noalloc_scratch_address(&scratch) != cudaSuccess) return S2_ERR_CUDA;
+  // The word sits at offset 0 of the scratch, exactly where a workspace keeps it.
+  return s2attn_device_status(scratch, S2ATTN_NOALLOC_SCRATCH_BYTES, cuda_stream);
 }

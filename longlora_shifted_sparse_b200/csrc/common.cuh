@@ -30,9 +30,23 @@ struct Params {
   float2* cs;       // (cos, sin) of (m / s) * theta_i, [N][d/2]
   float* Dsum;      // rowsum(dO * O), [B][Hq][N]
   unsigned* status; // device status word (bit 0: a bounded wait expired)
+  // failure-path testing: the time limit of every bounded wait, and which kernel (if any)
+  // withholds one barrier arrival so that a wait expires (InjectSite; 0 in normal calls)
+  unsigned long long wait_limit_ns;
+  int inject;
 };
 
+// Where a failure-path self-test withholds one arrival (the issuer of CTA 0 skips the
+// commit that would complete a score tile): kInjectFwd in the forward (score tile A, key
+// tile 1 of its first item), kInjectDkdv in the dK/dV pass (S^T of pair 1).
+enum InjectSite : int { kInjectNone = 0, kInjectFwd = 1, kInjectDkdv = 2 };
+
 enum StatusBits : unsigned { kStatusTimeout = 1u };
+// Time limit of one bounded wait in a normal call (2 s: far beyond any wait of a working
+// kernel, short enough that a stuck launch ends with an error instead of hanging).
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// The same limit in the failure-path self-tests, which make a wait expire on purpose.
+constexpr unsigned long long kSelftestWaitLimitNs = 50000000ull;
 // Words after the status word (same 256-byte block of the workspace): the work-item
 // counters of the persistent kernels. The RoPE pass zeroes them all at the start of every
 // forward, the row-sum pass at the start of every backward.

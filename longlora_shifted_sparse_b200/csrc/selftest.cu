@@ -21,8 +21,8 @@ __global__ void __launch_bounds__(32, 1) wait_timeout_kernel(unsigned* status, u
     fence_barrier_init();
   }
   __syncthreads();
-  Abort ab{&abort_flag, status};
-  mbar_wait(smem_addr(&bar), 0, ab, limit_ns);  // nothing arrives: expires by design
+  Abort ab{&abort_flag, status, limit_ns};
+  mbar_wait(smem_addr(&bar), 0, ab);  // nothing arrives: expires by design
 }
 
 __global__ void exp2_poly_kernel(const float* x, float* y, int n) {

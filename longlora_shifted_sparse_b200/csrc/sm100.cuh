@@ -67,27 +67,26 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
   return ok != 0;
 }
 
-// Shared abort state of one CTA: a flag in shared memory plus the call's global status word.
-struct Abort {
-  volatile int* flag;   // shared memory
-  unsigned* status;     // global memory (workspace)
-};
-
-// Time limit of one wait. Every wait in the tcgen05 kernels is bounded by it; on expiry the
-// waiter records the timeout in the status word, raises the CTA's abort flag and returns
-// false. Every other wait of the CTA, and of every other CTA of the launch (they poll the
-// status word), then gives up at its next check.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
 // Longest sleep of one try-wait in the slow path; the abort flag, the status word and the
 // clock are checked every 16 try-waits.
 constexpr uint32_t kWaitSleepNs = 20000u;
+
+// Shared abort state of one CTA: a flag in shared memory, the call's global status word and
+// the time limit of one wait. Every wait in the tcgen05 kernels is bounded by that limit; on
+// expiry the waiter records the timeout in the status word, raises the CTA's abort flag and
+// returns false. Every other wait of the CTA, and of every other CTA of the launch (they
+// poll the status word), then gives up at its next check.
+struct Abort {
+  volatile int* flag;   // shared memory
+  unsigned* status;     // global memory (workspace)
+  uint64_t limit_ns;
+};
 
 // kRegion gives each register budget of a kernel that splits its registers (setmaxnreg) its
 // own copy of the out-of-line slow path: a function called from two budgets cannot be
 // allocated for both.
 template <int kRegion = 0>
-static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, Abort ab,
-                                                   uint64_t limit_ns) {
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, Abort ab) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 0;; ++i) {
     if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
@@ -97,7 +96,7 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity
         *ab.flag = 1;
         return false;
       }
-      if (global_timer_ns() - t0 > limit_ns) {
+      if (global_timer_ns() - t0 > ab.limit_ns) {
         atomicOr(ab.status, 1u);
         *ab.flag = 1;
         __threadfence_block();
@@ -108,10 +107,29 @@ static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity
 }
 
 template <int kRegion = 0>
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, Abort ab,
-                                          uint64_t limit_ns = kWaitLimitNs) {
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, Abort ab) {
   if (mbar_try_wait(bar, parity)) return true;
-  return mbar_wait_slow<kRegion>(bar, parity, ab, limit_ns);
+  return mbar_wait_slow<kRegion>(bar, parity, ab);
+}
+
+// Wait that drains asynchronous work a CTA started (TMA loads into its shared memory, MMAs
+// reading or writing its TMEM) before the CTA exits or frees TMEM. It is used on every exit
+// path, also after an abort, so it ignores the abort flag and the status word and is bounded
+// by the time limit alone; on expiry it records a timeout like any other wait. Only phases
+// whose arrivals were issued already (a load in flight, a commit of this thread) are
+// drained this way, so in a working kernel it always returns true.
+template <int kRegion = 0>
+static __device__ __noinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity,
+                                                    unsigned* status, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 0;; ++i) {
+    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+    if ((i & 15u) == 15u && global_timer_ns() - t0 > limit_ns) {
+      atomicOr(status, 1u);
+      return false;
+    }
+  }
 }
 
 // ------------------------------------------------------------------------------ TMA

@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int np = R * nq;       // (query head, query tile) pairs
   const int mk0 = src_row(g * p.G + kt * kTile, sh, p.G, p.N);
 
-  Abort ab{&abort_flag, p.status};
+  Abort ab{&abort_flag, p.status, p.wait_limit_ns};
   if (threadIdx.x == 0) {
     abort_flag = *reinterpret_cast<volatile unsigned*>(p.status) != 0u;
     mbar_init(smem_addr(&bars.kv_full), 1);
@@ -321,13 +321,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(sDO + kBoxBytes, &tm_do, db, 64, h, b * p.N + mq0);
         ndo_issued = n + 1;
       }
-      int no_abort = 0;
-      Abort local{&no_abort, p.status};
       for (int n = nq_issued - 1; n >= 0 && n >= nq_issued - kQStages; n--)
-        mbar_wait(smem_addr(&bars.q_full[n % kQStages]), (n / kQStages) & 1, local);
+        mbar_wait_drain(smem_addr(&bars.q_full[n % kQStages]), (n / kQStages) & 1, p.status,
+                        p.wait_limit_ns);
       for (int n = ndo_issued - 1; n >= 0 && n >= ndo_issued - kDOStages; n--)
-        mbar_wait(smem_addr(&bars.do_full[n % kDOStages]), (n / kDOStages) & 1, local);
-      mbar_wait(kvb, 0, local);
+        mbar_wait_drain(smem_addr(&bars.do_full[n % kDOStages]), (n / kDOStages) & 1, p.status,
+                        p.wait_limit_ns);
+      mbar_wait_drain(kvb, 0, p.status, p.wait_limit_ns);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
@@ -342,7 +342,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kD / 16; kk++)
           mma_ss(tmem + colST, kmajor_desc(sK, kk), kmajor_desc(sQ, kk), idesc_s, kk > 0);
-        mma_commit(smem_addr(&bars.st_full));
+        // failure-path self-test: CTA 0 (key tile 0, at least two pairs) withholds the
+        // arrival of S^T(1), so that the math warps and then this thread wait in vain
+        if (!(p.inject == kInjectDkdv && blockIdx.x == 0 && n == 1))
+          mma_commit(smem_addr(&bars.st_full));
         return true;
       };
       auto issue_dpt = [&](int n) -> bool {  // dP^T(n) = V dO_n^T
@@ -389,9 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mma_commit(smem_addr(&bars.acc_done));
       mma_commit(smem_addr(&bars.drain));
-      int no_abort = 0;
-      Abort local{&no_abort, p.status};
-      mbar_wait(smem_addr(&bars.drain), 0, local);
+      mbar_wait_drain(smem_addr(&bars.drain), 0, p.status, p.wait_limit_ns);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ per key row math
@@ -599,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned* const next_item = p.status + kDqWorkCounter;
 
-  Abort ab{&abort_flag, p.status};
+  Abort ab{&abort_flag, p.status, p.wait_limit_ns};
   if (threadIdx.x == 0) {
     abort_flag = 0;
     mbar_init(smem_addr(&bars.q_full), 1);
@@ -688,13 +689,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // the last load into each ring stage (the latest phase of its barrier) and a Q/dO load
       // not yet consumed land before the CTA can exit (own time limit, no abort)
-      int no_abort = 0;
-      Abort local{&no_abort, p.status};
       for (int t = nk - 1; t >= 0 && t >= nk - kKStages; t--)
-        mbar_wait(smem_addr(&bars.k_full[t % kKStages]), (t / kKStages) & 1, local);
+        mbar_wait_drain(smem_addr(&bars.k_full[t % kKStages]), (t / kKStages) & 1, p.status,
+                        p.wait_limit_ns);
       for (int t = nv - 1; t >= 0 && t >= nv - kVStages; t--)
-        mbar_wait(smem_addr(&bars.v_full[t % kVStages]), (t / kVStages) & 1, local);
-      if (q_last >= 0) mbar_wait(qfull, q_last & 1, local);
+        mbar_wait_drain(smem_addr(&bars.v_full[t % kVStages]), (t / kVStages) & 1, p.status,
+                        p.wait_limit_ns);
+      if (q_last >= 0) mbar_wait_drain(qfull, q_last & 1, p.status, p.wait_limit_ns);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer: S
@@ -735,9 +736,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) mma_commit(qempty);  // Q is no longer read once these S have completed
       }
       mma_commit(smem_addr(&bars.drain[0]));
-      int no_abort = 0;
-      Abort local{&no_abort, p.status};
-      mbar_wait(smem_addr(&bars.drain[0]), 0, local);
+      mbar_wait_drain(smem_addr(&bars.drain[0]), 0, p.status, p.wait_limit_ns);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------------ MMA issuer: dP
@@ -778,9 +777,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) mma_commit(qempty);  // dO is no longer read once these dP have completed
       }
       mma_commit(smem_addr(&bars.drain[1]));
-      int no_abort = 0;
-      Abort local{&no_abort, p.status};
-      mbar_wait(smem_addr(&bars.drain[1]), 0, local);
+      mbar_wait_drain(smem_addr(&bars.drain[1]), 0, p.status, p.wait_limit_ns);
     }
   } else if (warp == 3) {
     // ------------------------------------------------------------------ MMA issuer: dQ
@@ -819,9 +816,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) mma_commit(smem_addr(&bars.acc_done));
       }
       mma_commit(smem_addr(&bars.drain[2]));
-      int no_abort = 0;
-      Abort local{&no_abort, p.status};
-      mbar_wait(smem_addr(&bars.drain[2]), 0, local);
+      mbar_wait_drain(smem_addr(&bars.drain[2]), 0, p.status, p.wait_limit_ns);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ per query row math

@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned* const next_item = p.status + kFwdWorkCounter;
 
-  Abort ab{&abort_flag, p.status};
+  Abort ab{&abort_flag, p.status, p.wait_limit_ns};
   if (threadIdx.x == 0) {
     abort_flag = 0;
     mbar_init(smem_addr(&bars.q_full), 1);
@@ -317,13 +317,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Let the loads in flight land before the CTA can exit: the last load into each ring
       // stage (the latest phase of its barrier) and a query load not yet consumed. These
       // waits ignore the abort flag (it may be set on this path) but keep their time limit.
-      int no_abort = 0;
-      Abort local{&no_abort, p.status};
       for (int t = nk - 1; t >= 0 && t >= nk - 2; t--)
-        mbar_wait(smem_addr(&bars.k_full[t & 1]), (t >> 1) & 1, local);
+        mbar_wait_drain(smem_addr(&bars.k_full[t & 1]), (t >> 1) & 1, p.status,
+                        p.wait_limit_ns);
       for (int t = nv - 1; t >= 0 && t >= nv - 2; t--)
-        mbar_wait(smem_addr(&bars.v_full[t & 1]), (t >> 1) & 1, local);
-      if (q_last >= 0) mbar_wait(smem_addr(&bars.q_full), q_last & 1, local);
+        mbar_wait_drain(smem_addr(&bars.v_full[t & 1]), (t >> 1) & 1, p.status,
+                        p.wait_limit_ns);
+      if (q_last >= 0)
+        mbar_wait_drain(smem_addr(&bars.q_full), q_last & 1, p.status, p.wait_limit_ns);
     } else if (warp == 1 && lane == 0) {
       // ------------------------------------------------------------------ MMA issuer
       const uint32_t idesc_qk = idesc_bf16_f32(kTile, kTile, false, false);
@@ -383,7 +384,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint64_t koff = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
                 mma_ss(tS, dQt + koff, dKj + koff, idesc_qk, kk > 0);
               }
-              mma_commit(smem_addr(&bars.s_full[t]));
+              // failure-path self-test: CTA 0 withholds the arrival of score tile B at key
+              // tile 1 of its first item (every item's tile B has at least two key tiles), so
+              // that tile's softmax warps and then this thread wait in vain until the limit
+              if (!(p.inject == kInjectFwd && blockIdx.x == 0 && k == 0 && t == 1 && j == 1))
+                mma_commit(smem_addr(&bars.s_full[t]));
             }
           }
           if (!ok) break;
@@ -395,9 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // every MMA issued above has completed before TMEM is released
       mma_commit(smem_addr(&bars.drain));
-      int no_abort = 0;
-      Abort local{&no_abort, p.status};
-      mbar_wait(smem_addr(&bars.drain), 0, local);
+      mbar_wait_drain(smem_addr(&bars.drain), 0, p.status, p.wait_limit_ns);
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));

@@ -22,6 +22,7 @@ S2_OK, S2_ERR_NULL, S2_ERR_SHAPE, S2_ERR_DTYPE, S2_ERR_HEADDIM, S2_ERR_ALIGN, \
     S2_ERR_WORKSPACE, S2_ERR_CUDA, S2_ERR_DEVICE_TIMEOUT, S2_ERR_ARG = range(10)
 S2_BF16, S2_FP32 = 0, 1
 S2_CAUSAL, S2_SHIFT_HALF, S2_SHIFT_ALTERNATE, S2_SHIFT_NONE = 0x01, 0x00, 0x10, 0x20
+S2_INJECT_FWD, S2_INJECT_DKDV = 1, 2
 SHIFT_PATTERNS = {"half": S2_SHIFT_HALF, "alternate": S2_SHIFT_ALTERNATE, "none": S2_SHIFT_NONE}
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # S2ATTN_NOALLOC_SCRATCH_BYTES
 
@@ -45,10 +46,14 @@ _lib.s2attn_bwd_after_fwd.argtypes = [_vp] * 9 + _SHAPE + [_vp, _sz, _vp]
 _lib.s2attn_bwd_after_fwd.restype = _i
 _lib.s2attn_fwd_noalloc.argtypes = [_vp] * 5 + _SHAPE + [_vp]
 _lib.s2attn_fwd_noalloc.restype = _i
+_lib.s2attn_noalloc_device_status.argtypes = [_vp]
+_lib.s2attn_noalloc_device_status.restype = _i
 _lib.s2attn_kernel_path.argtypes = [_i] * 8
 _lib.s2attn_kernel_path.restype = _i
 _lib.s2attn_selftest_wait_timeout.argtypes = [_vp, _sz, _vp]
 _lib.s2attn_selftest_wait_timeout.restype = _i
+_lib.s2attn_selftest_inject.argtypes = [_i] + [_vp] * 9 + _SHAPE + [_vp, _sz, _vp]
+_lib.s2attn_selftest_inject.restype = _i
 _lib.s2attn_selftest_exp2.argtypes = [_vp, _vp, _i, _vp]
 _lib.s2attn_selftest_exp2.restype = _i
 _lib.s2attn_device_status.argtypes = [_vp, _sz, _vp]
@@ -71,9 +76,11 @@ s2attn_fwd = _lib.s2attn_fwd
 s2attn_bwd = _lib.s2attn_bwd
 s2attn_bwd_after_fwd = _lib.s2attn_bwd_after_fwd
 s2attn_fwd_noalloc = _lib.s2attn_fwd_noalloc
+s2attn_noalloc_device_status = _lib.s2attn_noalloc_device_status
 s2attn_kernel_path = _lib.s2attn_kernel_path
 s2attn_device_status = _lib.s2attn_device_status
 s2attn_selftest_wait_timeout = _lib.s2attn_selftest_wait_timeout
+s2attn_selftest_inject = _lib.s2attn_selftest_inject
 s2attn_selftest_exp2 = _lib.s2attn_selftest_exp2
 s2attn_profile_enable = _lib.s2attn_profile_enable
 s2attn_profile_num_kernels = _lib.s2attn_profile_num_kernels
@@ -148,9 +155,12 @@ def workspace(B, N, Hq, Hkv, d, dtype_code, device):
 
 
 def forward(q, k, v, G: int, pi_scale: float, rope_base: float = 10000.0, causal: bool = True,
-            ws=None, out=None, lse=None, shift: str = "half"):
+            ws=None, out=None, lse=None, shift: str = "half", check_status: bool = False):
     """q [B,N,Hq,d], k/v [B,N,Hkv,d] CUDA tensors -> (o, lse). shift picks the shifted
-    heads: "half" (the method), "alternate" (odd kv heads) or "none"."""
+    heads: "half" (the method), "alternate" (odd kv heads) or "none".
+
+    check_status=True waits for the stream after the launch and raises S2Error if a bounded
+    wait in a kernel expired (the outputs are then undefined)."""
     import torch
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
@@ -162,16 +172,20 @@ def forward(q, k, v, G: int, pi_scale: float, rope_base: float = 10000.0, causal
     check(s2attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
                      B, N, Hq, Hkv, d, G, mode(causal, shift), pi_scale, rope_base, dt,
                      ws.data_ptr(), ws.numel(), _stream_ptr(q.device)))
+    if check_status:
+        check(device_status(ws))
     return o, lse
 
 
 def backward(q, k, v, o, lse, dout, G: int, pi_scale: float, rope_base: float = 10000.0,
              causal: bool = True, ws=None, grads=None, after_forward: bool = False,
-             shift: str = "half"):
+             shift: str = "half", check_status: bool = False):
     """Returns (dq, dk, dv) for the forward that produced (o, lse).
 
     after_forward=True calls s2attn_bwd_after_fwd: `ws` must then be the workspace the
-    forward of these q, k used, unchanged since (it holds their rotation)."""
+    forward of these q, k used, unchanged since (it holds their rotation).
+    check_status=True waits for the stream after the launch and raises S2Error if a bounded
+    wait in a kernel expired (the gradients are then undefined)."""
     import torch
     B, N, Hq, d = q.shape
     Hkv = k.shape[2]
@@ -188,12 +202,22 @@ def backward(q, k, v, o, lse, dout, G: int, pi_scale: float, rope_base: float = 
                      dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                      B, N, Hq, Hkv, d, G, mode(causal, shift), pi_scale, rope_base, dt,
                      ws.data_ptr(), ws.numel(), _stream_ptr(q.device)))
+    if check_status:
+        check(device_status(ws))
     return dq, dk, dv
 
 
 def device_status(ws) -> int:
-    import torch
+    """Waits for the current stream, then reads and clears the status word of `ws`."""
     return s2attn_device_status(ws.data_ptr(), ws.numel(), _stream_ptr(ws.device))
+
+
+def noalloc_device_status(device=None) -> int:
+    """Status of the last s2attn_fwd_noalloc on `device` (waits for its current stream)."""
+    import torch
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    with torch.cuda.device(dev):
+        return s2attn_noalloc_device_status(_stream_ptr(dev))
 
 
 def _make_function():
@@ -218,8 +242,13 @@ def _make_function():
         def backward(ctx, do):
             q, k, v, o, lse, ws = ctx.saved_tensors
             G, pi_scale, rope_base, causal, shift = ctx.args
+            # The backward's first kernel resets the workspace's status word, so a bounded
+            # wait that expired in the forward is read here, before it would be lost, and the
+            # backward's own status right after it (the workspace is dropped afterwards):
+            # two stream synchronisations per backward.
+            check(device_status(ws))
             dq, dk, dv = backward(q, k, v, o, lse, do.contiguous(), G, pi_scale, rope_base, causal,
-                                  ws=ws, after_forward=True, shift=shift)
+                                  ws=ws, after_forward=True, shift=shift, check_status=True)
             return dq, dk, dv, None, None, None, None, None
 
     return S2AttnFunction

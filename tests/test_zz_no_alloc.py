@@ -4,12 +4,16 @@ cannot afford cudaMalloc's implicit synchronisation, a C caller with no allocato
 scratch is a fixed array inside the library instead of a caller-provided workspace.
 
 The test calls it through the C ABI twice in a row and checks each result against the
-workspace-based s2attn_fwd on the same inputs, within the parity tolerances of the other GPU
-tests. It lives in a file of its own, collected last, and needs no state from other tests.
+workspace-based s2attn_fwd on the same inputs and against the fp64 oracle, within the parity
+tolerances of the other GPU tests, and reads the call's device status through
+s2attn_noalloc_device_status (the no-allocation caller cannot address the status word in
+the library's scratch). It lives in a file of its own, collected last, and needs no state
+from other tests.
 """
 import pytest
 import torch
 
+import oracle
 import synth
 from tests import gpu_helpers as H
 
@@ -41,6 +45,7 @@ def test_noalloc_forward_matches_workspace_forward(s2, case):
     assert s2.s2attn_workspace_bytes(B, N, Hq, Hkv, d, code) <= s2.NOALLOC_SCRATCH_BYTES
     o_ref, lse_ref = s2.forward(tq, tk, tv, G, s, causal=causal)
     torch.cuda.synchronize()
+    o_or, lse_or = oracle.fwd(q, k, v, G, s, causal=causal)
     stream = torch.cuda.current_stream().cuda_stream
     for _ in range(2):
         o = torch.full_like(o_ref, float("nan"))
@@ -49,9 +54,13 @@ def test_noalloc_forward_matches_workspace_forward(s2, case):
                                    lse.data_ptr(), B, N, Hq, Hkv, d, G, int(causal), s, 10000.0,
                                    code, stream)
         assert rc == s2.S2_OK, s2.s2attn_status_string(rc)
+        assert s2.s2attn_noalloc_device_status(stream) == s2.S2_OK
         torch.cuda.synchronize()
-        H.assert_close_o(H.to_host_f64(o), H.to_host_f64(o_ref), dt)
-        H.assert_close_lse(H.to_host_f64(lse), H.to_host_f64(lse_ref), dt)
+        o_h, lse_h = H.to_host_f64(o), H.to_host_f64(lse)
+        H.assert_close_o(o_h, H.to_host_f64(o_ref), dt)
+        H.assert_close_lse(lse_h, H.to_host_f64(lse_ref), dt)
+        H.assert_close_o(o_h, o_or, dt, "o vs oracle")
+        H.assert_close_lse(lse_h, lse_or, dt, "lse vs oracle")
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(s2):
@@ -63,3 +72,11 @@ def test_noalloc_rejects_shapes_beyond_its_scratch(s2):
                                torch.cuda.current_stream().cuda_stream)
     assert rc == s2.S2_ERR_WORKSPACE
     assert bool((small == 0).all())
+
+
+def test_noalloc_status_query_reads_and_clears(s2):
+    """The status query needs no workspace and allocates nothing; after a clean call it
+    reports S2_OK, and reading it twice gives S2_OK both times (reading clears the word)."""
+    stream = torch.cuda.current_stream().cuda_stream
+    assert s2.s2attn_noalloc_device_status(stream) == s2.S2_OK
+    assert s2.noalloc_device_status() == s2.S2_OK
