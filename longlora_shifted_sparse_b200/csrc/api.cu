@@ -128,7 +128,7 @@ constexpr size_t kAlign = 256;
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct WsLayout {
-  size_t qr, kr, cs, dsum, status, total;
+  size_t qr, kr, cs, dsum, rowterms, status, total;
 };
 
 bool shape_ok(int B, int N, int Hq, int Hkv, int G) {
@@ -159,6 +159,8 @@ WsLayout ws_layout(int B, int N, int Hq, int Hkv, int d, int dt) {
   off = align_up(off + (size_t)N * (d / 2) * sizeof(float2));
   w.dsum = off;
   off = align_up(off + (size_t)B * Hq * N * sizeof(float));
+  w.rowterms = off;
+  off = align_up(off + (size_t)B * Hq * N * 16 * 2);
   w.total = off;
   return w;
 }
@@ -221,6 +223,7 @@ Params make_params(int B, int N, int Hq, int Hkv, int d, int G, int mode, float 
   p.kr = c + w.kr;
   p.cs = reinterpret_cast<float2*>(c + w.cs);
   p.Dsum = reinterpret_cast<float*>(c + w.dsum);
+  p.rowterms = c + w.rowterms;
   p.status = reinterpret_cast<unsigned*>(c + w.status);
   p.wait_limit_ns = kWaitLimitNs;
   p.inject = kInjectNone;

@@ -29,6 +29,10 @@ struct Params {
   void* kr;         // rotated k, [B][Hkv][N][d], original token order
   float2* cs;       // (cos, sin) of (m / s) * theta_i, [N][d/2]
   float* Dsum;      // rowsum(dO * O), [B][Hq][N]
+  // per query row, the backward's row terms as a 16-element bf16 row [B][Hq][N][16]:
+  // -LSE*sqrt(d) split into three bf16 parts (elements 0..2), -D into two (3, 4), zeros.
+  // The tensor-core dK/dV pass adds them to S^T and dP^T as one more MMA k-step.
+  void* rowterms;
   unsigned* status; // device status word (bit 0: a bounded wait expired)
   // failure-path testing: the time limit of every bounded wait, and which kernel (if any)
   // withholds one barrier arrival so that a wait expires (InjectSite; 0 in normal calls)

@@ -148,7 +148,24 @@ __global__ void __launch_bounds__(256) bwd_rowsum_bf16_d128_kernel(Params p) {
       const int h = (int)(r % p.Hq);
       const long bm = r / p.Hq;
       const int m = (int)(bm % p.N), b = (int)(bm / p.N);
-      p.Dsum[((size_t)b * p.Hq + h) * p.N + m] = acc;
+      const size_t row = ((size_t)b * p.Hq + h) * p.N + m;
+      p.Dsum[row] = acc;
+      // the row terms of the tensor-core dK/dV pass: -LSE*sqrt(d) and -D as sums of bf16
+      // parts (each part the rounding of what the previous ones left), exact to ~2^-24 and
+      // ~2^-16 relative
+      const float nl = -p.lse[row] / p.scale;
+      const __nv_bfloat16 l0 = __float2bfloat16_rn(nl);
+      const float r1 = nl - __bfloat162float(l0);
+      const __nv_bfloat16 l1 = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 l2 = __float2bfloat16_rn(r1 - __bfloat162float(l1));
+      const __nv_bfloat16 d0 = __float2bfloat16_rn(-acc);
+      const __nv_bfloat16 d1 = __float2bfloat16_rn(-acc - __bfloat162float(d0));
+      const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
+      __nv_bfloat162 w[4] = {__halves2bfloat162(l0, l1), __halves2bfloat162(l2, d0),
+                             __halves2bfloat162(d1, z), __halves2bfloat162(z, z)};
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.rowterms) + row * 16);
+      dst[0] = *reinterpret_cast<const uint4*>(w);
+      dst[1] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
 }

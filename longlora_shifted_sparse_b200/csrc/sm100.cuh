@@ -156,6 +156,32 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// TMA tile store from shared memory (bulk-group completion). Same coordinate rules as the
+// loads; the coordinates of a store are never negative here.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y,
+                                             int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_group() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Waits until every committed bulk store of this thread has finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_group_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Makes this thread's generic-proxy shared-memory writes visible to the async proxy (TMA
+// stores, tensor-core operand reads).
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Prefetch of a tile into L2 (no shared memory, no barrier): a later load of the same box
 // then hits in L2. Same coordinate rules as the loads (x * element size a multiple of 16).
 __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int x, int y) {
@@ -299,6 +325,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
          | ((b_mn_major ? 1u : 0u) << 16)            // B major-ness
          | ((uint32_t)(N >> 3) << 17)                // N / 8
          | ((uint32_t)(M >> 4) << 24);               // M / 16
+}
+
+// Shared-memory matrix descriptor, 32-byte swizzle, K-major: rows of 16 bf16 (32 bytes),
+// 8-row groups 256 bytes apart; one MMA k-step covers the whole row.
+__device__ __forceinline__ uint64_t smem_desc_sw32(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;             // leading offset: unused for this layout
+  d |= (uint64_t)(256u >> 4) << 32;    // stride offset: 8 rows x 32 bytes
+  d |= (uint64_t)1u << 46;             // version
+  d |= (uint64_t)6u << 61;             // swizzle: 32B
+  return d;
 }
 
 // Shared-memory matrix descriptor, 128-byte swizzle, sm100 layout version 1.

@@ -73,12 +73,6 @@ __device__ __forceinline__ uint64_t score_pair(const uint32_t (&x0)[32], const u
                 : f2pack(__uint_as_float(x1[c - 32]), __uint_as_float(x1[c - 31]));
 }
 
-// -LSE log2(e) of query rows c, c+1 of a warp's 64 (lane l holds rows l and 32 + l).
-__device__ __forceinline__ uint64_t lse_pair(const float (&nl2)[2], int c) {
-  return f2pack(__shfl_sync(0xffffffffu, nl2[c >> 5], c & 31),
-                __shfl_sync(0xffffffffu, nl2[c >> 5], (c + 1) & 31));
-}
-
 // K-major operand (128 rows x 128 bf16 in two 64-column SW128 boxes), k-step kk.
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t tile_saddr, int kk) {
   return smem_desc_sw128(tile_saddr + (kk >> 2) * kBoxBytes + (kk & 3) * 32, 16, 1024);
@@ -105,19 +99,15 @@ __device__ __forceinline__ uint64_t opaque64(uint64_t v) {
   return r;
 }
 
-// Column c of a thread's 64 probabilities takes its exponential from the FMA-pipe polynomial
-// (fastmath.cuh) when bit c of the mask is set, else from the MUFU unit; off the diagonal
-// tiles only (no -inf scores there; the polynomial clamps its argument at -125). On a B200,
-// 32k workload, moving 1/8, 1/4 or 3/8 of a pass's exponentials to the polynomial left it
-// as fast or slowed it (dQ 2.96 -> 2.94 / 3.01 / 3.17 ms, dK/dV 4.41 -> 4.49 / 4.68 ms), so
-// both masks default to 0 (all exponentials on the MUFU).
-#ifndef S2_DKDV_POLY_MASK
-#define S2_DKDV_POLY_MASK 0x0ull
-#endif
+// Column c of a thread's 64 probabilities in the dQ pass takes its exponential from the
+// FMA-pipe polynomial (fastmath.cuh) when bit c of the mask is set, else from the MUFU unit;
+// off the diagonal tiles only (no -inf scores there; the polynomial clamps its argument at
+// -125). On a B200, 32k workload, moving 1/8, 1/4 or 3/8 of the exponentials to the
+// polynomial left the pass as fast or slowed it (2.96 -> 2.94 / 3.01 / 3.17 ms), so the
+// mask defaults to 0 (all exponentials on the MUFU).
 #ifndef S2_DQ_POLY_MASK
 #define S2_DQ_POLY_MASK 0x0ull
 #endif
-constexpr unsigned long long kDkdvPolyMask = S2_DKDV_POLY_MASK;
 constexpr unsigned long long kDqPolyMask = S2_DQ_POLY_MASK;
 template <unsigned long long kMask>
 __device__ __forceinline__ float exp2_mixed(float x, int c) {
@@ -146,13 +136,12 @@ __device__ __forceinline__ void pin_regs(float (&x)[64]) {
   for (int c = 0; c < 64; c++) asm volatile("" : "+f"(x[c]));
 }
 
-// TMEM column of the bf16 A operand for k-step kk (16 K rows = 8 packed columns). Each
-// math warp owns 64 K rows (columns c0 = 0 or 64 of the tile) and writes them chunk by
-// chunk (32 K rows each) into the 32 fp32 columns it has just read:
-//   dQ pass: dS at region + c0 + 16 * chunk .. + 16          -> packed_col(region, kk, 16)
-//   dK/dV:   P^T at region + c0 + 32 * chunk, dS^T 16 later  -> packed_col(region, kk, 32)
-__device__ __forceinline__ uint32_t packed_col(uint32_t region, int kk, int chunk_stride) {
-  return region + (kk >> 2) * 64 + ((kk >> 1) & 1) * chunk_stride + (kk & 1) * 8;
+// TMEM column of the bf16 A operand for k-step kk (16 K rows = 8 packed columns) in the dQ
+// pass. Each math warp owns 64 K rows (columns c0 = 0 or 64 of the tile) and writes dS
+// chunk by chunk (32 K rows each) into the first 16 of each 32 fp32 columns it has just
+// read: region + c0 + 16 * chunk .. + 16.
+__device__ __forceinline__ uint32_t packed_col(uint32_t region, int kk) {
+  return region + (kk >> 2) * 64 + ((kk >> 1) & 1) * 16 + (kk & 1) * 8;
 }
 
 // Rotates a chunk of 32 consecutive fp32 columns (16 channel pairs starting at pair p0)
@@ -168,13 +157,6 @@ __device__ __forceinline__ void unrotate_pack(const uint32_t (&x)[32], const flo
   }
 }
 
-__device__ __forceinline__ void scale_pack(const uint32_t (&x)[32], float scale, uint4 (&out)[4]) {
-  uint32_t* w = reinterpret_cast<uint32_t*>(out);
-#pragma unroll
-  for (int t = 0; t < 16; t++)
-    w[t] = pack_bf16x2(__uint_as_float(x[2 * t]) * scale, __uint_as_float(x[2 * t + 1]) * scale);
-}
-
 __device__ __forceinline__ void store_row64(__nv_bfloat16* dst, const uint4 (&a)[4]) {
   uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
@@ -183,30 +165,50 @@ __device__ __forceinline__ void store_row64(__nv_bfloat16* dst, const uint4 (&a)
 
 // ================================================================================ dK / dV
 
-// smem: K | V | Q stages 0..2 | dO stages 0..1
-constexpr int kQStages = 3, kDOStages = 2;
+// smem: K | V | Q stages 0..2 (each a 32 KB tile followed by its 4 KB row-term block) | dO |
+// the two constant row-term operands (4 KB each). After the last pair the K, V region holds
+// the (cos, sin) rows of the key tile and Q stages 0, 1 the bf16 dK, dV tiles on their way out.
+constexpr int kQStages = 3;
+constexpr uint32_t kTermBytes = kTile * 16 * 2;              // 128 rows x 16 bf16, SW32
+constexpr uint32_t kQStageBytes = kTileBytes + kTermBytes;
+constexpr uint32_t kKVOffK = 0;
+constexpr uint32_t kKVOffV = kTileBytes;
+constexpr uint32_t kKVOffQ = 2 * kTileBytes;
+constexpr uint32_t kKVOffDO = kKVOffQ + kQStages * kQStageBytes;
+constexpr uint32_t kKVOffKTerm = kKVOffDO + kTileBytes;
+constexpr uint32_t kKVOffVTerm = kKVOffKTerm + kTermBytes;
+constexpr uint32_t kKVSmem = kKVOffVTerm + kTermBytes + 1024;
 #ifndef S2_DKDV_PREFETCH_AHEAD
 #define S2_DKDV_PREFETCH_AHEAD 2
 #endif
 constexpr int kPrefetchAhead = S2_DKDV_PREFETCH_AHEAD;  // pairs between L2 prefetch and use
-constexpr uint32_t kKVOffK = 0;
-constexpr uint32_t kKVOffV = kTileBytes;
-constexpr uint32_t kKVOffQ = 2 * kTileBytes;
-constexpr uint32_t kKVOffDO = (2 + kQStages) * kTileBytes;
-constexpr uint32_t kKVSmem = (2 + kQStages + kDOStages) * kTileBytes + 1024;
+constexpr uint32_t kCsBoxBytes = kTile * 32 * 4;         // 128 rows x 32 floats
 
 struct DkdvBarriers {
-  uint64_t kv_full;
+  uint64_t kv_full, cs_full;
   uint64_t q_full[kQStages], q_empty[kQStages];
-  uint64_t do_full[kDOStages], do_empty[kDOStages];
-  uint64_t st_full, st_consumed, dpt_full, pds_ready;
-  uint64_t acc_done, drain;
+  uint64_t do_full, do_empty;
+  uint64_t st_full, p_ready, dpt_full, ds_ready;
+  uint64_t kv_free, acc_done, drain;
 };
+
+// One row of the constant operand of the row-term k-step: bf16 ones at the given element
+// positions of the 16, the same in both 16-byte halves (so the row reads the same under the
+// 32-byte swizzle whichever half comes first; the row-term rows are zero in elements 8..15).
+__device__ __forceinline__ uint4 term_row_half(int first, int count) {
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  for (int e = first; e < first + count; e++) w[e >> 1] |= 0x3F80u << ((e & 1) * 16);
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     tc_dkdv_kernel(const Params p, const __grid_constant__ CUtensorMap tm_q,
                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   const __grid_constant__ CUtensorMap tm_do) {
+                   const __grid_constant__ CUtensorMap tm_do,
+                   const __grid_constant__ CUtensorMap tm_terms,
+                   const __grid_constant__ CUtensorMap tm_cs,
+                   const __grid_constant__ CUtensorMap tm_dk,
+                   const __grid_constant__ CUtensorMap tm_dv) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -228,22 +230,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int np = R * nq;       // (query head, query tile) pairs
   const int mk0 = src_row(g * p.G + kt * kTile, sh, p.G, p.N);
 
+  // the constant operands of the row-term k-step: ones against -LSE*sqrt(d) (elements
+  // 0..2) for S^T, against -D (elements 3, 4) for dP^T
+  {
+    const uint4 kt_half = term_row_half(0, 3), vt_half = term_row_half(3, 2);
+    uint4* kterm = reinterpret_cast<uint4*>(smem + kKVOffKTerm);
+    uint4* vterm = reinterpret_cast<uint4*>(smem + kKVOffVTerm);
+    for (int i = threadIdx.x; i < (int)(kTermBytes / 16); i += kThreads) {
+      kterm[i] = kt_half;
+      vterm[i] = vt_half;
+    }
+    fence_proxy_async_shared();
+  }
   Abort ab{&abort_flag, p.status, p.wait_limit_ns};
   if (threadIdx.x == 0) {
     abort_flag = *reinterpret_cast<volatile unsigned*>(p.status) != 0u;
     mbar_init(smem_addr(&bars.kv_full), 1);
+    mbar_init(smem_addr(&bars.cs_full), 1);
     for (int s = 0; s < kQStages; s++) {
       mbar_init(smem_addr(&bars.q_full[s]), 1);
       mbar_init(smem_addr(&bars.q_empty[s]), 1);
     }
-    for (int s = 0; s < kDOStages; s++) {
-      mbar_init(smem_addr(&bars.do_full[s]), 1);
-      mbar_init(smem_addr(&bars.do_empty[s]), 1);
-    }
+    mbar_init(smem_addr(&bars.do_full), 1);
+    mbar_init(smem_addr(&bars.do_empty), 1);
     mbar_init(smem_addr(&bars.st_full), 1);
-    mbar_init(smem_addr(&bars.st_consumed), kMathThreads);
+    mbar_init(smem_addr(&bars.p_ready), kMathThreads);
     mbar_init(smem_addr(&bars.dpt_full), 1);
-    mbar_init(smem_addr(&bars.pds_ready), kMathThreads);
+    mbar_init(smem_addr(&bars.ds_ready), kMathThreads);
+    mbar_init(smem_addr(&bars.kv_free), 1);
     mbar_init(smem_addr(&bars.acc_done), 1);
     mbar_init(smem_addr(&bars.drain), 1);
     fence_barrier_init();
@@ -255,6 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = tmem_base_sh;
   const uint32_t colST = 0, colDPT = 128, colDV = 256, colDK = 384;
   const uint32_t sK = smem_addr(smem + kKVOffK), sV = smem_addr(smem + kKVOffV);
+  const uint32_t sDO = smem_addr(smem + kKVOffDO);
   const bool skip = abort_flag != 0;
 
   // Pairs run query tile it0 .. T-1 of query head kvh*R, then of the next head, and so on.
@@ -276,12 +291,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (skip) {
   } else if (warp == 0) {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------ TMA producer: K, V, Q
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
+      tma_prefetch_desc(&tm_terms);
+      tma_prefetch_desc(&tm_cs);
       const uint32_t kvb = smem_addr(&bars.kv_full);
       mbar_arrive_expect_tx(kvb, 2 * kTileBytes);
       const int krow = (b * p.Hkv + kvh) * p.N + mk0;
@@ -289,12 +306,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_2d(sK + kBoxBytes, &tm_k, kvb, 64, krow);
       tma_load_3d(sV, &tm_v, kvb, 0, kvh, b * p.N + mk0);
       tma_load_3d(sV + kBoxBytes, &tm_v, kvb, 64, kvh, b * p.N + mk0);
-      int nq_issued = 0, ndo_issued = 0;
+      {
+        // the K, V tiles of the CTA that will most likely follow this one on an SM (one
+        // SM's worth of CTAs later) into L2, so that its first loads hit there
+        unsigned nsm;
+        asm("mov.u32 %0, %%nsmid;" : "=r"(nsm));
+        const int nx = (int)blockIdx.x + (int)nsm;
+        if (nx < (int)gridDim.x) {
+          int kt2, bkg2;
+          chunked_lpt(nx, p.B * p.Hkv * ng, T, bkg2, kt2);
+          const int g2 = bkg2 % ng, bk2 = bkg2 / ng;
+          const int kvh2 = bk2 % p.Hkv, b2 = bk2 / p.Hkv;
+          const int mk2 = src_row(g2 * p.G + kt2 * kTile, kv_head_shifted(kvh2, p), p.G, p.N);
+          const int krow2 = (b2 * p.Hkv + kvh2) * p.N + mk2;
+          tma_prefetch_l2_2d(&tm_k, 0, krow2);
+          tma_prefetch_l2_2d(&tm_k, 64, krow2);
+          tma_prefetch_l2_3d(&tm_v, 0, kvh2, b2 * p.N + mk2);
+          tma_prefetch_l2_3d(&tm_v, 64, kvh2, b2 * p.N + mk2);
+        }
+      }
+      int nq_issued = 0;
       PairCursor pc = pair_first(), pf = pair_first();
       for (int t = 0; t < kPrefetchAhead; t++) pair_next(pf);
       for (int n = 0; n < np; n++, pair_next(pc), pair_next(pf)) {
         const int h = pc.h, mq0 = pair_row0(pc);
-        const int sq = n % kQStages, sd = n % kDOStages;
+        const int sq = n % kQStages;
         // the Q and dO tiles of pair n + kPrefetchAhead into L2 before this thread blocks on
         // a free ring stage: their loads into shared memory then hit in L2
         if (n + kPrefetchAhead < np) {
@@ -307,87 +343,111 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!mbar_wait(smem_addr(&bars.q_empty[sq]), ((n / kQStages) & 1) ^ 1, ab)) break;
         const uint32_t qb = smem_addr(&bars.q_full[sq]);
-        const uint32_t sQ = smem_addr(smem + kKVOffQ + sq * kTileBytes);
-        mbar_arrive_expect_tx(qb, kTileBytes);
+        const uint32_t sQ = smem_addr(smem + kKVOffQ + sq * kQStageBytes);
+        mbar_arrive_expect_tx(qb, kQStageBytes);
         const int qrow = (b * p.Hq + h) * p.N + mq0;
         tma_load_2d(sQ, &tm_q, qb, 0, qrow);
         tma_load_2d(sQ + kBoxBytes, &tm_q, qb, 64, qrow);
+        tma_load_2d(sQ + kTileBytes, &tm_terms, qb, 0, qrow);
         nq_issued = n + 1;
-        if (!mbar_wait(smem_addr(&bars.do_empty[sd]), ((n / kDOStages) & 1) ^ 1, ab)) break;
-        const uint32_t db = smem_addr(&bars.do_full[sd]);
-        const uint32_t sDO = smem_addr(smem + kKVOffDO + sd * kTileBytes);
-        mbar_arrive_expect_tx(db, kTileBytes);
-        tma_load_3d(sDO, &tm_do, db, 0, h, b * p.N + mq0);
-        tma_load_3d(sDO + kBoxBytes, &tm_do, db, 64, h, b * p.N + mq0);
-        ndo_issued = n + 1;
+      }
+      // once the last MMA that reads K and V has completed, the (cos, sin) rows of the key
+      // tile (the epilogue's inverse rotation) take their place
+      bool cs_issued = false;
+      if (nq_issued == np && mbar_wait(smem_addr(&bars.kv_free), 0, ab)) {
+        const uint32_t cb = smem_addr(&bars.cs_full);
+        mbar_arrive_expect_tx(cb, 4 * kCsBoxBytes);
+        for (int x = 0; x < 4; x++) tma_load_2d(sK + x * kCsBoxBytes, &tm_cs, cb, 32 * x, mk0);
+        cs_issued = true;
       }
       for (int n = nq_issued - 1; n >= 0 && n >= nq_issued - kQStages; n--)
         mbar_wait_drain(smem_addr(&bars.q_full[n % kQStages]), (n / kQStages) & 1, p.status,
                         p.wait_limit_ns);
-      for (int n = ndo_issued - 1; n >= 0 && n >= ndo_issued - kDOStages; n--)
-        mbar_wait_drain(smem_addr(&bars.do_full[n % kDOStages]), (n / kDOStages) & 1, p.status,
-                        p.wait_limit_ns);
       mbar_wait_drain(kvb, 0, p.status, p.wait_limit_ns);
+      if (cs_issued) mbar_wait_drain(smem_addr(&bars.cs_full), 0, p.status, p.wait_limit_ns);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------------ TMA producer: dO
+    if (lane == 0) {
+      int ndo_issued = 0;
+      PairCursor pc = pair_first();
+      for (int n = 0; n < np; n++, pair_next(pc)) {
+        if (!mbar_wait(smem_addr(&bars.do_empty), (n & 1) ^ 1, ab)) break;
+        const uint32_t db = smem_addr(&bars.do_full);
+        const int mq0 = pair_row0(pc);
+        mbar_arrive_expect_tx(db, kTileBytes);
+        tma_load_3d(sDO, &tm_do, db, 0, pc.h, b * p.N + mq0);
+        tma_load_3d(sDO + kBoxBytes, &tm_do, db, 64, pc.h, b * p.N + mq0);
+        ndo_issued = n + 1;
+      }
+      if (ndo_issued > 0)
+        mbar_wait_drain(smem_addr(&bars.do_full), (ndo_issued - 1) & 1, p.status,
+                        p.wait_limit_ns);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
       const uint32_t idesc_g = idesc_bf16_f32(kTile, kD, false, true);
-      auto issue_st = [&](int n) -> bool {  // S^T(n) = K Q_n^T
+      const uint64_t dKT = smem_desc_sw32(smem_addr(smem + kKVOffKTerm));
+      const uint64_t dVT = smem_desc_sw32(smem_addr(smem + kKVOffVTerm));
+      auto stage_q = [&](int n) { return smem_addr(smem + kKVOffQ + (n % kQStages) * kQStageBytes); };
+      // S^T(n) - LSE*sqrt(d) = K Q_n^T + 1 (row terms)^T: eight k-steps and the row-term step
+      auto issue_st = [&](int n) -> bool {
         const int sq = n % kQStages;
         if (!mbar_wait(smem_addr(&bars.q_full[sq]), (n / kQStages) & 1, ab)) return false;
         tc_fence_after();
-        const uint32_t sQ = smem_addr(smem + kKVOffQ + sq * kTileBytes);
+        const uint32_t sQ = stage_q(n);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; kk++)
           mma_ss(tmem + colST, kmajor_desc(sK, kk), kmajor_desc(sQ, kk), idesc_s, kk > 0);
+        mma_ss(tmem + colST, dKT, smem_desc_sw32(sQ + kTileBytes), idesc_s, 1u);
         // failure-path self-test: CTA 0 (key tile 0, at least two pairs) withholds the
         // arrival of S^T(1), so that the math warps and then this thread wait in vain
         if (!(p.inject == kInjectDkdv && blockIdx.x == 0 && n == 1))
           mma_commit(smem_addr(&bars.st_full));
         return true;
       };
-      auto issue_dpt = [&](int n) -> bool {  // dP^T(n) = V dO_n^T
-        const int sd = n % kDOStages;
-        if (!mbar_wait(smem_addr(&bars.do_full[sd]), (n / kDOStages) & 1, ab)) return false;
+      // dP^T(n) - D = V dO_n^T + 1 (row terms)^T (the row terms sit in Q stage n)
+      auto issue_dpt = [&](int n) -> bool {
+        if (!mbar_wait(smem_addr(&bars.do_full), n & 1, ab)) return false;
         tc_fence_after();
-        const uint32_t sDO = smem_addr(smem + kKVOffDO + sd * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; kk++)
           mma_ss(tmem + colDPT, kmajor_desc(sV, kk), kmajor_desc(sDO, kk), idesc_s, kk > 0);
+        mma_ss(tmem + colDPT, dVT, smem_desc_sw32(stage_q(n) + kTileBytes), idesc_s, 1u);
         mma_commit(smem_addr(&bars.dpt_full));
         return true;
       };
-      // issue order: S^T(0) dP^T(0) S^T(1) | dV(0) dK(0) dP^T(1) S^T(2) | dV(1) ...
-      // After the math warps publish P^T, dS^T of pair n the gradient MMAs of n and dP^T of
-      // n+1 go first (the next math phase waits for them); S^T of n+2 then fills the tensor
-      // pipe while the math warps work on pair n+1.
+      // Per pair n: dV(n) once the math warps have written P^T(n) over S^T(n), then S^T(n+1)
+      // over it (the MMAs run in issue order); dK(n) once they have written dS^T(n) over
+      // dP^T(n), then dP^T(n+1) over it. The math warps' exponentials of pair n+1 then run
+      // while dK(n) and dP^T(n+1) occupy the tensor cores.
       bool ok = mbar_wait(smem_addr(&bars.kv_full), 0, ab);
       tc_fence_after();
       if (ok && np > 0) ok = issue_st(0) && issue_dpt(0);
-      if (ok && np > 1) ok = mbar_wait(smem_addr(&bars.st_consumed), 0, ab) && issue_st(1);
+      if (ok && np == 1) mma_commit(smem_addr(&bars.kv_free));
       for (int n = 0; ok && n < np; n++) {
         const uint32_t ph = n & 1;
-        if (!mbar_wait(smem_addr(&bars.pds_ready), ph, ab)) break;
+        if (!mbar_wait(smem_addr(&bars.p_ready), ph, ab)) break;
         tc_fence_after();
-        const uint32_t sQ = smem_addr(smem + kKVOffQ + (n % kQStages) * kTileBytes);
-        const uint32_t sDO = smem_addr(smem + kKVOffDO + (n % kDOStages) * kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; kk++)
-          mma_ts(tmem + colDV, tmem + packed_col(colDPT, kk, 32), mn_desc(sDO, kk), idesc_g,
-                 (n > 0 || kk > 0));
-        mma_commit(smem_addr(&bars.do_empty[n % kDOStages]));
+          mma_ts(tmem + colDV, tmem + colST + (kk >> 2) * 64 + (kk & 3) * 8, mn_desc(sDO, kk),
+                 idesc_g, (n > 0 || kk > 0));
+        mma_commit(smem_addr(&bars.do_empty));
+        if (n + 1 < np && !issue_st(n + 1)) break;
+        if (!mbar_wait(smem_addr(&bars.ds_ready), ph, ab)) break;
+        tc_fence_after();
+        const uint32_t sQ = stage_q(n);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; kk++)
-          mma_ts(tmem + colDK, tmem + packed_col(colDPT + 16, kk, 32), mn_desc(sQ, kk), idesc_g,
-                 (n > 0 || kk > 0));
+          mma_ts(tmem + colDK, tmem + colDPT + (kk >> 2) * 64 + (kk & 3) * 8, mn_desc(sQ, kk),
+                 idesc_g, (n > 0 || kk > 0));
         mma_commit(smem_addr(&bars.q_empty[n % kQStages]));
-        if (n + 1 < np && !issue_dpt(n + 1)) break;
-        // S^T(n+2) once the math warps hold S^T(n+1) in registers
-        if (n + 2 < np) {
-          if (!mbar_wait(smem_addr(&bars.st_consumed), (n + 1) & 1, ab)) break;
-          if (!issue_st(n + 2)) break;
+        if (n + 1 < np) {
+          if (!issue_dpt(n + 1)) break;
+          if (n + 2 == np) mma_commit(smem_addr(&bars.kv_free));  // the last reader of K, V
         }
       }
       mma_commit(smem_addr(&bars.acc_done));
@@ -402,114 +462,126 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tST = tmem + lane_off + colST + c0;
     const uint32_t tDPT = tmem + lane_off + colDPT + c0;
-    const float sl2 = p.scale_log2;
-    const uint64_t sl2x2 = f2pack(sl2, sl2);
-    // LSE and D of this warp's 64 query rows: lane l holds rows c0 + l and c0 + 32 + l;
-    // loaded one pair ahead and broadcast with shuffles
-    auto load_ld = [&](const PairCursor& pc, float (&l2)[2], float (&dd)[2]) {
-      const size_t base = ((size_t)b * p.Hq + pc.h) * p.N + pair_row0(pc) + c0 + lane;
-      l2[0] = -__ldg(p.lse + base) * kLog2e;
-      l2[1] = -__ldg(p.lse + base + 32) * kLog2e;
-      dd[0] = __ldg(p.Dsum + base);
-      dd[1] = __ldg(p.Dsum + base + 32);
-    };
-    float nl2[2], dsum[2], nl2_next[2] = {0.f, 0.f}, dsum_next[2] = {0.f, 0.f};
-    PairCursor cur = pair_first(), nxt = pair_first();
-    if (np > 0) load_ld(cur, nl2, dsum);
-    pair_next(nxt);
+    const uint64_t sl2x2 = f2pack(p.scale_log2, p.scale_log2);
+    PairCursor cur = pair_first();
     bool ok = true;
     for (int n = 0; n < np; n++) {
-      if (n + 1 < np) load_ld(nxt, nl2_next, dsum_next);
       const bool diag = p.causal && cur.iq == kt;
-      cur = nxt;
-      pair_next(nxt);
+      pair_next(cur);
       ok = mbar_wait(smem_addr(&bars.st_full), n & 1, ab);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
+      // P^T = exp2((S^T - LSE sqrt(d)) log2(e) / sqrt(d)); the row terms came with the MMA
       float pr[64];
       {
         uint32_t x0[32], x1[32];
         tmem_ld32(tST, x0);
         tmem_ld32(tST + 32, x1);
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(smem_addr(&bars.st_consumed));  // S^T may now be overwritten
-        if (diag) {
-          mask_scores(x0, x1, row - c0, 0);  // query row c0+c before key row: P = 0
+        if (diag) mask_scores(x0, x1, row - c0, 0);  // query row c0+c before key row: P = 0
 #pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            float a0, a1;
-            f2unpack(ffma2(score_pair(x0, x1, c), sl2x2, lse_pair(nl2, c)), a0, a1);
-            pr[c] = fast_exp2(a0);
-            pr[c + 1] = fast_exp2(a1);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 64; c += 2) {
-            float a0, a1;
-            f2unpack(ffma2(score_pair(x0, x1, c), sl2x2, lse_pair(nl2, c)), a0, a1);
-            pr[c] = exp2_mixed<kDkdvPolyMask>(a0, c);
-            pr[c + 1] = exp2_mixed<kDkdvPolyMask>(a1, c + 1);
-          }
+        for (int c = 0; c < 64; c += 2) {
+          float a0, a1;
+          f2unpack(fmul2(score_pair(x0, x1, c), sl2x2), a0, a1);
+          pr[c] = fast_exp2(a0);
+          pr[c + 1] = fast_exp2(a1);
         }
-        pin_regs(pr);
+        uint32_t pp[32];
+#pragma unroll
+        for (int t = 0; t < 32; t++) pp[t] = pack_bf16x2(pr[2 * t], pr[2 * t + 1]);
+        tmem_st32(tST, pp);  // P^T of these 64 query rows over their scores, bf16 pairs
       }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_addr(&bars.p_ready));
       ok = mbar_wait(smem_addr(&bars.dpt_full), n & 1, ab);
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after();
+      // dS^T = P^T (dP^T - D); the row terms came with the MMA
       {
         uint32_t x0[32], x1[32];
         tmem_ld32(tDPT, x0);
         tmem_ld32(tDPT + 32, x1);
         tmem_wait_ld();
+        uint32_t pd[32];
 #pragma unroll
-        for (int ch = 0; ch < 2; ch++) {
-          uint32_t pp[16], pd[16];
-#pragma unroll
-          for (int t = 0; t < 16; t++) {
-            const int c = ch * 32 + 2 * t;
-            const float d0 = __shfl_sync(0xffffffffu, dsum[ch], 2 * t);
-            const float d1 = __shfl_sync(0xffffffffu, dsum[ch], 2 * t + 1);
-            float s0, s1;
-            f2unpack(fmul2(f2pack(pr[c], pr[c + 1]), fsub2(score_pair(x0, x1, c), f2pack(d0, d1))),
-                     s0, s1);
-            pp[t] = pack_bf16x2(pr[c], pr[c + 1]);
-            pd[t] = pack_bf16x2(s0, s1);
-          }
-          tmem_st16(tDPT + ch * 32, pp);       // P^T of these 32 query rows
-          tmem_st16(tDPT + ch * 32 + 16, pd);  // dS^T
+        for (int t = 0; t < 32; t++) {
+          float s0, s1;
+          f2unpack(fmul2(f2pack(pr[2 * t], pr[2 * t + 1]), score_pair(x0, x1, 2 * t)), s0, s1);
+          pd[t] = pack_bf16x2(s0, s1);
         }
+        tmem_st32(tDPT, pd);  // dS^T over dP^T
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_addr(&bars.pds_ready));
-      nl2[0] = nl2_next[0]; nl2[1] = nl2_next[1];
-      dsum[0] = dsum_next[0]; dsum[1] = dsum_next[1];
+      mbar_arrive(smem_addr(&bars.ds_ready));
     }
+    // Epilogue, taken by all eight math warps together or by none (every wait above is
+    // bounded, so each warp gets here): dk = R^T (dK / sqrt(d)) and dv = dV as bf16 tiles in
+    // shared memory (Q stages 0 and 1, 128-byte swizzle), then two TMA stores each.
     if (ok) {
       ok = mbar_wait(smem_addr(&bars.acc_done), 0, ab);
       __syncwarp();
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
+      ok = mbar_wait(smem_addr(&bars.cs_full), 0, ab);
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (named_bar_and(1, kMathThreads, ok)) {
       tc_fence_after();
-      const int m = src_row(g * p.G + kt * kTile + row, sh, p.G, p.N);
-      const size_t off = ((size_t)(b * p.N + m) * p.Hkv + kvh) * kD + c0;
-      const float2* cs_row = p.cs + (size_t)m * (kD / 2);
+      const int sw = row & 7;
+      uint8_t* const stage_dk = smem + kKVOffQ + (c0 >> 6) * kBoxBytes + row * 128;
+      uint8_t* const stage_dv = smem + kKVOffQ + kQStageBytes + (c0 >> 6) * kBoxBytes + row * 128;
 #pragma unroll
       for (int ch = 0; ch < 2; ch++) {
+        // (cos, sin) of this row's channel pairs c0/2 + 16ch .. +15: box c0/32 + ch of the
+        // table rows, 16-byte chunk j at j ^ (row & 7)
+        const uint8_t* cs_row = smem + ((c0 >> 5) + ch) * kCsBoxBytes + row * 128;
         uint32_t x[32];
-        uint4 o[4];
         tmem_ld32(tmem + lane_off + colDK + c0 + ch * 32, x);
         tmem_wait_ld();
-        unrotate_pack(x, cs_row, (c0 + ch * 32) / 2, p.scale, o);
-        store_row64(static_cast<__nv_bfloat16*>(p.dk) + off + ch * 32, o);
+        uint32_t w[16];
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+          const float4 cs = *reinterpret_cast<const float4*>(cs_row + ((j ^ sw) << 4));
+#pragma unroll
+          for (int e = 0; e < 2; e++) {
+            const int t = 2 * j + e;
+            const float c = e ? cs.z : cs.x, s = e ? cs.w : cs.y;
+            const float x0 = __uint_as_float(x[2 * t]) * p.scale;
+            const float x1 = __uint_as_float(x[2 * t + 1]) * p.scale;
+            w[t] = pack_bf16x2(fmaf(x0, c, x1 * s), fmaf(-x0, s, x1 * c));
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; u++)
+          *reinterpret_cast<uint4*>(stage_dk + (((4 * ch + u) ^ sw) << 4)) =
+              make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
         tmem_ld32(tmem + lane_off + colDV + c0 + ch * 32, x);
         tmem_wait_ld();
-        scale_pack(x, 1.f, o);
-        store_row64(static_cast<__nv_bfloat16*>(p.dv) + off + ch * 32, o);
+#pragma unroll
+        for (int t = 0; t < 16; t++)
+          w[t] = pack_bf16x2(__uint_as_float(x[2 * t]), __uint_as_float(x[2 * t + 1]));
+#pragma unroll
+        for (int u = 0; u < 4; u++)
+          *reinterpret_cast<uint4*>(stage_dv + (((4 * ch + u) ^ sw) << 4)) =
+              make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+      }
+      fence_proxy_async_shared();
+      named_bar_sync(1, kMathThreads);
+      if (warp == 4 && lane == 0) {
+        const uint32_t sdk = smem_addr(smem + kKVOffQ);
+        const uint32_t sdv = smem_addr(smem + kKVOffQ + kQStageBytes);
+        tma_store_3d(&tm_dk, sdk, 0, kvh, b * p.N + mk0);
+        tma_store_3d(&tm_dk, sdk + kBoxBytes, 64, kvh, b * p.N + mk0);
+        tma_store_3d(&tm_dv, sdv, 0, kvh, b * p.N + mk0);
+        tma_store_3d(&tm_dv, sdv + kBoxBytes, 64, kvh, b * p.N + mk0);
+        bulk_commit_group();
+        bulk_wait_group_read0();  // shared memory may be released once the stores read it
       }
     }
   }
@@ -808,7 +880,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t acc0 = j > 0;
 #pragma unroll
           for (int kk = 0; kk < kTile / 16; kk++)
-            mma_ts(tmem + colDQ, tmem + packed_col(colDP + (gq & 1) * 128, kk, 16),
+            mma_ts(tmem + colDQ, tmem + packed_col(colDP + (gq & 1) * 128, kk),
                    dkm + mn_koff(kk), idesc_g, kk ? 1u : acc0);
           mma_commit(smem_addr(&bars.dq_done[gq & 1]));
           mma_commit(smem_addr(&bars.k_empty[sk]));
@@ -949,14 +1021,29 @@ cudaError_t make_bwd_maps(const Params& p, CUtensorMap* tq, CUtensorMap* tk, CUt
 }  // namespace
 
 cudaError_t launch_tc_bwd_dkdv(const Params& p, cudaStream_t st) {
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tterms, tcs, tdk, tdv;
   cudaError_t e = make_bwd_maps(p, &tq, &tk, &tv, &tdo);
   if (e) return e;
+  // row terms: rows of 16 bf16 (32 bytes), one per (b, query head, token), 32-byte swizzle
+  if ((e = make_tmap_2d(&tterms, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, CU_TENSOR_MAP_SWIZZLE_32B,
+                        p.rowterms, 16, (uint64_t)p.B * p.Hq * p.N, 32, 16, kTile)))
+    return e;
+  // (cos, sin) table: one row of d floats per token, boxes of 32 floats x 128 tokens
+  if ((e = make_tmap_2d(&tcs, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, CU_TENSOR_MAP_SWIZZLE_128B, p.cs,
+                        kD, (uint64_t)p.N, kD * 4, 32, kTile)))
+    return e;
+  if ((e = make_tmap_bf16_3d(&tdk, p.dk, kD, p.Hkv, (uint64_t)p.B * p.N, kD * 2,
+                             (uint64_t)p.Hkv * kD * 2, 64, kTile)))
+    return e;
+  if ((e = make_tmap_bf16_3d(&tdv, p.dv, kD, p.Hkv, (uint64_t)p.B * p.N, kD * 2,
+                             (uint64_t)p.Hkv * kD * 2, 64, kTile)))
+    return e;
   if ((e = cudaFuncSetAttribute(tc_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kKVSmem)))
     return e;
   const long tiles = (long)p.B * p.Hkv * (p.N / p.G) * (p.G / kTile);
-  tc_dkdv_kernel<<<dim3((unsigned)tiles), dim3(kThreads), kKVSmem, st>>>(p, tq, tk, tv, tdo);
+  tc_dkdv_kernel<<<dim3((unsigned)tiles), dim3(kThreads), kKVSmem, st>>>(p, tq, tk, tv, tdo,
+                                                                        tterms, tcs, tdk, tdv);
   return cudaGetLastError();
 }
 
