@@ -61,7 +61,9 @@ typedef enum {
   S2_ERR_WORKSPACE = 6,      /* workspace NULL or ws_bytes < s2attn_workspace_bytes(...) */
   S2_ERR_CUDA = 7,           /* a CUDA runtime/driver call failed */
   S2_ERR_DEVICE_TIMEOUT = 8, /* a bounded device-side wait expired (see s2attn_device_status) */
-  S2_ERR_ARG = 9             /* pi_scale or rope_base not finite and > 0, or a bad mode */
+  S2_ERR_ARG = 9,            /* pi_scale or rope_base not finite and > 0, or a bad mode */
+  S2_ERR_STALE_WORKSPACE = 10 /* (device status) s2attn_bwd_after_fwd was given a workspace
+                                 whose rotation came from another forward */
 } s2_status;
 
 /* The `mode` argument of the attention calls: S2_CAUSAL or 0, ORed with one S2_SHIFT_*
@@ -90,8 +92,9 @@ typedef enum {
  * depend on G or mode). Returns 0 for arguments that s2attn_fwd would reject with
  * S2_ERR_SHAPE, S2_ERR_HEADDIM or S2_ERR_DTYPE. The workspace holds the rotated q and k
  * (head-major, original token order), the RoPE cos/sin table, the backward's row sums
- * D = rowsum(dO * O), the device status word and the work counters of the persistent
- * kernels. A workspace serves one call at a time: calls whose kernels may overlap on the
+ * D = rowsum(dO * O) and per-row terms (-LSE and -D as bf16 parts, 32 bytes per query
+ * row), the device status word, the fingerprint of the rotation and the work counters of
+ * the persistent kernels. A workspace serves one call at a time: calls whose kernels may overlap on the
  * GPU (e.g. on two streams) need a workspace each. */
 S2_API size_t s2attn_workspace_bytes(int B, int N, int H_q, int H_kv, int d, int dtype);
 
@@ -119,9 +122,13 @@ S2_API s2_status s2attn_bwd(const void* q, const void* k, const void* v, const v
 /* Backward that reuses the forward's rotation: identical arguments, semantics and outputs
  * to s2attn_bwd, but it skips the RoPE + PI pass (one read of q, k and one write of the
  * rotated q~, k~ and of the (cos, sin) table) and reads those from the workspace instead.
- * Precondition, not checked: `workspace` is the one s2attn_fwd used for these same q, k
- * and shape/pi_scale/rope_base/dtype arguments, and neither it (beyond the status word) nor
- * q, k changed since. This is the training-loop order (forward, then backward of the same
+ * Precondition: `workspace` is the one s2attn_fwd used for these same q, k and
+ * shape/G/mode/pi_scale/rope_base/dtype arguments, and neither it (beyond the status word)
+ * nor q, k changed since. The forward records a fingerprint of those arguments (with the q
+ * and k pointers) in the workspace; this call compares it on the device and, on a mismatch,
+ * leaves S2_ERR_STALE_WORKSPACE for s2attn_device_status() and its gradients are undefined
+ * (the tensor-core kernels skip their work). New contents written into the same q, k
+ * buffers are not detected. This is the training-loop order (forward, then backward of the same
  * batch); the method is unchanged, the rotation is computed once per step instead of twice
  * ("LongLoRA: Efficient 100k Context LLM Fine-Tuning Guide", Step 1 applies RoPE once). The
  * status word is reset at the start, as in every other call. */
@@ -173,8 +180,10 @@ S2_API s2_status s2attn_noalloc_device_status(void* cuda_stream);
 S2_API int s2attn_kernel_path(int B, int N, int H_q, int H_kv, int d, int G, int mode, int dtype);
 
 /* Waits for cuda_stream, then reads and clears the device status word of the workspace
- * used by the last call on it: S2_OK, or S2_ERR_DEVICE_TIMEOUT if a bounded wait in a
- * kernel expired (that kernel's outputs are then undefined). S2_ERR_CUDA on a CUDA error. */
+ * used by the last call on it: S2_OK, S2_ERR_DEVICE_TIMEOUT if a bounded wait in a kernel
+ * expired (that kernel's outputs are then undefined), or S2_ERR_STALE_WORKSPACE if
+ * s2attn_bwd_after_fwd found another forward's rotation there (its gradients were not
+ * computed). S2_ERR_CUDA on a CUDA error. */
 S2_API s2_status s2attn_device_status(void* workspace, size_t ws_bytes, void* cuda_stream);
 
 /* Self-test of the device-side failure path: enqueues one tiny kernel whose bounded wait

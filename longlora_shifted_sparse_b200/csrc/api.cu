@@ -232,6 +232,23 @@ Params make_params(int B, int N, int Hq, int Hkv, int d, int G, int mode, float 
 
 s2_status to_status(cudaError_t e) { return e == cudaSuccess ? S2_OK : S2_ERR_CUDA; }
 
+// FNV-1a (64-bit) over the arguments that determine the rotation a call leaves in (or
+// expects from) the workspace. Set after the q and k pointers are.
+void set_fingerprint(Params& p, int mode, int dtype) {
+  uint64_t h = 1469598103934665603ull;
+  auto mix = [&h](const void* x, size_t n) {
+    const unsigned char* c = static_cast<const unsigned char*>(x);
+    for (size_t i = 0; i < n; i++) h = (h ^ c[i]) * 1099511628211ull;
+  };
+  const int ints[8] = {p.B, p.N, p.Hq, p.Hkv, p.d, p.G, mode, dtype};
+  mix(ints, sizeof(ints));
+  mix(&p.pi_scale, sizeof(float));
+  mix(&p.rope_base, sizeof(float));
+  mix(&p.q, sizeof(void*));
+  mix(&p.k, sizeof(void*));
+  p.fingerprint = h;
+}
+
 }  // namespace
 }  // namespace s2
 
@@ -263,6 +280,7 @@ s2_status s2attn_fwd(const void* q, const void* k, const void* v, void* o, float
     return S2_ERR_ALIGN;
   Params p = make_params(B, N, H_q, H_kv, d, G, mode, pi_scale, rope_base, dtype, workspace);
   p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
+  set_fingerprint(p, mode, dtype);
   return to_status(enqueue_forward(p, dtype, static_cast<cudaStream_t>(cuda_stream)));
 }
 
@@ -286,6 +304,8 @@ s2_status backward_impl(const void* q, const void* k, const void* v, const void*
   Params p = make_params(B, N, H_q, H_kv, d, G, mode, pi_scale, rope_base, dtype, workspace);
   p.q = q; p.k = k; p.v = v; p.o = const_cast<void*>(o); p.lse = const_cast<float*>(lse);
   p.dout = dout; p.dq = dq; p.dk = dk; p.dv = dv;
+  set_fingerprint(p, mode, dtype);
+  p.check_fingerprint = !rotate;
   if (inject != kInjectNone) {
     p.inject = inject;
     p.wait_limit_ns = kSelftestWaitLimitNs;
@@ -342,7 +362,7 @@ s2_status s2attn_device_status(void* workspace, size_t ws_bytes, void* cuda_stre
   if (word != 0) {
     if (cudaMemsetAsync(workspace, 0, sizeof(word), s) != cudaSuccess) return S2_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return S2_ERR_CUDA;
-    return S2_ERR_DEVICE_TIMEOUT;
+    return (word & kStatusStale) ? S2_ERR_STALE_WORKSPACE : S2_ERR_DEVICE_TIMEOUT;
   }
   return S2_OK;
 }
@@ -375,6 +395,7 @@ s2_status s2attn_selftest_inject(int site, const void* q, const void* k, const v
     return S2_ERR_ALIGN;
   Params p = make_params(B, N, H_q, H_kv, d, G, mode, pi_scale, rope_base, dtype, workspace);
   p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
+  set_fingerprint(p, mode, dtype);
   p.inject = kInjectFwd;
   p.wait_limit_ns = kSelftestWaitLimitNs;
   return to_status(enqueue_forward(p, dtype, static_cast<cudaStream_t>(cuda_stream)));
@@ -400,6 +421,8 @@ const char* s2attn_status_string(int status) {
     case S2_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
     case S2_ERR_ARG: return "invalid argument (pi_scale, rope_base finite and > 0; mode = "
                              "S2_CAUSAL or 0 | one S2_SHIFT_* pattern)";
+    case S2_ERR_STALE_WORKSPACE: return "s2attn_bwd_after_fwd: the workspace's rotation "
+                                        "belongs to another forward (other q, k or arguments)";
     default: return "unknown status";
   }
 }
@@ -528,6 +551,7 @@ extern "C" s2_status s2attn_fwd_noalloc(const void* q, const void* k, const void
   // everything else the kernels read from the scratch is written earlier in the same call.
   Params p = make_params(B, N, H_q, H_kv, d, G, mode, pi_scale, rope_base, dtype, scratch);
   p.q = q; p.k = k; p.v = v; p.o = o; p.lse = lse;
+  set_fingerprint(p, mode, dtype);
   return to_status(enqueue_forward(p, dtype, static_cast<cudaStream_t>(cuda_stream)));
 }
 

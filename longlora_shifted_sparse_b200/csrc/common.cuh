@@ -38,6 +38,11 @@ struct Params {
   // withholds one barrier arrival so that a wait expires (InjectSite; 0 in normal calls)
   unsigned long long wait_limit_ns;
   int inject;
+  // hash of the call's arguments that determine the rotation held in the workspace (shape,
+  // mode, pi_scale, rope_base, dtype, the q and k pointers): a call that rotates stores it
+  // in the status block; a backward that reuses the rotation compares it (check_fingerprint)
+  unsigned long long fingerprint;
+  int check_fingerprint;
 };
 
 // Where a failure-path self-test withholds one arrival (the issuer of CTA 0 skips the
@@ -45,7 +50,11 @@ struct Params {
 // tile 1 of its first item), kInjectDkdv in the dK/dV pass (S^T of pair 1).
 enum InjectSite : int { kInjectNone = 0, kInjectFwd = 1, kInjectDkdv = 2 };
 
-enum StatusBits : unsigned { kStatusTimeout = 1u };
+// Status word bits: a bounded wait expired; a backward that reuses the forward's rotation
+// found a workspace whose last rotation came from other arguments (its kernels then skip).
+enum StatusBits : unsigned { kStatusTimeout = 1u, kStatusStale = 2u };
+// Words 8 and 9 of the workspace's 256-byte status block: the fingerprint of the rotation.
+constexpr int kFingerprintWord = 8;
 // Time limit of one bounded wait in a normal call (2 s: far beyond any wait of a working
 // kernel, short enough that a stuck launch ends with an error instead of hanging).
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;

@@ -35,12 +35,15 @@ __device__ inline uint4 rotate_vec(uint4 raw, const float2* __restrict__ cs_row)
 
 // (cos, sin) of (m / s) * base^(-2i/d) for every token m and pair i. The first kernel of
 // every forward and of every backward that rotates: it also resets the status word and the
-// persistent kernels' work counters.
+// persistent kernels' work counters, and records which arguments the rotation belongs to.
 __global__ void __launch_bounds__(256) rope_table_kernel(Params p) {
   const int half = p.d / 2;
   const long total = (long)p.N * half;
-  if (blockIdx.x == 0 && threadIdx.x == 0)
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
     for (int c = 0; c <= kNumWorkCounters; c++) p.status[c] = 0u;
+    p.status[kFingerprintWord] = (unsigned)p.fingerprint;
+    p.status[kFingerprintWord + 1] = (unsigned)(p.fingerprint >> 32);
+  }
   // the block size, hence the grid stride, is a multiple of d/2 (the launcher sizes it so),
   // so a thread keeps one pair index i and computes its frequency once
   const long stride = (long)gridDim.x * blockDim.x;

@@ -86,16 +86,25 @@ __global__ void __launch_bounds__(256) simt_fwd_kernel(Params p) {
   if (lane == 0) p.lse[((size_t)b * p.Hq + h) * p.N + m] = mx + logf(l);
 }
 
+// The backward's first kernel when it reuses the forward's rotation: the call starts with a
+// clean status word (no kernel of this launch reads it) and the work counters of the
+// persistent kernels that follow at 0. With check_fingerprint, a workspace whose last
+// rotation came from other arguments sets the stale bit, and the kernels that follow skip.
+__device__ inline void backward_status_reset(const Params& p) {
+  for (int c = 0; c <= kNumWorkCounters; c++) p.status[c] = 0u;
+  if (p.check_fingerprint) {
+    const unsigned long long f = (unsigned long long)p.status[kFingerprintWord] |
+                                 ((unsigned long long)p.status[kFingerprintWord + 1] << 32);
+    if (f != p.fingerprint) p.status[0] = kStatusStale;
+  }
+}
+
 // D[b][h][m] = sum_c dO[b][m][h][c] * O[b][m][h][c] (fp32), one warp per row.
 template <typename T, int DPL>
 __global__ void __launch_bounds__(256) bwd_rowsum_kernel(Params p) {
   const int lane = threadIdx.x & 31;
   const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  // the backward's first kernel when it reuses the forward's rotation: the call starts
-  // with a clean status word (no kernel of this launch reads it) and the work counters of
-  // the persistent kernels that follow at 0
-  if (blockIdx.x == 0 && threadIdx.x == 0)
-    for (int c = 0; c <= kNumWorkCounters; c++) p.status[c] = 0u;
+  if (blockIdx.x == 0 && threadIdx.x == 0) backward_status_reset(p);
   if (warp >= (long)p.B * p.N * p.Hq) return;
   const int h = (int)(warp % p.Hq);
   const long bm = warp / p.Hq;
@@ -108,15 +117,16 @@ __global__ void __launch_bounds__(256) bwd_rowsum_kernel(Params p) {
   if (lane == 0) p.Dsum[((size_t)b * p.Hq + h) * p.N + m] = D;
 }
 
-// D = rowsum(dO * O) for bf16 rows of 128 (the tensor-core path's shape), HBM-bound: rows
-// [B][N][Hq] are contiguous, so 8 consecutive rows (2 KB) go to one warp, a half-warp per
-// row and 16 bytes per lane, with all 8 loads of dO and O issued before the first use.
+// D = rowsum(dO * O) for bf16 rows of 128 (the tensor-core path's shape), HBM-bound, plus
+// the row terms of the tensor-core dK/dV pass. Rows are taken in [B][Hq][N] order, 8
+// consecutive tokens of one head per warp (a half-warp per row, 16 bytes per lane, all 8
+// loads of dO and O issued before the first use), so that the LSE reads and the D and
+// row-term writes of a warp are contiguous; each dO / O row is 256 contiguous bytes.
 __global__ void __launch_bounds__(256) bwd_rowsum_bf16_d128_kernel(Params p) {
   constexpr int kRowsPerWarp = 8;
   const int lane = threadIdx.x & 31, half = lane >> 4, chunk = lane & 15;
   const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (blockIdx.x == 0 && threadIdx.x == 0)  // see bwd_rowsum_kernel
-    for (int c = 0; c <= kNumWorkCounters; c++) p.status[c] = 0u;
+  if (blockIdx.x == 0 && threadIdx.x == 0) backward_status_reset(p);
   const long rows = (long)p.B * p.N * p.Hq;
   const long r0 = warp * kRowsPerWarp;
   if (r0 >= rows) return;
@@ -125,8 +135,14 @@ __global__ void __launch_bounds__(256) bwd_rowsum_bf16_d128_kernel(Params p) {
   uint4 a[kRowsPerWarp / 2], c[kRowsPerWarp / 2];
 #pragma unroll
   for (int i = 0; i < kRowsPerWarp / 2; i++) {
-    const long r = r0 + 2 * i + half;
-    const long e = r < rows ? r * 16 + chunk : 0;  // 16 uint4 per row
+    const long r = r0 + 2 * i + half;  // row (b, h, m) in [B][Hq][N] order
+    long e = 0;
+    if (r < rows) {
+      const int m = (int)(r % p.N);
+      const long bh = r / p.N;
+      const int h = (int)(bh % p.Hq), b = (int)(bh / p.Hq);
+      e = (((long)b * p.N + m) * p.Hq + h) * 16 + chunk;  // 16 uint4 per row
+    }
     a[i] = __ldcs(dO + e);
     c[i] = __ldcs(O + e);
   }
@@ -145,15 +161,11 @@ __global__ void __launch_bounds__(256) bwd_rowsum_bf16_d128_kernel(Params p) {
     for (int o = 8; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     const long r = r0 + 2 * i + half;
     if (chunk == 0 && r < rows) {
-      const int h = (int)(r % p.Hq);
-      const long bm = r / p.Hq;
-      const int m = (int)(bm % p.N), b = (int)(bm / p.N);
-      const size_t row = ((size_t)b * p.Hq + h) * p.N + m;
-      p.Dsum[row] = acc;
+      p.Dsum[r] = acc;
       // the row terms of the tensor-core dK/dV pass: -LSE*sqrt(d) and -D as sums of bf16
       // parts (each part the rounding of what the previous ones left), exact to ~2^-24 and
       // ~2^-16 relative
-      const float nl = -p.lse[row] / p.scale;
+      const float nl = -p.lse[r] / p.scale;
       const __nv_bfloat16 l0 = __float2bfloat16_rn(nl);
       const float r1 = nl - __bfloat162float(l0);
       const __nv_bfloat16 l1 = __float2bfloat16_rn(r1);
@@ -163,7 +175,7 @@ __global__ void __launch_bounds__(256) bwd_rowsum_bf16_d128_kernel(Params p) {
       const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
       __nv_bfloat162 w[4] = {__halves2bfloat162(l0, l1), __halves2bfloat162(l2, d0),
                              __halves2bfloat162(d1, z), __halves2bfloat162(z, z)};
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.rowterms) + row * 16);
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.rowterms) + r * 16);
       dst[0] = *reinterpret_cast<const uint4*>(w);
       dst[1] = make_uint4(0u, 0u, 0u, 0u);
     }

@@ -19,7 +19,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libs2attn.so")
 
 S2_OK, S2_ERR_NULL, S2_ERR_SHAPE, S2_ERR_DTYPE, S2_ERR_HEADDIM, S2_ERR_ALIGN, \
-    S2_ERR_WORKSPACE, S2_ERR_CUDA, S2_ERR_DEVICE_TIMEOUT, S2_ERR_ARG = range(10)
+    S2_ERR_WORKSPACE, S2_ERR_CUDA, S2_ERR_DEVICE_TIMEOUT, S2_ERR_ARG, \
+    S2_ERR_STALE_WORKSPACE = range(11)
 S2_BF16, S2_FP32 = 0, 1
 S2_CAUSAL, S2_SHIFT_HALF, S2_SHIFT_ALTERNATE, S2_SHIFT_NONE = 0x01, 0x00, 0x10, 0x20
 S2_INJECT_FWD, S2_INJECT_DKDV = 1, 2

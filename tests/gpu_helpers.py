@@ -2,10 +2,27 @@
 through its C ABI, bring results back, and compare them with the oracle's."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
 import synth
+
+# With S2_PARITY_REPORT=<path>, every comparison appends one JSON line (test, quantity,
+# measured error, bound) to that file: the margins of each parity case against its bound.
+_REPORT = os.environ.get("S2_PARITY_REPORT")
+
+
+def _record(what: str, kind: str, err: float, bound: float) -> None:
+    if not _REPORT:
+        return
+    test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0]
+    with open(_REPORT, "a") as f:
+        f.write(json.dumps({"test": test, "what": what, "kind": kind, "err": err,
+                            "bound": bound}) + "\n")
+
 
 # Tolerances. bf16 inputs with fp32 accumulation: max-abs 2e-2 on O, relative L2 1e-2 on
 # dq, dk, dv; LSE absolute 5e-3 (scores carry the bf16 rounding of the rotated q and k).
@@ -46,6 +63,7 @@ def max_abs(a, b) -> float:
 def assert_close_o(got, ref, dtype, what="o"):
     if dtype == "bf16":
         e = max_abs(got, ref)
+        _record(what, "max-abs", e, TOL_BF16_O_MAXABS)
         assert e <= TOL_BF16_O_MAXABS, "%s max-abs %.3e" % (what, e)
     else:
         assert_close_f32(got, ref, what)
@@ -54,6 +72,7 @@ def assert_close_o(got, ref, dtype, what="o"):
 def assert_close_grad(got, ref, dtype, what):
     if dtype == "bf16":
         e = rel_l2(got, ref)
+        _record(what, "rel-L2", e, TOL_BF16_GRAD_RELL2)
         assert e <= TOL_BF16_GRAD_RELL2, "%s rel-L2 %.3e" % (what, e)
     else:
         assert_close_f32(got, ref, what)
@@ -63,6 +82,8 @@ def assert_close_f32(got, ref, what):
     e = rel_l2(got, ref)
     m = max_abs(got, ref)
     bound = TOL_F32_REL * float(np.abs(ref).max())
+    _record(what, "rel-L2", e, TOL_F32_REL)
+    _record(what, "max-abs/max|ref|", m / max(float(np.abs(ref).max()), 1e-300), TOL_F32_REL)
     assert e <= TOL_F32_REL, "%s rel-L2 %.3e" % (what, e)
     assert m <= bound, "%s max-abs %.3e > %.3e" % (what, m, bound)
 
@@ -70,6 +91,7 @@ def assert_close_f32(got, ref, what):
 def assert_close_lse(got, ref, dtype, what="lse"):
     tol = TOL_BF16_LSE_ABS if dtype == "bf16" else TOL_F32_LSE_ABS
     e = max_abs(got, ref)
+    _record(what, "abs", e, tol)
     assert e <= tol, "%s abs %.3e" % (what, e)
 
 

@@ -35,7 +35,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(10):
+    for code in range(11):
         assert lib.s2attn_status_string(code) and lib.s2attn_status_string(code) != "unknown status"
     assert lib.s2attn_status_string(99) == "unknown status"
 

@@ -129,3 +129,32 @@ def test_autograd_backward_reports_a_forward_timeout(s2):
     o = s2.s2_attention(tq, tk, tv, w.G, w.pi_scale)
     o.backward(tdo)
     assert bool(torch.isfinite(tq.grad).all())
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_backward_after_forward_detects_another_forwards_workspace(s2, dtype):
+    """s2attn_bwd_after_fwd reuses the rotation the forward left in the workspace. A call
+    whose arguments or q/k buffers differ from that forward's is caught on the device and
+    reported as S2_ERR_STALE_WORKSPACE; the matching call still works afterwards."""
+    w = Workload("stale", 1, 1024, 4, 2, 128, 256, 2.0, dtype, 0.5, True, seed=24)
+    q, k, v, do = H.inputs(w)
+    tq, tk, tv, tdo = (H.to_device(x, dtype) for x in (q, k, v, do))
+    code = s2.S2_BF16 if dtype == "bf16" else s2.S2_FP32
+    ws = s2.workspace(w.B, w.N, w.Hq, w.Hkv, w.d, code, torch.device("cuda"))
+    o, lse = s2.forward(tq, tk, tv, w.G, w.pi_scale, ws=ws)
+    good = s2.backward(tq, tk, tv, o, lse, tdo, w.G, w.pi_scale, ws=ws, after_forward=True)
+    assert s2.device_status(ws) == s2.S2_OK
+    before = [_bits(t) for t in good]
+    scratch = tuple(torch.empty_like(t) for t in good)
+    # another PI scale than the forward's
+    s2.backward(tq, tk, tv, o, lse, tdo, w.G, 4.0, ws=ws, after_forward=True, grads=scratch)
+    assert s2.device_status(ws) == s2.S2_ERR_STALE_WORKSPACE
+    # another q buffer (same contents): the rotation in the workspace is not its rotation
+    s2.backward(tq.clone(), tk, tv, o, lse, tdo, w.G, w.pi_scale, ws=ws, after_forward=True,
+                grads=scratch)
+    assert s2.device_status(ws) == s2.S2_ERR_STALE_WORKSPACE
+    # the forward's own arguments still match, and give the same gradients bit for bit
+    again = s2.backward(tq, tk, tv, o, lse, tdo, w.G, w.pi_scale, ws=ws, after_forward=True)
+    assert s2.device_status(ws) == s2.S2_OK
+    for a, b in zip(before, (_bits(t) for t in again)):
+        assert torch.equal(a, b)
