@@ -88,8 +88,8 @@ def _kernel_work(name, w, es):
         return "hbm", 2.0 * w.B * w.N * (w.Hq + w.Hkv) * w.d * es + w.N * w.d * 4, "GB/s"
     elif name == "rope_table":    # write the cos/sin table
         return "hbm", w.N * w.d * 4.0, "GB/s"
-    elif name == "bwd_rowsum":
-        return "hbm", 2.0 * w.B * w.N * w.Hq * w.d * es + 4.0 * w.B * w.Hq * w.N, "GB/s"
+    elif name == "bwd_rowsum":    # read dO, O, LSE; write D and the 32-byte row terms
+        return "hbm", 2.0 * w.B * w.N * w.Hq * w.d * es + 40.0 * w.B * w.Hq * w.N, "GB/s"
     else:
         return None, 0.0, None
     return ("tensor" if name.endswith("_tc") else "alu"), work, "TFLOP/s"
