@@ -109,6 +109,15 @@ __device__ __forceinline__ uint64_t opaque64(uint64_t v) {
 #define S2_DQ_POLY_MASK 0x0ull
 #endif
 constexpr unsigned long long kDqPolyMask = S2_DQ_POLY_MASK;
+// The dK/dV pass: bit t set sends the exponentials of column pair t (columns 2t, 2t+1 of a
+// math warp's 64) to the packed FMA-pipe polynomial, off the diagonal tiles. On a B200, 32k
+// workload, 1/8, 1/4 and 1/2 of them there gave 3.52 / 3.62 / 3.68 ms against 3.59-3.68 ms
+// with none (within run-to-run noise): the pass is not bound by the MUFU, so the default
+// is none.
+#ifndef S2_DKDV_POLY_MASK
+#define S2_DKDV_POLY_MASK 0x0u
+#endif
+constexpr unsigned kDkdvPolyMask = S2_DKDV_POLY_MASK;
 template <unsigned long long kMask>
 __device__ __forceinline__ float exp2_mixed(float x, int c) {
   return ((kMask >> c) & 1ull) ? exp2_poly(x) : fast_exp2(x);
@@ -479,13 +488,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tST, x0);
         tmem_ld32(tST + 32, x1);
         tmem_wait_ld();
-        if (diag) mask_scores(x0, x1, row - c0, 0);  // query row c0+c before key row: P = 0
+        if (diag) {
+          mask_scores(x0, x1, row - c0, 0);  // query row c0+c before key row: P = 0
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          float a0, a1;
-          f2unpack(fmul2(score_pair(x0, x1, c), sl2x2), a0, a1);
-          pr[c] = fast_exp2(a0);
-          pr[c + 1] = fast_exp2(a1);
+          for (int c = 0; c < 64; c += 2) {
+            float a0, a1;
+            f2unpack(fmul2(score_pair(x0, x1, c), sl2x2), a0, a1);
+            pr[c] = fast_exp2(a0);
+            pr[c + 1] = fast_exp2(a1);
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 64; c += 2) {
+            const uint64_t a = fmul2(score_pair(x0, x1, c), sl2x2);
+            if ((kDkdvPolyMask >> (c >> 1)) & 1u) {
+              f2unpack(exp2_poly2(a), pr[c], pr[c + 1]);
+            } else {
+              float a0, a1;
+              f2unpack(a, a0, a1);
+              pr[c] = fast_exp2(a0);
+              pr[c + 1] = fast_exp2(a1);
+            }
+          }
         }
         uint32_t pp[32];
 #pragma unroll

@@ -67,11 +67,12 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
 
 // Column pairs (bit c2 of a 16-bit mask, per 32-column chunk) whose exponentials go to the
-// FMA-pipe exp2 instead of the MUFU unit. At d = 128 the MUFU needs as many cycles per key
-// tile as the tensor cores, but with two softmax warps per scheduler the softmax is bound
-// by instruction latency, not by the MUFU: on a B200 moving 25% / 37.5% / 50% of the
-// exponentials to the FMA pipe slowed the 32k forward from 2.32 ms to 2.52 / 2.84 / 3.10 ms.
-// So every exponential stays on the MUFU unless a build overrides this mask.
+// FMA-pipe exp2 (packed pairs) instead of the MUFU unit. At d = 128 the MUFU needs as many
+// cycles per key tile as the tensor cores. On a B200 moving 25% / 37.5% / 50% of the
+// exponentials to the scalar form of the polynomial slowed the 32k forward from 2.32 ms to
+// 2.52 / 2.84 / 3.10 ms; with the packed form, 12.5% / 25% / 31% gave 2.08 / 2.09 / 2.14 ms
+// against 2.04-2.05 ms with none. So every exponential stays on the MUFU unless a build
+// overrides this mask.
 #ifndef S2_FWD_POLY_MASK
 #define S2_FWD_POLY_MASK 0x0000u
 #endif
@@ -136,13 +137,13 @@ __device__ __forceinline__ float write_p64(const uint32_t (&x0)[32], const uint3
     for (int c2 = 0; c2 < 16; c2++) {
       const float s0 = __uint_as_float(ch ? x1[2 * c2] : x0[2 * c2]);
       const float s1 = __uint_as_float(ch ? x1[2 * c2 + 1] : x0[2 * c2 + 1]);
-      float a0, a1;
-      f2unpack(ffma2(f2pack(s0, s1), sl2x2, nmx2), a0, a1);
+      const uint64_t a = ffma2(f2pack(s0, s1), sl2x2, nmx2);
       float p0, p1;
       if ((kPolyMask >> c2) & 1u) {
-        p0 = exp2_poly(a0);
-        p1 = exp2_poly(a1);
+        f2unpack(exp2_poly2(a), p0, p1);
       } else {
+        float a0, a1;
+        f2unpack(a, a0, a1);
         p0 = fast_exp2(a0);
         p1 = fast_exp2(a1);
       }
