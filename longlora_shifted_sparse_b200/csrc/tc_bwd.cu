@@ -395,7 +395,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the issue loop (warp-uniform control flow and descriptors); one
+    // elected lane issues each MMA and commit.
+    {
       const uint32_t idesc_s = idesc_bf16_f32(kTile, kTile, false, false);
       const uint32_t idesc_g = idesc_bf16_f32(kTile, kD, false, true);
       const uint64_t dKT = smem_desc_sw32(smem_addr(smem + kKVOffKTerm));
@@ -404,63 +406,64 @@ __global__ void __launch_bounds__(kThreads, 1)
       // S^T(n) - LSE*sqrt(d) = K Q_n^T + 1 (row terms)^T: eight k-steps and the row-term step
       auto issue_st = [&](int n) -> bool {
         const int sq = n % kQStages;
-        if (!mbar_wait(smem_addr(&bars.q_full[sq]), (n / kQStages) & 1, ab)) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.q_full[sq]), (n / kQStages) & 1, ab)))
+          return false;
         tc_fence_after();
         const uint32_t sQ = stage_q(n);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; kk++)
-          mma_ss(tmem + colST, kmajor_desc(sK, kk), kmajor_desc(sQ, kk), idesc_s, kk > 0);
-        mma_ss(tmem + colST, dKT, smem_desc_sw32(sQ + kTileBytes), idesc_s, 1u);
+          mma_ss_elect(tmem + colST, kmajor_desc(sK, kk), kmajor_desc(sQ, kk), idesc_s, kk > 0);
+        mma_ss_elect(tmem + colST, dKT, smem_desc_sw32(sQ + kTileBytes), idesc_s, 1u);
         // failure-path self-test: CTA 0 (key tile 0, at least two pairs) withholds the
         // arrival of S^T(1), so that the math warps and then this thread wait in vain
         if (!(p.inject == kInjectDkdv && blockIdx.x == 0 && n == 1))
-          mma_commit(smem_addr(&bars.st_full));
+          mma_commit_elect(smem_addr(&bars.st_full));
         return true;
       };
       // dP^T(n) - D = V dO_n^T + 1 (row terms)^T (the row terms sit in Q stage n)
       auto issue_dpt = [&](int n) -> bool {
-        if (!mbar_wait(smem_addr(&bars.do_full), n & 1, ab)) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.do_full), n & 1, ab))) return false;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kD / 16; kk++)
-          mma_ss(tmem + colDPT, kmajor_desc(sV, kk), kmajor_desc(sDO, kk), idesc_s, kk > 0);
-        mma_ss(tmem + colDPT, dVT, smem_desc_sw32(stage_q(n) + kTileBytes), idesc_s, 1u);
-        mma_commit(smem_addr(&bars.dpt_full));
+          mma_ss_elect(tmem + colDPT, kmajor_desc(sV, kk), kmajor_desc(sDO, kk), idesc_s, kk > 0);
+        mma_ss_elect(tmem + colDPT, dVT, smem_desc_sw32(stage_q(n) + kTileBytes), idesc_s, 1u);
+        mma_commit_elect(smem_addr(&bars.dpt_full));
         return true;
       };
       // Per pair n: dV(n) once the math warps have written P^T(n) over S^T(n), then S^T(n+1)
       // over it (the MMAs run in issue order); dK(n) once they have written dS^T(n) over
       // dP^T(n), then dP^T(n+1) over it. The math warps' exponentials of pair n+1 then run
       // while dK(n) and dP^T(n+1) occupy the tensor cores.
-      bool ok = mbar_wait(smem_addr(&bars.kv_full), 0, ab);
+      bool ok = __all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.kv_full), 0, ab));
       tc_fence_after();
       if (ok && np > 0) ok = issue_st(0) && issue_dpt(0);
-      if (ok && np == 1) mma_commit(smem_addr(&bars.kv_free));
+      if (ok && np == 1) mma_commit_elect(smem_addr(&bars.kv_free));
       for (int n = 0; ok && n < np; n++) {
         const uint32_t ph = n & 1;
-        if (!mbar_wait(smem_addr(&bars.p_ready), ph, ab)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.p_ready), ph, ab))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; kk++)
-          mma_ts(tmem + colDV, tmem + colST + (kk >> 2) * 64 + (kk & 3) * 8, mn_desc(sDO, kk),
+          mma_ts_elect(tmem + colDV, tmem + colST + (kk >> 2) * 64 + (kk & 3) * 8, mn_desc(sDO, kk),
                  idesc_g, (n > 0 || kk > 0));
-        mma_commit(smem_addr(&bars.do_empty));
+        mma_commit_elect(smem_addr(&bars.do_empty));
         if (n + 1 < np && !issue_st(n + 1)) break;
-        if (!mbar_wait(smem_addr(&bars.ds_ready), ph, ab)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.ds_ready), ph, ab))) break;
         tc_fence_after();
         const uint32_t sQ = stage_q(n);
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; kk++)
-          mma_ts(tmem + colDK, tmem + colDPT + (kk >> 2) * 64 + (kk & 3) * 8, mn_desc(sQ, kk),
+          mma_ts_elect(tmem + colDK, tmem + colDPT + (kk >> 2) * 64 + (kk & 3) * 8, mn_desc(sQ, kk),
                  idesc_g, (n > 0 || kk > 0));
-        mma_commit(smem_addr(&bars.q_empty[n % kQStages]));
+        mma_commit_elect(smem_addr(&bars.q_empty[n % kQStages]));
         if (n + 1 < np) {
           if (!issue_dpt(n + 1)) break;
-          if (n + 2 == np) mma_commit(smem_addr(&bars.kv_free));  // the last reader of K, V
+          if (n + 2 == np) mma_commit_elect(smem_addr(&bars.kv_free));  // the last reader of K, V
         }
       }
-      mma_commit(smem_addr(&bars.acc_done));
-      mma_commit(smem_addr(&bars.drain));
+      mma_commit_elect(smem_addr(&bars.acc_done));
+      mma_commit_elect(smem_addr(&bars.drain));
       mbar_wait_drain(smem_addr(&bars.drain), 0, p.status, p.wait_limit_ns);
     }
   } else if (warp >= 4) {

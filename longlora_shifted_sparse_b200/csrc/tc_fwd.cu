@@ -326,8 +326,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         p.wait_limit_ns);
       if (q_last >= 0)
         mbar_wait_drain(smem_addr(&bars.q_full), q_last & 1, p.status, p.wait_limit_ns);
-    } else if (warp == 1 && lane == 0) {
+    } else if (warp == 1) {
       // ------------------------------------------------------------------ MMA issuer
+      // The whole warp runs the issue loop (warp-uniform control flow and descriptors);
+      // one elected lane issues each MMA and commit.
       const uint32_t idesc_qk = idesc_bf16_f32(kTile, kTile, false, false);
       const uint32_t idesc_pv = idesc_bf16_f32(kTile, kD, false, true);
       // Descriptors are built once; a k-step or a stage only adds a constant to the start
@@ -342,18 +344,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pcnt[2] = {0u, 0u};       // p_full phases consumed per query tile
       bool ok = true;
       for (int k = 0; ok; k++) {
-        if (!mbar_wait(smem_addr(&bars.q_full), k & 1, ab)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.q_full), k & 1, ab))) break;
         const int item = item_slot[k & 1];
         if (item < 0) break;
         const FwdItem it = decode_item(p, item);
         tc_fence_after();
         for (int j = 0; j <= it.nB; j++) {
           const int gj = kv + j, gjj = gj - 1;   // ring positions of key tiles j and j - 1
-          if (j >= 1 && !mbar_wait(smem_addr(&bars.v_full[gjj & 1]), (gjj >> 1) & 1, ab)) {
+          if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.v_full[gjj & 1]),
+                                                             (gjj >> 1) & 1, ab))) {
             ok = false;
             break;
           }
-          if (j < it.nB && !mbar_wait(smem_addr(&bars.k_full[gj & 1]), (gj >> 1) & 1, ab)) {
+          if (j < it.nB && !__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.k_full[gj & 1]),
+                                                              (gj >> 1) & 1, ab))) {
             ok = false;
             break;
           }
@@ -368,40 +372,45 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nt = t ? it.nB : it.nA;
             const uint32_t tS = tmem + t * 128, tO = tmem + 256 + t * 128;
             if (j >= 1 && j - 1 < nt) {
-              if (!mbar_wait(smem_addr(&bars.p_full[t]), pcnt[t] & 1, ab)) { ok = false; break; }
+              if (!__all_sync(0xffffffffu,
+                              mbar_wait(smem_addr(&bars.p_full[t]), pcnt[t] & 1, ab))) {
+                ok = false;
+                break;
+              }
               pcnt[t]++;
               tc_fence_after();
               const uint32_t acc0 = j > 1;
 #pragma unroll
               for (int kk = 0; kk < kTile / 16; kk++)  // P of key rows 64h.. at column 64h;
-                mma_ts(tO, tS + (kk >> 2) * 64 + (kk & 3) * 8,  // V k-step = 16 rows
+                mma_ts_elect(tO, tS + (kk >> 2) * 64 + (kk & 3) * 8,  // V k-step = 16 rows
                        dVj + (uint64_t)(kk * (2048 >> 4)), idesc_pv, kk ? 1u : acc0);
-              if (j == nt) mma_commit(smem_addr(&bars.o_final[t]));
+              if (j == nt) mma_commit_elect(smem_addr(&bars.o_final[t]));
             }
             if (j < nt) {
               const uint64_t dQt = dQj + (uint64_t)(t * kTileDesc);
 #pragma unroll
               for (int kk = 0; kk < kD / 16; kk++) {
                 const uint64_t koff = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
-                mma_ss(tS, dQt + koff, dKj + koff, idesc_qk, kk > 0);
+                mma_ss_elect(tS, dQt + koff, dKj + koff, idesc_qk, kk > 0);
               }
               // failure-path self-test: CTA 0 withholds the arrival of score tile B at key
               // tile 1 of its first item (every item's tile B has at least two key tiles), so
               // that tile's softmax warps and then this thread wait in vain until the limit
               if (!(p.inject == kInjectFwd && blockIdx.x == 0 && k == 0 && t == 1 && j == 1))
-                mma_commit(smem_addr(&bars.s_full[t]));
+                mma_commit_elect(smem_addr(&bars.s_full[t]));
             }
           }
           if (!ok) break;
-          if (j == it.nB - 1) mma_commit(smem_addr(&bars.q_empty));  // last QK^T of the item
-          if (j >= 1) mma_commit(smem_addr(&bars.v_empty[gjj & 1]));
-          if (j < it.nB) mma_commit(smem_addr(&bars.k_empty[gj & 1]));
+          if (j == it.nB - 1) mma_commit_elect(smem_addr(&bars.q_empty));  // last QK^T of the item
+          if (j >= 1) mma_commit_elect(smem_addr(&bars.v_empty[gjj & 1]));
+          if (j < it.nB) mma_commit_elect(smem_addr(&bars.k_empty[gj & 1]));
         }
         kv += it.nB;
       }
       // every MMA issued above has completed before TMEM is released
-      mma_commit(smem_addr(&bars.drain));
+      mma_commit_elect(smem_addr(&bars.drain));
       mbar_wait_drain(smem_addr(&bars.drain), 0, p.status, p.wait_limit_ns);
+      __syncwarp();
     }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
