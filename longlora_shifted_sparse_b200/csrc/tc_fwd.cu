@@ -351,16 +351,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int j = 0; j <= it.nB; j++) {
           const int gj = kv + j, gjj = gj - 1;   // ring positions of key tiles j and j - 1
+          // V_{j-1} before the first PV, K_j only before the first QK^T: a PV never waits
+          // for the key tile that follows it
           if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.v_full[gjj & 1]),
                                                              (gjj >> 1) & 1, ab))) {
             ok = false;
             break;
           }
-          if (j < it.nB && !__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.k_full[gj & 1]),
-                                                              (gj >> 1) & 1, ab))) {
-            ok = false;
-            break;
-          }
+          bool k_ready = false;
           tc_fence_after();
           // opaque per-iteration bases: the per-k-step descriptors are formed by one add at
           // their MMA instead of being hoisted out of the loop into (spilled) registers
@@ -386,7 +384,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                        dVj + (uint64_t)(kk * (2048 >> 4)), idesc_pv, kk ? 1u : acc0);
               if (j == nt) mma_commit_elect(smem_addr(&bars.o_final[t]));
             }
+            // V_{j-1} is free once the last PV that reads it has been issued (tile B's)
+            if (t == 1 && j >= 1) mma_commit_elect(smem_addr(&bars.v_empty[gjj & 1]));
             if (j < nt) {
+              if (!k_ready) {
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.k_full[gj & 1]),
+                                                       (gj >> 1) & 1, ab))) {
+                  ok = false;
+                  break;
+                }
+                k_ready = true;
+                tc_fence_after();
+              }
               const uint64_t dQt = dQj + (uint64_t)(t * kTileDesc);
 #pragma unroll
               for (int kk = 0; kk < kD / 16; kk++) {
@@ -402,7 +411,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (!ok) break;
           if (j == it.nB - 1) mma_commit_elect(smem_addr(&bars.q_empty));  // last QK^T of the item
-          if (j >= 1) mma_commit_elect(smem_addr(&bars.v_empty[gjj & 1]));
           if (j < it.nB) mma_commit_elect(smem_addr(&bars.k_empty[gj & 1]));
         }
         kv += it.nB;

@@ -64,6 +64,11 @@ SMALL = [
     ("f32_d128_g96", 1, 384, 4, 2, 128, 96, 3.0, "f32", True),
     ("f32_d256_noncausal", 1, 128, 2, 2, 256, 32, 1.0, "f32", False),
     ("f32_g2_minimal", 1, 8, 2, 2, 32, 2, 1.0, "f32", True),
+    # head dims of 3, 5, 6 and 7 elements per lane on the CUDA-core kernels
+    ("bf16_d96_gqa", 1, 384, 4, 2, 96, 128, 2.0, "bf16", True),
+    ("f32_d160_noncausal", 1, 256, 2, 2, 160, 64, 1.5, "f32", False),
+    ("bf16_d192", 1, 256, 2, 2, 192, 64, 3.0, "bf16", True),
+    ("f32_d224_b2", 2, 128, 2, 2, 224, 32, 1.0, "f32", True),
 ]
 
 
