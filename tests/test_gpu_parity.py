@@ -25,13 +25,16 @@ def s2():
 
 
 def _run(s2, w, q, k, v, do):
+    """Forward (and backward) through the library; every call's device status is checked, so
+    an expired wait shows up as such rather than as wrong numbers."""
     tq, tk, tv = (H.to_device(x, w.dtype) for x in (q, k, v))
-    o, lse = s2.forward(tq, tk, tv, w.G, w.pi_scale, w.rope_base, w.causal, shift=w.shift)
+    o, lse = s2.forward(tq, tk, tv, w.G, w.pi_scale, w.rope_base, w.causal, shift=w.shift,
+                        check_status=True)
     grads = None
     if do is not None:
         tdo = H.to_device(do, w.dtype)
         grads = s2.backward(tq, tk, tv, o, lse, tdo, w.G, w.pi_scale, w.rope_base, w.causal,
-                            shift=w.shift)
+                            shift=w.shift, check_status=True)
     torch.cuda.synchronize()
     return o, lse, grads
 
@@ -64,6 +67,9 @@ SMALL = [
     ("f32_d128_g96", 1, 384, 4, 2, 128, 96, 3.0, "f32", True),
     ("f32_d256_noncausal", 1, 128, 2, 2, 256, 32, 1.0, "f32", False),
     ("f32_g2_minimal", 1, 8, 2, 2, 32, 2, 1.0, "f32", True),
+    # several work items per CTA in the persistent kernels (forward 256 items, dQ 512, on
+    # 148 CTAs), compared in full: the item-to-item hand-over of their rings
+    ("bf16_multi_item_gqa", 1, 8192, 8, 4, 128, 1024, 2.0, "bf16", True),
     # head dims of 3, 5, 6 and 7 elements per lane on the CUDA-core kernels
     ("bf16_d96_gqa", 1, 384, 4, 2, 96, 128, 2.0, "bf16", True),
     ("f32_d160_noncausal", 1, 256, 2, 2, 160, 64, 1.5, "f32", False),
