@@ -118,67 +118,77 @@ __global__ void __launch_bounds__(256) bwd_rowsum_kernel(Params p) {
 }
 
 // D = rowsum(dO * O) for bf16 rows of 128 (the tensor-core path's shape), HBM-bound, plus
-// the row terms of the tensor-core dK/dV pass. Rows are taken in [B][Hq][N] order, 8
-// consecutive tokens of one head per warp (a half-warp per row, 16 bytes per lane, all 8
-// loads of dO and O issued before the first use), so that the LSE reads and the D and
-// row-term writes of a warp are contiguous; each dO / O row is 256 contiguous bytes.
+// the row terms of the tensor-core dK/dV pass. A CTA takes kRowsumTokens consecutive tokens
+// of one batch entry with all their heads: those dO and O rows are contiguous in memory and
+// are read front to back (a half-warp per 256-byte row, 16 bytes per lane, four rows of each
+// tensor in flight per half-warp); the row sums go through shared memory and are written
+// head by head, so that the LSE reads and the D and row-term writes are contiguous too.
+constexpr int kRowsumTokens = 16;
+
+__device__ inline void write_row_terms(const Params& p, size_t row, float D) {
+  // -LSE*sqrt(d) and -D as sums of bf16 parts (each part the rounding of what the previous
+  // ones left), exact to ~2^-24 and ~2^-16 relative
+  const float nl = -p.lse[row] / p.scale;
+  const __nv_bfloat16 l0 = __float2bfloat16_rn(nl);
+  const float r1 = nl - __bfloat162float(l0);
+  const __nv_bfloat16 l1 = __float2bfloat16_rn(r1);
+  const __nv_bfloat16 l2 = __float2bfloat16_rn(r1 - __bfloat162float(l1));
+  const __nv_bfloat16 d0 = __float2bfloat16_rn(-D);
+  const __nv_bfloat16 d1 = __float2bfloat16_rn(-D - __bfloat162float(d0));
+  const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
+  __nv_bfloat162 w[4] = {__halves2bfloat162(l0, l1), __halves2bfloat162(l2, d0),
+                         __halves2bfloat162(d1, z), __halves2bfloat162(z, z)};
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.rowterms) + row * 16);
+  dst[0] = *reinterpret_cast<const uint4*>(w);
+  dst[1] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 __global__ void __launch_bounds__(256) bwd_rowsum_bf16_d128_kernel(Params p) {
-  constexpr int kRowsPerWarp = 8;
-  const int lane = threadIdx.x & 31, half = lane >> 4, chunk = lane & 15;
-  const long warp = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  extern __shared__ float dsh[];  // [kRowsumTokens][Hq]
+  const int chunk = threadIdx.x & 15;                          // 16-byte piece of a row
+  const int hw = threadIdx.x >> 4, nhw = blockDim.x >> 4;  // half-warp id and count
   if (blockIdx.x == 0 && threadIdx.x == 0) backward_status_reset(p);
-  const long rows = (long)p.B * p.N * p.Hq;
-  const long r0 = warp * kRowsPerWarp;
-  if (r0 >= rows) return;
-  const uint4* dO = reinterpret_cast<const uint4*>(p.dout);
-  const uint4* O = reinterpret_cast<const uint4*>(p.o);
-  uint4 a[kRowsPerWarp / 2], c[kRowsPerWarp / 2];
+  const int blocks_per_b = (p.N + kRowsumTokens - 1) / kRowsumTokens;
+  const int b = blockIdx.x / blocks_per_b;
+  const int m0 = (blockIdx.x - b * blocks_per_b) * kRowsumTokens;
+  const int ntok = min(kRowsumTokens, p.N - m0);
+  const int nrows = ntok * p.Hq;  // rows (token, head) of this CTA, contiguous in dO and O
+  const uint4* dO = reinterpret_cast<const uint4*>(p.dout) + ((size_t)b * p.N + m0) * p.Hq * 16;
+  const uint4* O = reinterpret_cast<const uint4*>(p.o) + ((size_t)b * p.N + m0) * p.Hq * 16;
+  for (int r0 = hw; r0 < nrows; r0 += 4 * nhw) {
+    uint4 a[4], c[4];
 #pragma unroll
-  for (int i = 0; i < kRowsPerWarp / 2; i++) {
-    const long r = r0 + 2 * i + half;  // row (b, h, m) in [B][Hq][N] order
-    long e = 0;
-    if (r < rows) {
-      const int m = (int)(r % p.N);
-      const long bh = r / p.N;
-      const int h = (int)(bh % p.Hq), b = (int)(bh / p.Hq);
-      e = (((long)b * p.N + m) * p.Hq + h) * 16 + chunk;  // 16 uint4 per row
+    for (int i = 0; i < 4; i++) {
+      const int r = r0 + i * nhw;
+      const size_t e = r < nrows ? (size_t)r * 16 + chunk : 0;
+      a[i] = __ldcs(dO + e);
+      c[i] = __ldcs(O + e);
     }
-    a[i] = __ldcs(dO + e);
-    c[i] = __ldcs(O + e);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+      const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a[i]);
+      const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&c[i]);
+      float acc = 0.f;
+#pragma unroll
+      for (int t = 0; t < 4; t++) {
+        const float2 xf = __bfloat1622float2(x[t]), yf = __bfloat1622float2(y[t]);
+        acc = fmaf(xf.x, yf.x, acc);
+        acc = fmaf(xf.y, yf.y, acc);
+      }
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      const int r = r0 + i * nhw;
+      if (chunk == 0 && r < nrows) dsh[r] = acc;  // [token][head]
+    }
   }
-#pragma unroll
-  for (int i = 0; i < kRowsPerWarp / 2; i++) {
-    const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&a[i]);
-    const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&c[i]);
-    float acc = 0.f;
-#pragma unroll
-    for (int t = 0; t < 4; t++) {
-      const float2 xf = __bfloat1622float2(x[t]), yf = __bfloat1622float2(y[t]);
-      acc = fmaf(xf.x, yf.x, acc);
-      acc = fmaf(xf.y, yf.y, acc);
-    }
-#pragma unroll
-    for (int o = 8; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    const long r = r0 + 2 * i + half;
-    if (chunk == 0 && r < rows) {
-      p.Dsum[r] = acc;
-      // the row terms of the tensor-core dK/dV pass: -LSE*sqrt(d) and -D as sums of bf16
-      // parts (each part the rounding of what the previous ones left), exact to ~2^-24 and
-      // ~2^-16 relative
-      const float nl = -p.lse[r] / p.scale;
-      const __nv_bfloat16 l0 = __float2bfloat16_rn(nl);
-      const float r1 = nl - __bfloat162float(l0);
-      const __nv_bfloat16 l1 = __float2bfloat16_rn(r1);
-      const __nv_bfloat16 l2 = __float2bfloat16_rn(r1 - __bfloat162float(l1));
-      const __nv_bfloat16 d0 = __float2bfloat16_rn(-acc);
-      const __nv_bfloat16 d1 = __float2bfloat16_rn(-acc - __bfloat162float(d0));
-      const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
-      __nv_bfloat162 w[4] = {__halves2bfloat162(l0, l1), __halves2bfloat162(l2, d0),
-                             __halves2bfloat162(d1, z), __halves2bfloat162(z, z)};
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.rowterms) + r * 16);
-      dst[0] = *reinterpret_cast<const uint4*>(w);
-      dst[1] = make_uint4(0u, 0u, 0u, 0u);
-    }
+  __syncthreads();
+  // head by head: consecutive threads take consecutive tokens of one head
+  for (int e = threadIdx.x; e < nrows; e += blockDim.x) {
+    const int h = e / ntok, t = e - h * ntok;
+    const size_t row = ((size_t)b * p.Hq + h) * p.N + m0 + t;
+    const float D = dsh[t * p.Hq + h];
+    p.Dsum[row] = D;
+    write_row_terms(p, row, D);
   }
 }
 
@@ -319,8 +329,14 @@ cudaError_t launch_simt_fwd(const Params& p, bool bf16, cudaStream_t st) {
 
 cudaError_t launch_bwd_rowsum(const Params& p, bool bf16, cudaStream_t st) {
   if (bf16 && p.d == 128) {
-    const long warps = ((long)p.B * p.Hq * p.N + 7) / 8;
-    bwd_rowsum_bf16_d128_kernel<<<(unsigned)((warps + 7) / 8), 256, 0, st>>>(p);
+    const long blocks = (long)p.B * ((p.N + kRowsumTokens - 1) / kRowsumTokens);
+    const size_t smem = (size_t)kRowsumTokens * p.Hq * sizeof(float);
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(bwd_rowsum_bf16_d128_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    bwd_rowsum_bf16_d128_kernel<<<(unsigned)blocks, 256, smem, st>>>(p);
     return cudaGetLastError();
   }
   dim3 grid = warp_grid((long)p.B * p.Hq * p.N);
