@@ -85,13 +85,15 @@ __host__ __device__ inline bool q_head_shifted(int h, const Params& p) {
 
 // Work order of the tensor-core kernels: CTA x of a grid of U units (b, kv head, group)
 // times W items per unit -> (unit, item), item 0 being a unit's heaviest item. Units are
-// taken kLptChunk at a time; inside a chunk the items run heaviest first across all of the
-// chunk's units. The last wave then holds only light items (longest-processing-time order,
-// a short tail), while the few units in flight keep the tiles they share resident in L2.
+// taken `chunk` at a time (kLptChunk unless the kernel sizes it); inside a chunk the items
+// run heaviest first across all of the chunk's units. The last wave then holds only light
+// items (longest-processing-time order, a short tail), while the few units in flight keep the
+// tiles they share resident in L2.
 constexpr int kLptChunk = 8;
-__device__ inline void chunked_lpt(int x, int U, int W, int& unit, int& item) {
-  const int c0 = x / (kLptChunk * W) * kLptChunk;
-  const int cc = min(kLptChunk, U - c0);
+__device__ inline void chunked_lpt(int x, int U, int W, int& unit, int& item,
+                                   int chunk = kLptChunk) {
+  const int c0 = x / (chunk * W) * chunk;
+  const int cc = min(chunk, U - c0);
   const int r = x - c0 * W;
   item = r / cc;
   unit = c0 + (r - item * cc);

@@ -14,14 +14,14 @@ using namespace sm100;
 
 __global__ void __launch_bounds__(32, 1) wait_timeout_kernel(unsigned* status, uint64_t limit_ns) {
   __shared__ uint64_t bar;
-  __shared__ int abort_flag;
+  __shared__ AbortState abort_state;
   if (threadIdx.x == 0) {
-    abort_flag = 0;
+    abort_state_init(abort_state, status, limit_ns, 0);
     mbar_init(smem_addr(&bar), 1);
     fence_barrier_init();
   }
   __syncthreads();
-  Abort ab{&abort_flag, status, limit_ns};
+  const Abort ab{smem_addr(&abort_state)};
   mbar_wait(smem_addr(&bar), 0, ab);  // nothing arrives: expires by design
 }
 

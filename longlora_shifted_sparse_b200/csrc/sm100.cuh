@@ -71,16 +71,34 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // clock are checked every 16 try-waits.
 constexpr uint32_t kWaitSleepNs = 20000u;
 
-// Shared abort state of one CTA: a flag in shared memory, the call's global status word and
+// Abort state of one CTA, in its shared memory: a flag, the call's global status word and
 // the time limit of one wait. Every wait in the tcgen05 kernels is bounded by that limit; on
 // expiry the waiter records the timeout in the status word, raises the CTA's abort flag and
 // returns false. Every other wait of the CTA, and of every other CTA of the launch (they
-// poll the status word), then gives up at its next check.
-struct Abort {
-  volatile int* flag;   // shared memory
+// poll the status word), then gives up at its next check. Thread 0 fills it in before the
+// CTA's first barrier.
+struct AbortState {
+  volatile int flag;
   unsigned* status;     // global memory (workspace)
   uint64_t limit_ns;
 };
+
+// What a wait is handed: the shared-memory address of the CTA's AbortState. One register,
+// where the state itself would keep six live through a whole issue loop; the waits read the
+// fields only on their slow path.
+struct Abort {
+  uint32_t state;
+  __device__ AbortState& get() const {
+    return *static_cast<AbortState*>(__cvta_shared_to_generic(state));
+  }
+};
+
+__device__ __forceinline__ void abort_state_init(AbortState& a, unsigned* status,
+                                                 uint64_t limit_ns, int flag) {
+  a.flag = flag;
+  a.status = status;
+  a.limit_ns = limit_ns;
+}
 
 // kRegion gives each register budget of a kernel that splits its registers (setmaxnreg) its
 // own copy of the out-of-line slow path: a function called from two budgets cannot be
@@ -88,17 +106,18 @@ struct Abort {
 template <int kRegion = 0>
 static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity, Abort ab) {
   const uint64_t t0 = global_timer_ns();
+  AbortState& st = ab.get();
   for (uint32_t i = 0;; ++i) {
     if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
     if ((i & 15u) == 15u) {
-      if (*ab.flag) return false;
-      if (*reinterpret_cast<volatile unsigned*>(ab.status) != 0u) {  // another CTA gave up
-        *ab.flag = 1;
+      if (st.flag) return false;
+      if (*reinterpret_cast<volatile unsigned*>(st.status) != 0u) {  // another CTA gave up
+        st.flag = 1;
         return false;
       }
-      if (global_timer_ns() - t0 > ab.limit_ns) {
-        atomicOr(ab.status, 1u);
-        *ab.flag = 1;
+      if (global_timer_ns() - t0 > st.limit_ns) {
+        atomicOr(st.status, 1u);
+        st.flag = 1;
         __threadfence_block();
         return false;
       }

@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   __shared__ DkdvBarriers bars;
   __shared__ uint32_t tmem_base_sh;
-  __shared__ int abort_flag;
+  __shared__ AbortState abort_state;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = p.G / kTile, ng = p.N / p.G, R = p.Hq / p.Hkv;
@@ -251,9 +251,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async_shared();
   }
-  Abort ab{&abort_flag, p.status, p.wait_limit_ns};
+  const Abort ab{smem_addr(&abort_state)};
   if (threadIdx.x == 0) {
-    abort_flag = *reinterpret_cast<volatile unsigned*>(p.status) != 0u;
+    abort_state_init(abort_state, p.status, p.wait_limit_ns,
+                     *reinterpret_cast<volatile unsigned*>(p.status) != 0u);
     mbar_init(smem_addr(&bars.kv_full), 1);
     mbar_init(smem_addr(&bars.cs_full), 1);
     for (int s = 0; s < kQStages; s++) {
@@ -279,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t colST = 0, colDPT = 128, colDV = 256, colDK = 384;
   const uint32_t sK = smem_addr(smem + kKVOffK), sV = smem_addr(smem + kKVOffV);
   const uint32_t sDO = smem_addr(smem + kKVOffDO);
-  const bool skip = abort_flag != 0;
+  const bool skip = abort_state.flag != 0;
 
   // Pairs run query tile it0 .. T-1 of query head kvh*R, then of the next head, and so on.
   // Each role walks them with a cursor (no division by nq: an integer division uses the
@@ -693,15 +694,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   __shared__ DqBarriers bars;
   __shared__ uint32_t tmem_base_sh;
-  __shared__ int abort_flag;
+  __shared__ AbortState abort_state;
   __shared__ int item_slot[2];  // the CTA's k-th item in slot k & 1 (-1: no more work)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned* const next_item = p.status + kDqWorkCounter;
 
-  Abort ab{&abort_flag, p.status, p.wait_limit_ns};
+  const Abort ab{smem_addr(&abort_state)};
   if (threadIdx.x == 0) {
-    abort_flag = 0;
+    abort_state_init(abort_state, p.status, p.wait_limit_ns, 0);
     mbar_init(smem_addr(&bars.q_full), 1);
     mbar_init(smem_addr(&bars.q_empty), kDqQEmptyArrivals);
     for (int s = 0; s < kKStages; s++) {

@@ -63,6 +63,7 @@ constexpr int kRegsOther = 64, kRegsSoftmax = 104;
 static_assert(128 * kRegsOther + (kThreads - 128) * kRegsSoftmax <= kThreads * 96,
               "register split exceeds the launch allocation");
 constexpr int kSoftmaxThreadsPerTile = 256;
+constexpr int kSoftmaxWarps = 2 * kSoftmaxThreadsPerTile / 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
 
@@ -85,7 +86,7 @@ constexpr uint32_t kOffV = 4 * kTileBytes;
 constexpr uint32_t kSmemBytes = 6 * kTileBytes + 1024;
 
 struct FwdBarriers {
-  uint64_t q_full, q_empty;
+  uint64_t q_full[2], q_empty[2];                 // per query tile; q_full[0] also publishes the item
   uint64_t k_full[2], k_empty[2];
   uint64_t v_full[2], v_empty[2];
   uint64_t s_full[2], p_full[2], o_final[2];  // index: query tile A = 0, B = 1
@@ -191,6 +192,20 @@ __device__ __forceinline__ void load_s64(uint32_t tS, bool diag, int first_col, 
   }
 }
 
+// Units per chunk of the work order: as many (b, kv head, group) units as keep about
+// kLptKVBudget bytes of K and V in flight, and at least kLptChunk. Short groups thus get
+// wide chunks: with few key tiles per item, a chunk of only kLptChunk units would start its
+// heaviest items late in the run and leave a long tail, while their K and V still fit L2.
+#ifndef S2_FWD_LPT_BUDGET_MB
+#define S2_FWD_LPT_BUDGET_MB 16
+#endif
+constexpr long long kLptKVBudget = (long long)S2_FWD_LPT_BUDGET_MB << 20;
+__device__ __forceinline__ int fwd_lpt_chunk(const Params& p) {
+  const long long unit_bytes = 2ll * p.G * kD * 2;   // K and V of one group, bf16
+  const long long c = kLptKVBudget / unit_bytes;
+  return c > kLptChunk ? (int)c : kLptChunk;
+}
+
 // A work item: two consecutive 128-row query tiles (A = qt0, B = qt0 + 1) of one
 // (batch, query head, group). Items are numbered in the chunked longest-first order.
 struct FwdItem {
@@ -201,7 +216,7 @@ struct FwdItem {
 __device__ __forceinline__ FwdItem decode_item(const Params& p, int item) {
   const int T = p.G / kTile, ng = p.N / p.G, R = p.Hq / p.Hkv;
   int inner, bkg;
-  chunked_lpt(item, p.B * p.Hkv * ng, (T / 2) * R, bkg, inner);
+  chunked_lpt(item, p.B * p.Hkv * ng, (T / 2) * R, bkg, inner, fwd_lpt_chunk(p));
   FwdItem it;
   const int pr = T / 2 - 1 - inner / R;
   it.g = bkg % ng;
@@ -230,8 +245,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~static_cast<uintptr_t>(1023));
   __shared__ FwdBarriers bars;
   __shared__ uint32_t tmem_base_sh;
-  __shared__ int abort_flag;
-  // the CTA's k-th work item sits in slot k & 1 (-1: no more work), published with q_full
+  __shared__ AbortState abort_state;
+  // the CTA's k-th work item sits in slot k & 1 (-1: no more work), published with q_full[0]
   __shared__ int item_slot[2];
   // row-max exchange between the two warps that share a row: [parity][tile][half][row]
   __shared__ float xmax[2][2][2][kTile];
@@ -240,12 +255,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   unsigned* const next_item = p.status + kFwdWorkCounter;
 
-  Abort ab{&abort_flag, p.status, p.wait_limit_ns};
+  const Abort ab{smem_addr(&abort_state)};
   if (threadIdx.x == 0) {
-    abort_flag = 0;
-    mbar_init(smem_addr(&bars.q_full), 1);
-    mbar_init(smem_addr(&bars.q_empty), 1);
+    abort_state_init(abort_state, p.status, p.wait_limit_ns, 0);
+    // Q_A is free once its last QK^T has completed (one commit) and every softmax warp has
+    // read the item id (one arrival per warp): the next item's id is only published then, so
+    // no softmax warp can fall two items behind the slot ring or the q_full[0] phases
+    mbar_init(smem_addr(&bars.q_empty[0]), 1 + kSoftmaxWarps);
+    mbar_init(smem_addr(&bars.q_empty[1]), 1);
     for (int s = 0; s < 2; s++) {
+      mbar_init(smem_addr(&bars.q_full[s]), 1);
       mbar_init(smem_addr(&bars.k_full[s]), 1);
       mbar_init(smem_addr(&bars.k_empty[s]), 1);
       mbar_init(smem_addr(&bars.v_full[s]), 1);
@@ -273,28 +292,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       int nk = 0, nv = 0;            // K and V tiles loaded so far (ring positions)
-      int q_last = -1;               // item index (k) of the latest Q load, -1 after the stop
+      int qa_last = -1, qb_last = -1;  // item index (k) of the latest Q_A / Q_B load
       for (int k = 0, ok = 1; ok; k++) {
         int item = (int)atomicAdd(next_item, 1u);
         // stop when the work is done or a CTA of this launch gave up
         if (item >= nitems || *reinterpret_cast<volatile unsigned*>(p.status) != 0u) item = -1;
-        // the query tiles of the previous item are no longer read
-        if (k > 0 && !mbar_wait(smem_addr(&bars.q_empty), (k - 1) & 1, ab)) break;
+        // Q_A of the previous item is no longer read and its id has been taken by all
+        if (k > 0 && !mbar_wait(smem_addr(&bars.q_empty[0]), (k - 1) & 1, ab)) break;
         item_slot[k & 1] = item;
-        const uint32_t qb = smem_addr(&bars.q_full);
+        const uint32_t qa = smem_addr(&bars.q_full[0]), qb = smem_addr(&bars.q_full[1]);
         if (item < 0) {
-          mbar_arrive(qb);  // completes the phase: the consumers read -1 and stop
-          q_last = -1;
+          mbar_arrive(qa);  // completes the phase: the consumers read -1 and stop
+          qa_last = -1;     // (the previous Q_A has been read, so it has landed)
           break;
         }
         const FwdItem it = decode_item(p, item);
-        mbar_arrive_expect_tx(qb, 2 * kTileBytes);
-        for (int t = 0; t < 2; t++) {
-          const int qrow = (it.b * p.Hq + it.h) * p.N + src_row(it.r0 + t * kTile, it.sh, p.G, p.N);
-          tma_load_2d(sQ + t * kTileBytes, &tm_q, qb, 0, qrow);
-          tma_load_2d(sQ + t * kTileBytes + kHalfBytes, &tm_q, qb, 64, qrow);
-        }
-        q_last = k;
+        const int qrow0 = (it.b * p.Hq + it.h) * p.N;
+        mbar_arrive_expect_tx(qa, kTileBytes);
+        tma_load_2d(sQ, &tm_q, qa, 0, qrow0 + src_row(it.r0, it.sh, p.G, p.N));
+        tma_load_2d(sQ + kHalfBytes, &tm_q, qa, 64, qrow0 + src_row(it.r0, it.sh, p.G, p.N));
+        qa_last = k;
         const int krow0 = (it.b * p.Hkv + it.kvh) * p.N;
         for (int j = 0; j < it.nB; j++) {
           const int s = nk & 1;
@@ -306,6 +323,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_2d(sK, &tm_k, smem_addr(&bars.k_full[s]), 0, krow0 + mk);
           tma_load_2d(sK + kHalfBytes, &tm_k, smem_addr(&bars.k_full[s]), 64, krow0 + mk);
           nk++;
+          if (j == 0) {
+            // Q_B after K_0: the next item's first QK^T (tile A) can start before this
+            // item's tile B has finished with the previous Q_B
+            if (k > 0 && !mbar_wait(smem_addr(&bars.q_empty[1]), (k - 1) & 1, ab)) {
+              ok = 0;
+              break;
+            }
+            const int qrow = qrow0 + src_row(it.r0 + kTile, it.sh, p.G, p.N);
+            mbar_arrive_expect_tx(qb, kTileBytes);
+            tma_load_2d(sQ + kTileBytes, &tm_q, qb, 0, qrow);
+            tma_load_2d(sQ + kTileBytes + kHalfBytes, &tm_q, qb, 64, qrow);
+            qb_last = k;
+          }
           if (!mbar_wait(smem_addr(&bars.v_empty[s]), ph ^ 1, ab)) { ok = 0; break; }
           const uint32_t sV = smem_addr(smem + kOffV + s * kTileBytes);
           mbar_arrive_expect_tx(smem_addr(&bars.v_full[s]), kTileBytes);
@@ -316,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // Let the loads in flight land before the CTA can exit: the last load into each ring
-      // stage (the latest phase of its barrier) and a query load not yet consumed. These
+      // stage (the latest phase of its barrier) and query loads not yet consumed. These
       // waits ignore the abort flag (it may be set on this path) but keep their time limit.
       for (int t = nk - 1; t >= 0 && t >= nk - 2; t--)
         mbar_wait_drain(smem_addr(&bars.k_full[t & 1]), (t >> 1) & 1, p.status,
@@ -324,8 +354,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = nv - 1; t >= 0 && t >= nv - 2; t--)
         mbar_wait_drain(smem_addr(&bars.v_full[t & 1]), (t >> 1) & 1, p.status,
                         p.wait_limit_ns);
-      if (q_last >= 0)
-        mbar_wait_drain(smem_addr(&bars.q_full), q_last & 1, p.status, p.wait_limit_ns);
+      if (qa_last >= 0)
+        mbar_wait_drain(smem_addr(&bars.q_full[0]), qa_last & 1, p.status, p.wait_limit_ns);
+      if (qb_last >= 0)
+        mbar_wait_drain(smem_addr(&bars.q_full[1]), qb_last & 1, p.status, p.wait_limit_ns);
     } else if (warp == 1) {
       // ------------------------------------------------------------------ MMA issuer
       // The whole warp runs the issue loop (warp-uniform control flow and descriptors);
@@ -340,21 +372,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dK = smem_desc_sw128(smem_addr(smem + kOffK), 16, 1024);
       const uint64_t dV = smem_desc_sw128(smem_addr(smem + kOffV), kHalfBytes, 1024);
       constexpr uint32_t kTileDesc = kTileBytes >> 4;
+      // Items run back to back in one ping-pong: an item's last PVs (key tile nB - 1) go out
+      // in the next item's first step, after its QK_A(0) and before its QK_B(0), so the
+      // tensor cores work on the next item while tile B's last softmax runs. Key tile j - 1
+      // of step j = 0 is then the previous item's last (ring position kv - 1); a flush step
+      // after the last item issues its final PVs.
       int kv = 0;                        // ring position of the item's key tile 0
-      uint32_t pcnt[2] = {0u, 0u};       // p_full phases consumed per query tile
       bool ok = true;
-      for (int k = 0; ok; k++) {
-        if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.q_full), k & 1, ab))) break;
+      int k = 0;
+      for (;; k++) {
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.q_full[0]), k & 1, ab))) {
+          ok = false;
+          break;
+        }
         const int item = item_slot[k & 1];
-        if (item < 0) break;
-        const FwdItem it = decode_item(p, item);
+        const bool flush = item < 0;     // no more items: only the previous item's PVs
+        if (flush && k == 0) break;
+        const FwdItem it = decode_item(p, flush ? 0 : item);
+        const int nA = flush ? 0 : it.nA, nB = flush ? 1 : it.nB;
         tc_fence_after();
-        for (int j = 0; j <= it.nB; j++) {
+        for (int j = 0; j < nB; j++) {
           const int gj = kv + j, gjj = gj - 1;   // ring positions of key tiles j and j - 1
+          const bool pv = j > 0 || k > 0;        // step j has PVs (of key tile j - 1)
           // V_{j-1} before the first PV, K_j only before the first QK^T: a PV never waits
           // for the key tile that follows it
-          if (j >= 1 && !__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.v_full[gjj & 1]),
-                                                             (gjj >> 1) & 1, ab))) {
+          if (pv && !__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.v_full[gjj & 1]),
+                                                       (gjj >> 1) & 1, ab))) {
             ok = false;
             break;
           }
@@ -367,53 +410,65 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t dQj = opaque64(dQ);
 #pragma unroll
           for (int t = 0; t < 2; t++) {
-            const int nt = t ? it.nB : it.nA;
+            const int nt = t ? nB : nA;
             const uint32_t tS = tmem + t * 128, tO = tmem + 256 + t * 128;
-            if (j >= 1 && j - 1 < nt) {
+            // PV of key tile j - 1: inside the item while j - 1 < nt; at j = 0 the previous
+            // item's last one (tile B always, tile A when not causal: it has nB key tiles)
+            if (j > 0 ? j - 1 < nt : (k > 0 && (t == 1 || !p.causal))) {
+              // p_full phases tile t consumed before: its key tiles in the earlier items
+              // plus j - 1 (tile B has nB per item, kv in all; causal tile A one less each)
+              const int pdone = t || !p.causal ? gjj : gjj - k;
               if (!__all_sync(0xffffffffu,
-                              mbar_wait(smem_addr(&bars.p_full[t]), pcnt[t] & 1, ab))) {
+                              mbar_wait(smem_addr(&bars.p_full[t]), pdone & 1, ab))) {
                 ok = false;
                 break;
               }
-              pcnt[t]++;
               tc_fence_after();
-              const uint32_t acc0 = j > 1;
+              const uint32_t acc0 = j != 1;  // only an item's key tile 0 starts O afresh
 #pragma unroll
               for (int kk = 0; kk < kTile / 16; kk++)  // P of key rows 64h.. at column 64h;
                 mma_ts_elect(tO, tS + (kk >> 2) * 64 + (kk & 3) * 8,  // V k-step = 16 rows
                        dVj + (uint64_t)(kk * (2048 >> 4)), idesc_pv, kk ? 1u : acc0);
-              if (j == nt) mma_commit_elect(smem_addr(&bars.o_final[t]));
+              if (j == 0 || j == nt) mma_commit_elect(smem_addr(&bars.o_final[t]));
             }
             // V_{j-1} is free once the last PV that reads it has been issued (tile B's)
-            if (t == 1 && j >= 1) mma_commit_elect(smem_addr(&bars.v_empty[gjj & 1]));
-            if (j < nt) {
-              if (!k_ready) {
-                if (!__all_sync(0xffffffffu, mbar_wait(smem_addr(&bars.k_full[gj & 1]),
-                                                       (gj >> 1) & 1, ab))) {
+            if (t == 1 && pv) mma_commit_elect(smem_addr(&bars.v_empty[gjj & 1]));
+            if (j < nt && !flush) {
+              // K_j before the step's first QK^T; Q_B before the item's first QK^T of tile B
+              // (K_0 is ready by then: every item has a QK_A(0), so one wait covers both)
+              const bool need_qb = t == 1 && j == 0;
+              if (!k_ready || need_qb) {
+                const uint32_t bar = need_qb ? smem_addr(&bars.q_full[1])
+                                             : smem_addr(&bars.k_full[gj & 1]);
+                const uint32_t par = need_qb ? (uint32_t)(k & 1) : (uint32_t)((gj >> 1) & 1);
+                if (!__all_sync(0xffffffffu, mbar_wait(bar, par, ab))) {
                   ok = false;
                   break;
                 }
                 k_ready = true;
-                tc_fence_after();
               }
+              tc_fence_after();
               const uint64_t dQt = dQj + (uint64_t)(t * kTileDesc);
 #pragma unroll
               for (int kk = 0; kk < kD / 16; kk++) {
-                const uint64_t koff = (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
+                const uint64_t koff =
+                    (uint64_t)(((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4);
                 mma_ss_elect(tS, dQt + koff, dKj + koff, idesc_qk, kk > 0);
               }
               // failure-path self-test: CTA 0 withholds the arrival of score tile B at key
-              // tile 1 of its first item (every item's tile B has at least two key tiles), so
-              // that tile's softmax warps and then this thread wait in vain until the limit
+              // tile 1 of its first item (every item's tile B has at least two key tiles),
+              // so that tile's softmax warps and then this thread wait in vain until the limit
               if (!(p.inject == kInjectFwd && blockIdx.x == 0 && k == 0 && t == 1 && j == 1))
                 mma_commit_elect(smem_addr(&bars.s_full[t]));
+              // Q_t is free after the last QK^T that reads it
+              if (j == nt - 1) mma_commit_elect(smem_addr(&bars.q_empty[t]));
             }
           }
           if (!ok) break;
-          if (j == it.nB - 1) mma_commit_elect(smem_addr(&bars.q_empty));  // last QK^T of the item
-          if (j < it.nB) mma_commit_elect(smem_addr(&bars.k_empty[gj & 1]));
+          if (!flush) mma_commit_elect(smem_addr(&bars.k_empty[gj & 1]));
         }
-        kv += it.nB;
+        if (!ok || flush) break;
+        kv += nB;
       }
       // every MMA issued above has completed before TMEM is released
       mma_commit_elect(smem_addr(&bars.drain));
@@ -439,10 +494,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Both warps of a row pass the same named barriers in the same order on every path, and
     // decide together whether to go on (a wait that gave up in one of them stops both).
     for (int k = 0;; k++) {
-      bool got = mbar_wait<1>(smem_addr(&bars.q_full), k & 1, ab);
+      bool got = mbar_wait<1>(smem_addr(&bars.q_full[0]), k & 1, ab);
       __syncwarp();
       got = __all_sync(0xffffffffu, got);
       const int item = got ? item_slot[k & 1] : -1;
+      __syncwarp();
+      if (item >= 0 && lane == 0) mbar_arrive(smem_addr(&bars.q_empty[0]));  // id taken
       if (!named_bar_and(bar_id, 64, item >= 0)) break;
       const FwdItem it = decode_item(p, item);
       const int qt = it.qt0 + t;
