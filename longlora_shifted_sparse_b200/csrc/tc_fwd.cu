@@ -201,9 +201,9 @@ __device__ __forceinline__ void load_s64(uint32_t tS, bool diag, int first_col, 
 #endif
 constexpr long long kLptKVBudget = (long long)S2_FWD_LPT_BUDGET_MB << 20;
 __device__ __forceinline__ int fwd_lpt_chunk(const Params& p) {
-  const long long unit_bytes = 2ll * p.G * kD * 2;   // K and V of one group, bf16
-  const long long c = kLptKVBudget / unit_bytes;
-  return c > kLptChunk ? (int)c : kLptChunk;
+  // kLptKVBudget / (K and V bytes of one group = 2 * G * d * 2), in 32-bit arithmetic
+  const int c = (int)(kLptKVBudget / (4 * kD)) / p.G;
+  return c > kLptChunk ? c : kLptChunk;
 }
 
 // A work item: two consecutive 128-row query tiles (A = qt0, B = qt0 + 1) of one
@@ -582,27 +582,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float ltot = xsum[t][row];
       if (!ok) break;
       tc_fence_after();
-      const int mrow = src_row(it.r0 + t * kTile + row, it.sh, p.G, p.N);
-      __nv_bfloat16* orow =
-          static_cast<__nv_bfloat16*>(p.o) + ((size_t)(it.b * p.N + mrow) * p.Hq + it.h) * kD + c0;
       const float inv_l = 1.f / ltot;
+      uint32_t w[32];  // the row's 64 outputs, bf16 pairs; 16-byte chunk c is w[4c .. 4c + 3]
 #pragma unroll
       for (int ch = 0; ch < 2; ch++) {
         uint32_t o[32];
         tmem_ld32(tO + ch * 32, o);
         tmem_wait_ld();
-        uint4 pk[4];
-        uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
         for (int c2 = 0; c2 < 16; c2++)
-          pw[c2] = pack_bf16x2(__uint_as_float(o[2 * c2]) * inv_l,
-                               __uint_as_float(o[2 * c2 + 1]) * inv_l);
-        uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
-#pragma unroll
-        for (int c4 = 0; c4 < 4; c4++) dst[c4] = pk[c4];
+          w[ch * 16 + c2] = pack_bf16x2(__uint_as_float(o[2 * c2]) * inv_l,
+                                        __uint_as_float(o[2 * c2 + 1]) * inv_l);
       }
+      // 8 x 8 transpose of the 16-byte chunks inside each group of eight lanes (three
+      // butterfly stages of shuffles): lane 8g + i then holds chunk i of the group's eight
+      // rows, so that each store below writes four whole 128-byte row segments where a
+      // store of the row a lane holds would write 16 bytes to each of 32 rows
+      const int l8 = lane & 7;
+#pragma unroll
+      for (int bit = 4; bit >= 1; bit >>= 1) {
+        const bool up = (l8 & bit) != 0;
+#pragma unroll
+        for (int c = 0; c < 8; c++) {
+          if (c & bit) continue;
+#pragma unroll
+          for (int e = 0; e < 4; e++) {
+            const uint32_t mine = w[4 * c + e], other = w[4 * (c ^ bit) + e];
+            const uint32_t got = __shfl_xor_sync(0xffffffffu, up ? mine : other, bit);
+            if (up)
+              w[4 * c + e] = got;
+            else
+              w[4 * (c ^ bit) + e] = got;
+          }
+        }
+      }
+      // the tile's rows are consecutive tokens from m0 (a 128-row tile never straddles the
+      // wrap of the roll, G / 2 being a multiple of 128)
+      const int m0 = src_row(it.r0 + t * kTile, it.sh, p.G, p.N);
+      const size_t rstride = (size_t)p.Hq * kD;
+      __nv_bfloat16* obase = static_cast<__nv_bfloat16*>(p.o) +
+                             ((size_t)(it.b * p.N + m0 + quarter * 32 + (lane & ~7)) * p.Hq +
+                              it.h) * kD + c0 + l8 * 8;
+#pragma unroll
+      for (int c = 0; c < 8; c++)
+        *reinterpret_cast<uint4*>(obase + c * rstride) =
+            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
       if (half == 0)
-        p.lse[((size_t)it.b * p.Hq + it.h) * p.N + mrow] =
+        p.lse[((size_t)it.b * p.Hq + it.h) * p.N + m0 + row] =
             (m + __log2f(ltot)) * 0.69314718055994531f;
     }
   }
