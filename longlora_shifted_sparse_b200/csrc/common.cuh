@@ -124,4 +124,30 @@ __device__ inline float warp_sum(float x) {
   return x;
 }
 
+// 8 x 8 transpose of 16-byte chunks inside each group of eight lanes of a warp. Lane 8g + i
+// passes in the eight chunks of its own row (chunk c = w[4c .. 4c + 3]) and gets back chunk i
+// of the group's eight rows (w[4c ..] = chunk i of row 8g + c): a store of chunk c then
+// writes one whole 128-byte row segment per eight lanes. Three butterfly stages of shuffles;
+// every index is static, so the array stays in registers.
+__device__ __forceinline__ void transpose_chunks8(uint32_t (&w)[32], int lane) {
+  const int l8 = lane & 7;
+#pragma unroll
+  for (int bit = 4; bit >= 1; bit >>= 1) {
+    const bool up = (l8 & bit) != 0;
+#pragma unroll
+    for (int c = 0; c < 8; c++) {
+      if (c & bit) continue;
+#pragma unroll
+      for (int e = 0; e < 4; e++) {
+        const uint32_t mine = w[4 * c + e], other = w[4 * (c ^ bit) + e];
+        const uint32_t got = __shfl_xor_sync(0xffffffffu, up ? mine : other, bit);
+        if (up)
+          w[4 * c + e] = got;
+        else
+          w[4 * (c ^ bit) + e] = got;
+      }
+    }
+  }
+}
+
 }  // namespace s2

@@ -7,8 +7,9 @@
 // roll of the shifted heads is never materialised, the attention kernels fold it into
 // their row coordinates.
 //
-// Two kernels. The first computes the (cos, sin) table once per call, [N][d/2], each entry
-// from an exact fp64 angle (sincos in fp64, rounded to fp32); the backward's inverse
+// Two kernels. The first computes the (cos, sin) table once per call, [N][d/2], in fp64
+// (sincos of the exact angle at the start of each run of tokens, the angle-addition
+// formulas along it), rounded to fp32; the backward's inverse
 // rotation reads the same table from the workspace. The second streams q and k in 16-byte
 // vectors, one CTA per token, and reads the token's table row (shared by all its heads,
 // an L1/L2 hit) next to each vector: no CTA waits on fp64 arithmetic.
@@ -36,26 +37,35 @@ __device__ inline uint4 rotate_vec(uint4 raw, const float2* __restrict__ cs_row)
 // (cos, sin) of (m / s) * base^(-2i/d) for every token m and pair i. The first kernel of
 // every forward and of every backward that rotates: it also resets the status word and the
 // persistent kernels' work counters, and records which arguments the rotation belongs to.
+// A thread takes one pair i and a run of kTableRun consecutive tokens: the run's first angle
+// in fp64 (pow, sincos), each next token by turning (cos, sin) through the step theta_i / s
+// with the angle-addition formulas, in fp64. Over a run that drifts by about 1e-15, far
+// below the fp32 rounding of the entries, at a fraction of a pow and a sincos per entry.
+constexpr int kTableRun = 16;
 __global__ void __launch_bounds__(256) rope_table_kernel(Params p) {
   const int half = p.d / 2;
-  const long total = (long)p.N * half;
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     for (int c = 0; c <= kNumWorkCounters; c++) p.status[c] = 0u;
     p.status[kFingerprintWord] = (unsigned)p.fingerprint;
     p.status[kFingerprintWord + 1] = (unsigned)(p.fingerprint >> 32);
   }
-  // the block size, hence the grid stride, is a multiple of d/2 (the launcher sizes it so),
-  // so a thread keeps one pair index i and computes its frequency once
+  const long runs = (long)((p.N + kTableRun - 1) / kTableRun) * half;
   const long stride = (long)gridDim.x * blockDim.x;
-  const long e0 = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  const int i = (int)(e0 % half);
-  const double theta = pow((double)p.rope_base, -2.0 * (double)i / (double)p.d);
-  for (long e = e0; e < total; e += stride) {
-    const int n = (int)(e / half);
-    const double phi = ((double)n / (double)p.pi_scale) * theta;
-    double sn, c;
-    sincos(phi, &sn, &c);
-    p.cs[e] = make_float2((float)c, (float)sn);
+  for (long e = (long)blockIdx.x * blockDim.x + threadIdx.x; e < runs; e += stride) {
+    const int i = (int)(e % half);                  // consecutive threads: consecutive pairs
+    const int n0 = (int)(e / half) * kTableRun;
+    const int n1 = min(n0 + kTableRun, p.N);
+    const double theta = pow((double)p.rope_base, -2.0 * (double)i / (double)p.d);
+    double ss, cs_step, sn, c;
+    sincos(theta / (double)p.pi_scale, &ss, &cs_step);
+    sincos(((double)n0 / (double)p.pi_scale) * theta, &sn, &c);
+    float2* dst = p.cs + (size_t)n0 * half + i;
+    for (int n = n0; n < n1; n++, dst += half) {
+      *dst = make_float2((float)c, (float)sn);
+      const double c_next = fma(c, cs_step, -sn * ss);
+      sn = fma(sn, cs_step, c * ss);
+      c = c_next;
+    }
   }
 }
 
@@ -113,13 +123,10 @@ __global__ void __launch_bounds__(256) rope_pi_kernel(Params p) {
 }
 
 cudaError_t launch_rope_table(const Params& p, cudaStream_t st) {
-  // a multiple of d/2 threads per block, so the grid stride is one too
-  const int half = p.d / 2;
-  const int threads = (256 / half) * half;
-  const long total = (long)p.N * half;
-  long blocks = (total + threads - 1) / threads;
+  const long runs = (long)((p.N + kTableRun - 1) / kTableRun) * (p.d / 2);
+  long blocks = (runs + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  rope_table_kernel<<<dim3((unsigned)blocks), dim3(threads), 0, st>>>(p);
+  rope_table_kernel<<<dim3((unsigned)blocks), dim3(256), 0, st>>>(p);
   return cudaGetLastError();
 }
 

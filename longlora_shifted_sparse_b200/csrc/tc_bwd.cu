@@ -155,21 +155,15 @@ __device__ __forceinline__ uint32_t packed_col(uint32_t region, int kk) {
 
 // Rotates a chunk of 32 consecutive fp32 columns (16 channel pairs starting at pair p0)
 // back by R(phi)^T, scales it, and packs it to bf16.
+// (32 packed bf16 pairs into w[off .. off + 15])
 __device__ __forceinline__ void unrotate_pack(const uint32_t (&x)[32], const float2* cs_row,
-                                              int p0, float scale, uint4 (&out)[4]) {
-  uint32_t* w = reinterpret_cast<uint32_t*>(out);
+                                              int p0, float scale, uint32_t (&w)[32], int off) {
 #pragma unroll
   for (int t = 0; t < 16; t++) {
     const float2 c = cs_row[p0 + t];
     const float x0 = __uint_as_float(x[2 * t]) * scale, x1 = __uint_as_float(x[2 * t + 1]) * scale;
-    w[t] = pack_bf16x2(fmaf(x0, c.x, x1 * c.y), fmaf(-x0, c.y, x1 * c.x));
+    w[off + t] = pack_bf16x2(fmaf(x0, c.x, x1 * c.y), fmaf(-x0, c.y, x1 * c.x));
   }
-}
-
-__device__ __forceinline__ void store_row64(__nv_bfloat16* dst, const uint4 (&a)[4]) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int t = 0; t < 4; t++) d4[t] = a[t];
 }
 
 // ================================================================================ dK / dV
@@ -1008,18 +1002,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      __nv_bfloat16* dq =
-          static_cast<__nv_bfloat16*>(p.dq) + ((size_t)(it.b * p.N + m) * p.Hq + it.h) * kD + c0;
       const float2* cs_row = p.cs + (size_t)m * (kD / 2);
+      uint32_t w[32];  // the row's 64 dQ values, bf16 pairs; 16-byte chunk c is w[4c .. 4c + 3]
 #pragma unroll
       for (int ch = 0; ch < 2; ch++) {
         uint32_t x[32];
-        uint4 o[4];
         tmem_ld32(tmem + lane_off + colDQ + c0 + ch * 32, x);
         tmem_wait_ld();
-        unrotate_pack(x, cs_row, (c0 + ch * 32) / 2, p.scale, o);
-        store_row64(dq + ch * 32, o);
+        unrotate_pack(x, cs_row, (c0 + ch * 32) / 2, p.scale, w, ch * 16);
       }
+      // stores of whole 128-byte row segments, eight lanes per row (the tile's rows are
+      // consecutive tokens from m - row: a 128-row tile never straddles the roll's wrap)
+      transpose_chunks8(w, lane);
+      __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(p.dq) +
+                          ((size_t)(it.b * p.N + m - row + (row & ~7)) * p.Hq + it.h) * kD +
+                          c0 + (lane & 7) * 8;
+#pragma unroll
+      for (int c = 0; c < 8; c++)
+        *reinterpret_cast<uint4*>(dq + (size_t)c * p.Hq * kD) =
+            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
       // the next item's first dQ MMA overwrites the accumulator only after this item's
       // dS of its first key tile, which these warps publish after the loads above
     }

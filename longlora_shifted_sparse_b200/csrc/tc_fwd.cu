@@ -594,35 +594,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           w[ch * 16 + c2] = pack_bf16x2(__uint_as_float(o[2 * c2]) * inv_l,
                                         __uint_as_float(o[2 * c2 + 1]) * inv_l);
       }
-      // 8 x 8 transpose of the 16-byte chunks inside each group of eight lanes (three
-      // butterfly stages of shuffles): lane 8g + i then holds chunk i of the group's eight
-      // rows, so that each store below writes four whole 128-byte row segments where a
-      // store of the row a lane holds would write 16 bytes to each of 32 rows
-      const int l8 = lane & 7;
-#pragma unroll
-      for (int bit = 4; bit >= 1; bit >>= 1) {
-        const bool up = (l8 & bit) != 0;
-#pragma unroll
-        for (int c = 0; c < 8; c++) {
-          if (c & bit) continue;
-#pragma unroll
-          for (int e = 0; e < 4; e++) {
-            const uint32_t mine = w[4 * c + e], other = w[4 * (c ^ bit) + e];
-            const uint32_t got = __shfl_xor_sync(0xffffffffu, up ? mine : other, bit);
-            if (up)
-              w[4 * c + e] = got;
-            else
-              w[4 * (c ^ bit) + e] = got;
-          }
-        }
-      }
+      // each store below then writes four whole 128-byte row segments, where a store of
+      // the row a lane holds would write 16 bytes to each of 32 rows
+      transpose_chunks8(w, lane);
       // the tile's rows are consecutive tokens from m0 (a 128-row tile never straddles the
       // wrap of the roll, G / 2 being a multiple of 128)
       const int m0 = src_row(it.r0 + t * kTile, it.sh, p.G, p.N);
       const size_t rstride = (size_t)p.Hq * kD;
       __nv_bfloat16* obase = static_cast<__nv_bfloat16*>(p.o) +
                              ((size_t)(it.b * p.N + m0 + quarter * 32 + (lane & ~7)) * p.Hq +
-                              it.h) * kD + c0 + l8 * 8;
+                              it.h) * kD + c0 + (lane & 7) * 8;
 #pragma unroll
       for (int c = 0; c < 8; c++)
         *reinterpret_cast<uint4*>(obase + c * rstride) =
