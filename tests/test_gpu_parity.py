@@ -70,6 +70,9 @@ SMALL = [
     # several work items per CTA in the persistent kernels (forward 256 items, dQ 512, on
     # 148 CTAs), compared in full: the item-to-item hand-over of their rings
     ("bf16_multi_item_gqa", 1, 8192, 8, 4, 128, 1024, 2.0, "bf16", True),
+    # the same with one query head per kv head (dQ 256 items; the last key tile of every
+    # group has a single (query head, query tile) pair in the dK/dV pass)
+    ("bf16_multi_item_mha", 1, 8192, 4, 4, 128, 1024, 2.0, "bf16", True),
     # head dims of 3, 5, 6 and 7 elements per lane on the CUDA-core kernels
     ("bf16_d96_gqa", 1, 384, 4, 2, 96, 128, 2.0, "bf16", True),
     ("f32_d160_noncausal", 1, 256, 2, 2, 160, 64, 1.5, "f32", False),
