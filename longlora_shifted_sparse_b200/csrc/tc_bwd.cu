@@ -99,16 +99,16 @@ __device__ __forceinline__ uint64_t opaque64(uint64_t v) {
   return r;
 }
 
-// Column c of a thread's 64 probabilities in the dQ pass takes its exponential from the
-// FMA-pipe polynomial (fastmath.cuh) when bit c of the mask is set, else from the MUFU unit;
+// The dQ pass: bit t set sends the exponentials of column pair t (columns 2t, 2t+1 of a
+// math warp's 64) to the packed FMA-pipe polynomial (fastmath.cuh), else to the MUFU unit;
 // off the diagonal tiles only (no -inf scores there; the polynomial clamps its argument at
-// -125). On a B200, 32k workload, moving 1/8, 1/4 or 3/8 of the exponentials to the
-// polynomial left the pass as fast or slowed it (2.96 -> 2.94 / 3.01 / 3.17 ms), so the
-// mask defaults to 0 (all exponentials on the MUFU).
+// -125). On a B200, 32k workload, 1/8, 1/4 and 3/8 of them there gave 2.65-2.68 /
+// 2.67-2.70 / 2.64-2.68 ms against 2.63-2.66 ms with none (within run-to-run noise): the
+// pass is not bound by the MUFU, so the default is none.
 #ifndef S2_DQ_POLY_MASK
-#define S2_DQ_POLY_MASK 0x0ull
+#define S2_DQ_POLY_MASK 0x0u
 #endif
-constexpr unsigned long long kDqPolyMask = S2_DQ_POLY_MASK;
+constexpr unsigned kDqPolyMask = S2_DQ_POLY_MASK;
 // The dK/dV pass: bit t set sends the exponentials of column pair t (columns 2t, 2t+1 of a
 // math warp's 64) to the packed FMA-pipe polynomial, off the diagonal tiles. On a B200, 32k
 // workload, 1/8, 1/4 and 1/2 of them there gave 3.52 / 3.62 / 3.68 ms against 3.59-3.68 ms
@@ -118,10 +118,6 @@ constexpr unsigned long long kDqPolyMask = S2_DQ_POLY_MASK;
 #define S2_DKDV_POLY_MASK 0x0u
 #endif
 constexpr unsigned kDkdvPolyMask = S2_DKDV_POLY_MASK;
-template <unsigned long long kMask>
-__device__ __forceinline__ float exp2_mixed(float x, int c) {
-  return ((kMask >> c) & 1ull) ? exp2_poly(x) : fast_exp2(x);
-}
 
 // Causal mask of a diagonal tile, applied to a thread's 64 raw scores (columns c = 0..63 of
 // its half) before the exponential: the score becomes -inf, so its probability is exactly 0.
@@ -961,10 +957,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
 #pragma unroll
             for (int c = 0; c < 64; c += 2) {
-              float a0, a1;
-              f2unpack(ffma2(score_pair(x0, x1, c), sl2x2, nlse2x2), a0, a1);
-              pr[c] = exp2_mixed<kDqPolyMask>(a0, c);
-              pr[c + 1] = exp2_mixed<kDqPolyMask>(a1, c + 1);
+              const uint64_t a = ffma2(score_pair(x0, x1, c), sl2x2, nlse2x2);
+              if ((kDqPolyMask >> (c >> 1)) & 1u) {
+                f2unpack(exp2_poly2(a), pr[c], pr[c + 1]);
+              } else {
+                float a0, a1;
+                f2unpack(a, a0, a1);
+                pr[c] = fast_exp2(a0);
+                pr[c + 1] = fast_exp2(a1);
+              }
             }
           }
           pin_regs(pr);
