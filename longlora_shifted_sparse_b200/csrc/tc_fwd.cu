@@ -10,12 +10,14 @@
 // above the diagonal are skipped, the diagonal tile is masked on group-local positions).
 //
 // Roles (640 threads, five warpgroups):
-//   warp 0       TMA producer: per work item Q_A and Q_B, then K_j, V_j into two 2-stage
-//                rings (each K/V tile serves both query tiles; the rings run on across
-//                the items of a CTA).
-//   warp 1       MMA issuer (one thread) and TMEM owner. Order per key tile j:
-//                PV_A(j-1), QK_A(j), PV_B(j-1), QK_B(j): while the tensor cores work on
-//                one tile, the other tile's softmax runs (ping-pong).
+//   warp 0       TMA producer: per work item Q_A, K_0, Q_B, then V_0, K_j, V_j into two
+//                2-stage rings (each K/V tile serves both query tiles; the rings run on
+//                across the items of a CTA). Q_A and Q_B have a buffer each.
+//   warp 1       MMA issuer (the warp runs the loop, one elected lane issues) and TMEM
+//                owner. Order per key tile j: PV_A(j-1), QK_A(j), PV_B(j-1), QK_B(j): while
+//                the tensor cores work on one tile, the other tile's softmax runs
+//                (ping-pong). The ping-pong runs on across a CTA's items: an item's last
+//                PVs go out in the next item's first step, after its QK_A(0).
 //   warps 2, 3   idle (they complete warpgroup 0, whose registers go to the softmax).
 //   warps 4..11  softmax of tile A; warps 12..19 softmax of tile B. A query row (= TMEM
 //                lane) is shared by two warps, one per 64-column half of S: each loads its
@@ -29,14 +31,16 @@
 //                same max. When S_t(j) has landed, PV_t(j-1) has completed (commit order),
 //                so the rescale needs no extra wait. Epilogue: each half stores its 64
 //                columns of O / l (l = sum of both partial sums) as bf16 at the token's
-//                original row; LSE = ln 2 * (m + log2 l).
+//                original row, whole 128-byte row segments per store after a shuffle
+//                transpose within groups of eight lanes; LSE = ln 2 * (m + log2 l).
 // TMEM: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
 // Persistent CTAs (one per SM) take work items from a counter in the workspace. Items are
-// numbered a few (b, kv head, group) units at a time, the heaviest tile pairs of those units
-// first, so the items in flight reuse K and V from L2 and the last items are light. Between
-// two items of a CTA the producer and the issuer run ahead: the next item's Q tiles load
-// once the last QK^T of the current one has completed, and its first QK^T MMAs run while
-// the softmax warps write the current item's output.
+// numbered a chunk of (b, kv head, group) units at a time, the heaviest tile pairs of those
+// units first, so the items in flight reuse K and V from L2 and the last items are light.
+// Between two items of a CTA the producer and the issuer run ahead: the next item's Q_A
+// loads once the last QK^T of the current tile A has completed (and every softmax warp has
+// taken the current item's id), its Q_B once tile B's has, and its first QK^T MMAs run
+// while the softmax warps finish the current item.
 // Every wait is bounded; on expiry the CTA records it in the status word and drains.
 #include "common.cuh"
 #include "fastmath.cuh"
