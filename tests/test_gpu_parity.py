@@ -73,6 +73,8 @@ SMALL = [
     # the same with one query head per kv head (dQ 256 items; the last key tile of every
     # group has a single (query head, query tile) pair in the dK/dV pass)
     ("bf16_multi_item_mha", 1, 8192, 4, 4, 128, 1024, 2.0, "bf16", True),
+    # and across batch entries: the unit number carries b (forward 256 items, dQ 512)
+    ("bf16_multi_item_b2", 2, 4096, 8, 4, 128, 1024, 4.0, "bf16", True),
     # head dims of 3, 5, 6 and 7 elements per lane on the CUDA-core kernels
     ("bf16_d96_gqa", 1, 384, 4, 2, 96, 128, 2.0, "bf16", True),
     ("f32_d160_noncausal", 1, 256, 2, 2, 160, 64, 1.5, "f32", False),
