@@ -149,19 +149,6 @@ __device__ __forceinline__ uint32_t packed_col(uint32_t region, int kk) {
   return region + (kk >> 2) * 64 + ((kk >> 1) & 1) * 16 + (kk & 1) * 8;
 }
 
-// Rotates a chunk of 32 consecutive fp32 columns (16 channel pairs starting at pair p0)
-// back by R(phi)^T, scales it, and packs it to bf16.
-// (32 packed bf16 pairs into w[off .. off + 15])
-__device__ __forceinline__ void unrotate_pack(const uint32_t (&x)[32], const float2* cs_row,
-                                              int p0, float scale, uint32_t (&w)[32], int off) {
-#pragma unroll
-  for (int t = 0; t < 16; t++) {
-    const float2 c = cs_row[p0 + t];
-    const float x0 = __uint_as_float(x[2 * t]) * scale, x1 = __uint_as_float(x[2 * t + 1]) * scale;
-    w[off + t] = pack_bf16x2(fmaf(x0, c.x, x1 * c.y), fmaf(-x0, c.y, x1 * c.x));
-  }
-}
-
 // ================================================================================ dK / dV
 
 // smem: K | V | Q stages 0..2 (each a 32 KB tile followed by its 4 KB row-term block) | dO |
@@ -1003,25 +990,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const float2* cs_row = p.cs + (size_t)m * (kD / 2);
-      uint32_t w[32];  // the row's 64 dQ values, bf16 pairs; 16-byte chunk c is w[4c .. 4c + 3]
+      // The fp32 accumulator is transposed first (8 x 8 chunks of four values within each
+      // group of eight lanes, per 32 columns): lane 8g + i then holds columns 4i .. 4i + 3
+      // of each 32-column block for the group's eight rows, so that its (cos, sin) entries
+      // (two pairs per row and block) are read 128 contiguous bytes per eight lanes and its
+      // stores are 64 contiguous bytes per eight lanes. The tile's rows are consecutive
+      // tokens from m - row (a 128-row tile never straddles the roll's wrap).
+      const int l8 = lane & 7;
+      const size_t tok0 = (size_t)(m - row + (row & ~7));  // token of the group's first row
+      uint32_t w[32];  // bf16 pairs: block ch, row c of the group -> w[16ch + 2c], w[16ch + 2c + 1]
 #pragma unroll
       for (int ch = 0; ch < 2; ch++) {
         uint32_t x[32];
         tmem_ld32(tmem + lane_off + colDQ + c0 + ch * 32, x);
         tmem_wait_ld();
-        unrotate_pack(x, cs_row, (c0 + ch * 32) / 2, p.scale, w, ch * 16);
+        transpose_chunks8(x, lane);
+        const float4* cs4 =
+            reinterpret_cast<const float4*>(p.cs + tok0 * (kD / 2) + (c0 + 32 * ch) / 2 + 2 * l8);
+#pragma unroll
+        for (int c = 0; c < 8; c++) {
+          const float4 cs = cs4[c * (kD / 4)];  // pairs 2 l8, 2 l8 + 1 of row c of the group
+#pragma unroll
+          for (int e = 0; e < 2; e++) {
+            const float cc = e ? cs.z : cs.x, sn = e ? cs.w : cs.y;
+            const float x0 = __uint_as_float(x[4 * c + 2 * e]) * p.scale;
+            const float x1 = __uint_as_float(x[4 * c + 2 * e + 1]) * p.scale;
+            w[16 * ch + 2 * c + e] = pack_bf16x2(fmaf(x0, cc, x1 * sn), fmaf(-x0, sn, x1 * cc));
+          }
+        }
       }
-      // stores of whole 128-byte row segments, eight lanes per row (the tile's rows are
-      // consecutive tokens from m - row: a 128-row tile never straddles the roll's wrap)
-      transpose_chunks8(w, lane);
       __nv_bfloat16* dq = static_cast<__nv_bfloat16*>(p.dq) +
-                          ((size_t)(it.b * p.N + m - row + (row & ~7)) * p.Hq + it.h) * kD +
-                          c0 + (lane & 7) * 8;
+                          ((size_t)it.b * p.N + tok0) * p.Hq * kD + (size_t)it.h * kD + c0 + 4 * l8;
 #pragma unroll
       for (int c = 0; c < 8; c++)
-        *reinterpret_cast<uint4*>(dq + (size_t)c * p.Hq * kD) =
-            make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+#pragma unroll
+        for (int ch = 0; ch < 2; ch++)
+          *reinterpret_cast<uint2*>(dq + (size_t)c * p.Hq * kD + 32 * ch) =
+              make_uint2(w[16 * ch + 2 * c], w[16 * ch + 2 * c + 1]);
       // the next item's first dQ MMA overwrites the accumulator only after this item's
       // dS of its first key tile, which these warps publish after the loads above
     }
