@@ -126,9 +126,10 @@ __device__ inline float warp_sum(float x) {
 
 // 8 x 8 transpose of 16-byte chunks inside each group of eight lanes of a warp. Lane 8g + i
 // passes in the eight chunks of its own row (chunk c = w[4c .. 4c + 3]) and gets back chunk i
-// of the group's eight rows (w[4c ..] = chunk i of row 8g + c): a store of chunk c then
-// writes one whole 128-byte row segment per eight lanes. Three butterfly stages of shuffles;
-// every index is static, so the array stays in registers.
+// of the group's eight rows (w[4c ..] = chunk i of row 8g + c): the eight lanes of a group
+// then hold one 128-byte segment of a row together, so that a store of chunk c, or a read
+// of data laid out like the row, touches whole segments. Three butterfly stages of
+// shuffles; every index is static, so the array stays in registers.
 __device__ __forceinline__ void transpose_chunks8(uint32_t (&w)[32], int lane) {
   const int l8 = lane & 7;
 #pragma unroll
